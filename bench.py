@@ -1,0 +1,328 @@
+#!/usr/bin/env python
+"""Benchmark of exact blockwise (ring) attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--sched auto|persistent|fused|unfused] [--order ring|tokenring]
+                    [--impl ours|reference]
+
+One step = one ra_ring_attention call over the workload (partition of Q, K, V
+into block order, block attention over every (query block, KV block) pair in
+schedule order with the merge rule, output in original order).  The metric is
+causal-adjusted attention throughput, 4 * B * Hq * D * P FLOPs per step with P
+the number of visible (query, key) pairs.  Inputs are resident in HBM when the
+timed region starts; L2 is flushed (a 256 MiB write) between timed steps,
+outside the timed events.  Each step is timed on the device with CUDA events;
+the attention kernel inside the call is timed with a second pair of events
+recorded by the library around its launch.  With N GPUs each rank runs the
+same workload on its own GPU (replicas, weak scaling; the method needs no
+exchange on one node here) and the slowest rank's time counts.
+
+--impl reference times the CPU fp64 oracle on the host cores instead (a
+bounded sample of the same workload).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from seeded_inputs import WORKLOADS, workload_inputs  # noqa: E402
+
+DEFAULT_WORKLOAD = "zigzag4k"
+DEFAULT_STEPS = {"tiny": 2000, "zigzag4k": 2000, "gqa24k": 400, "long1m": 3}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=None)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    p.add_argument("--sched", default="auto", choices=["auto", "persistent", "fused", "unfused"])
+    p.add_argument("--order", default="ring", choices=["ring", "tokenring"])
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    a = p.parse_args()
+    if a.steps is None:
+        a.steps = DEFAULT_STEPS[a.workload]
+    if a.warmup < 3:
+        p.error("--warmup must be >= 3")
+    return a
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def workload_config(w, args, l2):
+    return {"workload": w.name, "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "n_blocks": w.n_blocks,
+            "causal": w.causal, "partition": w.partition, "in_dtype": w.in_dtype, "out_dtype": w.out_dtype,
+            "sched": args.sched, "order": args.order, "l2": l2, "parallelism": f"replicas{args.gpus}"}
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def oracle_sample(w, budget_s: float = 15.0):
+    """Times the oracle's blockwise path (the method in fp64) on a bounded
+    sample: the first h query heads (with their KV heads) of batch 0."""
+    import numpy as np  # noqa: F401
+    from oracle import blockwise as K
+    from seeded_inputs import attention_inputs
+    q, k, v = workload_inputs(w) if w.S <= 24000 else attention_inputs(1, 32768, w.Hq, w.Hkv, w.D, w.in_dtype, 0)
+    S = q.shape[1]
+    n = w.n_blocks
+    g = w.gqa_groups
+    flops_head = 4.0 * w.D * (S * (S + 1) // 2 if w.causal else S * S)
+    t0 = time.perf_counter()
+    K.blockwise_attention(q[:1, :, :1], k[:1, :, :1], v[:1, :, :1], n, w.causal, w.partition, 1)
+    t1 = time.perf_counter() - t0
+    heads = max(1, min(w.Hq, int(budget_s / max(t1, 1e-3)) - 1))
+    t0 = time.perf_counter()
+    nkv = (heads + g - 1) // g
+    K.blockwise_attention(q[:1, :, :heads], k[:1, :, :nkv], v[:1, :, :nkv], n, w.causal, w.partition, g)
+    dt = time.perf_counter() - t0
+    cores = len(os.sched_getaffinity(0))
+    sample = (f"oracle blockwise path (fp64 NumPy) on batch 0, query heads 0..{heads - 1} of {w.Hq}, "
+              f"S={S}" + ("" if S == w.S else f" (sequence shortened from {w.S})"))
+    return flops_head * heads / dt / 1e12, cores, sample, dt
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    per_step = []
+    budget = max(1.0, 120.0 / max(args.steps + args.warmup, 1))
+    for _ in range(args.warmup):  # untimed
+        oracle_sample(w, budget_s=0.0)
+    for _ in range(args.steps):
+        v, cores, sample, dt = oracle_sample(w, budget_s=budget)
+        per_step.append(v)
+    value = statistics.median(per_step)
+    line = {"impl": "reference", "metric": "causal-adj attention TFLOP/s (% of dense bf16 peak)", "value": value,
+            "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded randn, bf16-rounded)", "config": workload_config(w, args, "n/a (CPU)"),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ----------------------------------------------------------------- clocks
+
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(gpu_id), "-lms", "100"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def launches_per_step(w, sched):
+    copy_inputs = w.partition == "zigzag" or w.in_dtype == "f32"
+    k = 3 if copy_inputs else 0
+    if sched in ("auto", "persistent"):
+        return k + 1
+    if sched == "fused":
+        return k + w.n_blocks + 2
+    return k + w.n_blocks + (w.n_blocks - 1) + 2
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    import blockwise_exact_attention_block_b200 as ra
+
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    q_h, k_h, v_h = workload_inputs(w)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    odt = torch.bfloat16 if w.out_dtype == "bf16" else torch.float32
+    out = torch.empty((w.B, w.S, w.Hq, w.D), dtype=odt, device=dev)
+    lse = torch.empty((w.B, w.S, w.Hq), dtype=torch.float32, device=dev)
+    need = ra.ra_ring_attention_workspace(w.B, w.S, w.Hq, w.D, w.n_blocks, w.gqa_groups, w.partition, q.dtype,
+                                          args.order, args.sched)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    stream = torch.cuda.current_stream(dev)
+
+    def step(events=None):
+        ra.ra_ring_attention(q, k, v, w.n_blocks, w.causal, w.partition, w.gqa_groups, out=out, lse=lse,
+                             workspace=ws, order=args.order, sched=args.sched, attn_events=events)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if ra.ra_get_device_status() != 0:
+        raise SystemExit("device status not OK after warm-up")
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    av = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = getattr(props, "uuid", None)
+    gpu_id = f"GPU-{gpu_id}" if gpu_id is not None and not str(gpu_id).startswith("GPU-") else gpu_id
+    clocks = Clocks(gpu_id if gpu_id is not None else local)
+    time.sleep(0.3)
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step(av[i])
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    attn_ms = [a.elapsed_time(b) for a, b in av]
+    total_ms = sum(step_ms)
+    tot = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
+    total_ms = float(tot.item())
+    status = ra.ra_get_device_status()
+
+    # end to end through the public call with host buffers: H2D of Q, K, V from
+    # pinned memory, the call, D2H of out and lse, every step
+    e2e = None
+    if not args.no_e2e:
+        qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        Ke = max(3, min(K, 200))
+
+        def e2e_step():
+            q.copy_(qp, non_blocking=True)
+            k.copy_(kp, non_blocking=True)
+            v.copy_(vp, non_blocking=True)
+            step()
+            out_h.copy_(out, non_blocking=True)
+            lse_h.copy_(lse, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
+        d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+        e2e = {"value": w.flops * world * Ke / (float(e_ms.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke}
+
+    pk, pk_kind = peaks()
+    attn_mean = statistics.mean(attn_ms)
+    sustained = attn_mean > 100.0
+    peak = pk["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    achieved = w.flops / (attn_mean * 1e-3) / 1e12
+    prof = os.path.join(ROOT, "profiles", f"attn_fwd_{w.name}.json")
+    traffic = None
+    if os.path.exists(prof):
+        traffic = json.load(open(prof)).get("dram_bytes_per_launch")
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": traffic, "kernel": "attn_fwd_kernel",
+            "peak_source": f"{pk_kind} {'sustained' if sustained else 'burst'} bf16 dense"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v_, cores, sample, _ = oracle_sample(w)
+        cpu = {"value": v_, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+    value = w.flops * world * K / (total_ms * 1e-3) / 1e12
+    line = {"metric": "causal-adj attention TFLOP/s (% of dense bf16 peak)", "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded randn, bf16-rounded)",
+            "config": workload_config(w, args, f"flushed ({L2_FLUSH_BYTES >> 20} MiB write between steps, "
+                                               f"L2 {l2_bytes >> 20} MiB)"),
+            "pct_of_peak": 100.0 * value / peak, "attn_kernel_ms": attn_mean, "roofline": roof,
+            "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "gpu_launches": K * launches_per_step(w, args.sched),
+            "device_status": ra.ra_status_string(status)}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0 if status == 0 else 1
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

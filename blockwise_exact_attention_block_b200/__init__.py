@@ -1,0 +1,216 @@
+"""Exact blockwise (ring) attention on one B200 - Python binding of libra_b200.so.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in ``include/ra.h``.  PyTorch supplies device
+memory and the current CUDA stream.  There is no CPU fallback: importing this
+package fails loudly when the library is missing, and every call raises
+``RAError`` on a non-OK status.
+
+Names follow the C ABI (``ra_block_attn``, ``ra_merge_partial``,
+``ra_ring_attention`` ...).  Layouts: q/out ``[B, S, Hq, D]``, k/v
+``[B, S, Hkv, D]``, lse ``[B, S, Hq]``, all contiguous.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libra_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m blockwise_exact_attention_block_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_WORKSPACE = 0, 1, 2, 3
+RA_ERR_CUDA, RA_ERR_TIMEOUT, RA_ERR_DEVICE_BOUNDS = 4, 5, 6
+RA_F32, RA_BF16 = 0, 1
+RA_PART_CONTIGUOUS, RA_PART_ZIGZAG = 0, 1
+RA_ORDER_RING, RA_ORDER_TOKENRING = 0, 1
+RA_SCHED_AUTO, RA_SCHED_UNFUSED, RA_SCHED_EPILOGUE_FUSED, RA_SCHED_PERSISTENT = 0, 1, 2, 3
+
+PARTITIONS = {"contiguous": RA_PART_CONTIGUOUS, "zigzag": RA_PART_ZIGZAG}
+ORDERS = {"ring": RA_ORDER_RING, "tokenring": RA_ORDER_TOKENRING}
+SCHEDS = {"auto": RA_SCHED_AUTO, "unfused": RA_SCHED_UNFUSED, "fused": RA_SCHED_EPILOGUE_FUSED,
+          "persistent": RA_SCHED_PERSISTENT}
+
+EXPORTED = ["ra_block_attn", "ra_merge_partial", "ra_merge_partials", "ra_ring_attention",
+            "ra_ring_attention_workspace", "ra_zigzag_permute", "ra_get_device_status",
+            "ra_status_string", "ra_version"]
+
+
+class ra_options(ctypes.Structure):
+    _fields_ = [("order", ctypes.c_int), ("sched", ctypes.c_int), ("attn_event_begin", ctypes.c_void_p),
+                ("attn_event_end", ctypes.c_void_p)]
+
+
+_vp, _i, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+_lib.ra_block_attn.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]
+_lib.ra_block_attn.restype = _i
+_lib.ra_merge_partial.argtypes = [_vp, _vp, _vp, _vp, _i64, _i, _vp]
+_lib.ra_merge_partial.restype = _i
+_lib.ra_merge_partials.argtypes = [ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp, _vp, _i64, _i, _vp]
+_lib.ra_merge_partials.restype = _i
+_lib.ra_ring_attention.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _sz,
+                                   ctypes.POINTER(ra_options), _vp]
+_lib.ra_ring_attention.restype = _i
+_lib.ra_ring_attention_workspace.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(ra_options)]
+_lib.ra_ring_attention_workspace.restype = _sz
+_lib.ra_zigzag_permute.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
+_lib.ra_zigzag_permute.restype = _i
+_lib.ra_get_device_status.argtypes = [_vp]
+_lib.ra_get_device_status.restype = _i
+_lib.ra_status_string.argtypes = [_i]
+_lib.ra_status_string.restype = ctypes.c_char_p
+_lib.ra_version.argtypes = []
+_lib.ra_version.restype = ctypes.c_char_p
+
+
+class RAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {ra_status_string(status)} ({status})")
+
+
+def _check(status: int, what: str) -> None:
+    if status != RA_OK:
+        raise RAError(status, what)
+
+
+def ra_status_string(status: int) -> str:
+    return _lib.ra_status_string(status).decode()
+
+
+def ra_version() -> str:
+    return _lib.ra_version().decode()
+
+
+def _stream(stream=None) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("tensors must be contiguous CUDA tensors")
+    return t.data_ptr()
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return RA_BF16
+    if dt == torch.float32:
+        return RA_F32
+    raise ValueError(f"unsupported dtype {dt}")
+
+
+def _opts(order: str, sched: str, events=None) -> ra_options:
+    o = ra_options(ORDERS[order], SCHEDS[sched], None, None)
+    if events is not None:
+        for ev in events:
+            if ev.cuda_event == 0:  # torch creates the CUDA event on its first record
+                ev.record()
+        o.attn_event_begin = events[0].cuda_event
+        o.attn_event_end = events[1].cuda_event
+    return o
+
+
+def ra_block_attn(q, k, v, S: int, n_blocks: int, q_block: int, kv_block: int, causal: bool,
+                  partition: str = "contiguous", block_out=None, block_lse=None, stream=None):
+    """One query block [B, L, Hq, D] against one KV block [B, L, Hkv, D] (bf16).
+
+    Returns (block_out fp32 [B, L, Hq, D], block_lse fp32 [B, L, Hq])."""
+    B, L, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if block_out is None:
+        block_out = torch.empty((B, L, Hq, D), dtype=torch.float32, device=q.device)
+    if block_lse is None:
+        block_lse = torch.empty((B, L, Hq), dtype=torch.float32, device=q.device)
+    _check(_lib.ra_block_attn(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q.dtype), B, S, n_blocks, q_block, kv_block,
+                              Hq, Hkv, D, int(bool(causal)), PARTITIONS[partition], _ptr(block_out),
+                              _ptr(block_lse), _stream(stream)), "ra_block_attn")
+    return block_out, block_lse
+
+
+def ra_merge_partial(out, lse, block_out, block_lse, stream=None):
+    """In place: (out, lse) <- merge rule with (block_out, block_lse); fp32, rows x D."""
+    D = out.shape[-1]
+    rows = lse.numel()
+    _check(_lib.ra_merge_partial(_ptr(out), _ptr(lse), _ptr(block_out), _ptr(block_lse), rows, D,
+                                 _stream(stream)), "ra_merge_partial")
+    return out, lse
+
+
+def ra_merge_partials(outs, lses, out=None, lse=None, stream=None):
+    """Fold k partials (lists of fp32 tensors) into one (out, lse) in a single pass."""
+    k = len(outs)
+    D = outs[0].shape[-1]
+    rows = lses[0].numel()
+    if out is None:
+        out = torch.empty_like(outs[0])
+    if lse is None:
+        lse = torch.empty_like(lses[0])
+    po = (_vp * k)(*[_ptr(t) for t in outs])
+    pl = (_vp * k)(*[_ptr(t) for t in lses])
+    _check(_lib.ra_merge_partials(po, pl, k, _ptr(out), _ptr(lse), rows, D, _stream(stream)), "ra_merge_partials")
+    return out, lse
+
+
+def ra_ring_attention_workspace(B, S, Hq, D, n_blocks, gqa_groups, partition="contiguous",
+                                in_dtype=torch.bfloat16, order="ring", sched="auto") -> int:
+    o = _opts(order, sched)
+    n = _lib.ra_ring_attention_workspace(B, S, Hq, D, n_blocks, gqa_groups, PARTITIONS[partition],
+                                         _dtype_code(in_dtype), ctypes.byref(o))
+    if n == ctypes.c_size_t(-1).value:
+        raise RAError(RA_ERR_INVALID_ARG, "ra_ring_attention_workspace")
+    return n
+
+
+def ra_ring_attention(q, k, v, n_blocks: int, causal: bool, partition: str = "contiguous",
+                      gqa_groups: int | None = None, out=None, out_dtype=torch.float32, lse=None,
+                      workspace=None, order: str = "ring", sched: str = "auto", stream=None,
+                      attn_events=None):
+    """The whole method on one GPU.  Returns (out [B, S, Hq, D], lse fp32 [B, S, Hq]).
+
+    attn_events: optional pair of torch.cuda.Event recorded around the
+    block-attention launches inside the call."""
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if gqa_groups is None:
+        gqa_groups = Hq // Hkv
+    if out is None:
+        out = torch.empty((B, S, Hq, D), dtype=out_dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, S, Hq), dtype=torch.float32, device=q.device)
+    need = ra_ring_attention_workspace(B, S, Hq, D, n_blocks, gqa_groups, partition, q.dtype, order, sched)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    o = _opts(order, sched, attn_events)
+    _check(_lib.ra_ring_attention(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q.dtype), B, S, Hq, D, n_blocks,
+                                  int(bool(causal)), PARTITIONS[partition], gqa_groups, _ptr(out),
+                                  _dtype_code(out.dtype), _ptr(lse), _ptr(workspace), ws_bytes, ctypes.byref(o),
+                                  _stream(stream)), "ra_ring_attention")
+    return out, lse
+
+
+def ra_zigzag_permute(src, n_blocks: int, inverse: bool = False, dst=None, stream=None):
+    """Rows of [B, S, H, D] between original and zigzag block order (bit-exact)."""
+    B, S, H, D = src.shape
+    if dst is None:
+        dst = torch.empty_like(src)
+    _check(_lib.ra_zigzag_permute(_ptr(src), _ptr(dst), B, S, H, D, src.element_size(), n_blocks,
+                                  int(bool(inverse)), _stream(stream)), "ra_zigzag_permute")
+    return dst
+
+
+def ra_get_device_status(stream=None) -> int:
+    """Reads and clears the device status word (synchronises the stream)."""
+    return _lib.ra_get_device_status(_stream(stream))

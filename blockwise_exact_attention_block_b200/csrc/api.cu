@@ -1,0 +1,501 @@
+// api.cu - the C ABI of libra_b200.so (include/ra.h): argument validation,
+// TMA tensor maps, and the block scheduler that replays the ring / TokenRing
+// order on one GPU.  The whole library is this one translation unit, so the
+// device status word in common.cuh has a single definition.
+//
+// Schedules (Anthology of the SOTA, SOTA-181: the query block stays, KV
+// blocks pass around the ring; TokenRing review, "Core claim" and "major
+// comments, Algorithm 1 (section 3.2)": the KV block stays, query blocks move
+// forward and partial results move back):
+//   ring:      query block r meets KV blocks r, r-1, r-2, ... (mod n)
+//   TokenRing: query block r meets KV blocks r, r+1, r+2, ... (mod n)
+// (TokenRing step s, 1-based, pairs KV block j with query block
+// (j - s + 1) mod n, i.e. query block r with KV block (r + s - 1) mod n.)
+#include <math.h>
+#include <stdio.h>
+
+#include <mutex>
+
+#include "attn_fwd.cuh"
+#include "merge.cuh"
+#include "permute.cuh"
+
+namespace {
+
+using namespace ra;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor viewed as [NB][L][H][D] (innermost last), box = 128 rows x 64
+// columns of one head, 128-byte swizzle.  Rows beyond L read as zero.
+bool make_map(CUtensorMap* m, const void* ptr, int D, int H, int L, int NB) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(NB)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
+                                 static_cast<cuuint64_t>(L) * H * D * 2};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kBM), 1};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline ra_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RA_OK : RA_ERR_CUDA; }
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+inline int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+struct Geom {
+  int B, S, n, L, c, Hq, Hkv, groups, D, zigzag, causal;
+};
+
+ra_status check_geom(int B, int S, int n, int Hq, int Hkv, int D, int partition, Geom* g) {
+  if (B < 1 || S < 1 || Hq < 1 || Hkv < 1 || n < 1) return RA_ERR_INVALID_ARG;
+  if (n > kMaxBlocks) return RA_ERR_UNSUPPORTED;
+  if (partition != RA_PART_CONTIGUOUS && partition != RA_PART_ZIGZAG) return RA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return RA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
+  if (S % n != 0) return RA_ERR_INVALID_ARG;
+  if (partition == RA_PART_ZIGZAG && S % (2 * n) != 0) return RA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * n > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
+  g->B = B;
+  g->S = S;
+  g->n = n;
+  g->L = S / n;
+  g->c = S / (2 * n);
+  g->Hq = Hq;
+  g->Hkv = Hkv;
+  g->groups = Hq / Hkv;
+  g->D = D;
+  g->zigzag = partition == RA_PART_ZIGZAG;
+  g->causal = 0;
+  return RA_OK;
+}
+
+AttnArgs base_args(const Geom& g) {
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = g.B;
+  a.S = g.S;
+  a.n = g.n;
+  a.L = g.L;
+  a.c = g.c;
+  a.Hq = g.Hq;
+  a.Hkv = g.Hkv;
+  a.groups = g.groups;
+  a.zigzag = g.zigzag;
+  a.causal = g.causal;
+  a.tiles_per_block = (g.L + kBM - 1) / kBM;
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(g.D)));
+  return a;
+}
+
+template <int D>
+ra_status launch_attn_t(const AttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                        cudaStream_t st) {
+  constexpr int NST = D == 128 ? 2 : 4;
+  using SL = AttnSmem<D, NST>;
+  static int attr_set[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, NST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SL::kBytes);
+    if (e != cudaSuccess) return RA_ERR_CUDA;
+    attr_set[dev] = 1;
+  }
+  const long long grid = static_cast<long long>(a.Hq) * a.B * a.nq * a.tiles_per_block;
+  if (grid <= 0) return RA_OK;
+  if (grid > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
+  attn_fwd_kernel<D, NST><<<static_cast<unsigned>(grid), kAttnThreads, SL::kBytes, st>>>(mq, mk, mv, a);
+  return cuda_status(cudaGetLastError());
+}
+
+ra_status launch_attn(int D, const AttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mk,
+                      const CUtensorMap& mv, cudaStream_t st) {
+  return D == 128 ? launch_attn_t<128>(a, mq, mk, mv, st) : launch_attn_t<64>(a, mq, mk, mv, st);
+}
+
+int grid_for(long long work, int per_block) {
+  const long long need = (work + per_block - 1) / per_block;
+  const long long cap = static_cast<long long>(sm_count()) * 16;
+  return static_cast<int>(need < 1 ? 1 : (need < cap ? need : cap));
+}
+
+ra_status launch_merge(float* out, float* lse, const float* bo, const float* bl, long long rows, int D,
+                       cudaStream_t st) {
+  const long long nvec = rows * (D / 4);
+  merge_partial_kernel<<<grid_for(nvec, kMergeThreads * kMergeUnroll), kMergeThreads, 0, st>>>(
+      out, lse, bo, bl, rows, D / 4);
+  return cuda_status(cudaGetLastError());
+}
+
+// Row move between original and block order, bit-exact, for rows and base
+// addresses that are multiples of 2 bytes.
+ra_status launch_permute_bytes(const void* src, void* dst, int B, const PermGeom& pg, long long row_bytes,
+                               int inverse, cudaStream_t st) {
+  const long long rows = static_cast<long long>(B) * pg.S;
+  // widest vector that divides the row size and both base addresses
+  const unsigned long long mix = reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst) |
+                                 static_cast<unsigned long long>(row_bytes);
+  const int width = (mix & 15) == 0 ? 16 : (mix & 7) == 0 ? 8 : (mix & 3) == 0 ? 4 : 2;
+  if (width == 16) {
+    const long long rv = row_bytes / 16;
+    permute_rows_kernel<uint4><<<grid_for(rows * rv, 256), 256, 0, st>>>(
+        static_cast<const uint4*>(src), static_cast<uint4*>(dst), B, pg, rv, inverse);
+  } else if (width == 8) {
+    const long long rv = row_bytes / 8;
+    permute_rows_kernel<uint2><<<grid_for(rows * rv, 256), 256, 0, st>>>(
+        static_cast<const uint2*>(src), static_cast<uint2*>(dst), B, pg, rv, inverse);
+  } else if (width == 4) {
+    const long long rv = row_bytes / 4;
+    permute_rows_kernel<uint32_t><<<grid_for(rows * rv, 256), 256, 0, st>>>(
+        static_cast<const uint32_t*>(src), static_cast<uint32_t*>(dst), B, pg, rv, inverse);
+  } else {
+    const long long rv = row_bytes / 2;
+    permute_rows_kernel<uint16_t><<<grid_for(rows * rv, 256), 256, 0, st>>>(
+        static_cast<const uint16_t*>(src), static_cast<uint16_t*>(dst), B, pg, rv, inverse);
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+PermGeom perm_geom(const Geom& g) {
+  PermGeom p;
+  p.S = g.S;
+  p.L = g.L;
+  p.c = g.c;
+  p.n = g.n;
+  p.zigzag = g.zigzag;
+  return p;
+}
+
+// Workspace plan of ra_ring_attention; offsets in bytes.
+struct Plan {
+  ra_sched sched;
+  bool copy_inputs;
+  size_t q, k, v, acc_out, acc_lse, part_out, part_lse, total;
+};
+
+Plan make_plan(const Geom& g, ra_dtype in_dtype, const ra_options* opts) {
+  Plan p;
+  memset(&p, 0, sizeof(p));
+  p.sched = opts ? opts->sched : RA_SCHED_AUTO;
+  if (p.sched == RA_SCHED_AUTO) p.sched = RA_SCHED_PERSISTENT;
+  p.copy_inputs = g.zigzag || in_dtype == RA_F32;
+  const size_t rows = static_cast<size_t>(g.B) * g.S;
+  size_t off = 0;
+  if (p.copy_inputs) {
+    p.q = off;
+    off = align256(off + rows * g.Hq * g.D * 2);
+    p.k = off;
+    off = align256(off + rows * g.Hkv * g.D * 2);
+    p.v = off;
+    off = align256(off + rows * g.Hkv * g.D * 2);
+  }
+  if (p.sched != RA_SCHED_PERSISTENT) {
+    p.acc_out = off;
+    off = align256(off + rows * g.Hq * g.D * 4);
+    p.acc_lse = off;
+    off = align256(off + rows * g.Hq * 4);
+    if (p.sched == RA_SCHED_UNFUSED) {
+      p.part_out = off;
+      off = align256(off + rows * g.Hq * g.D * 4);
+      p.part_lse = off;
+      off = align256(off + rows * g.Hq * 4);
+    }
+  }
+  p.total = off;
+  return p;
+}
+
+bool valid_opts(const ra_options* o) {
+  if (!o) return true;
+  if (o->order != RA_ORDER_RING && o->order != RA_ORDER_TOKENRING) return false;
+  return o->sched >= RA_SCHED_AUTO && o->sched <= RA_SCHED_PERSISTENT;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ra_status_string(ra_status s) {
+  switch (s) {
+    case RA_OK: return "RA_OK";
+    case RA_ERR_INVALID_ARG: return "RA_ERR_INVALID_ARG";
+    case RA_ERR_UNSUPPORTED: return "RA_ERR_UNSUPPORTED";
+    case RA_ERR_WORKSPACE: return "RA_ERR_WORKSPACE";
+    case RA_ERR_CUDA: return "RA_ERR_CUDA";
+    case RA_ERR_TIMEOUT: return "RA_ERR_TIMEOUT";
+    case RA_ERR_DEVICE_BOUNDS: return "RA_ERR_DEVICE_BOUNDS";
+  }
+  return "RA_ERR_UNKNOWN";
+}
+
+const char* ra_version(void) { return "ra_b200 0.1 (sm_100a)"; }
+
+ra_status ra_get_device_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return RA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return RA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return RA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return RA_ERR_CUDA;
+  }
+  return static_cast<ra_status>(v);
+}
+
+ra_status ra_block_attn(const void* q, const void* k, const void* v, ra_dtype in_dtype, int B, int S,
+                        int n_blocks, int q_block, int kv_block, int Hq, int Hkv, int D, int causal,
+                        ra_partition partition, float* block_out, float* block_lse, void* stream) {
+  Geom g;
+  ra_status s = check_geom(B, S, n_blocks, Hq, Hkv, D, partition, &g);
+  if (s != RA_OK) return s;
+  if (in_dtype != RA_BF16) return in_dtype == RA_F32 ? RA_ERR_UNSUPPORTED : RA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !block_out || !block_lse) return RA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(block_out) || !aligned16(block_lse))
+    return RA_ERR_INVALID_ARG;
+  if (q_block < 0 || q_block >= n_blocks || kv_block < 0 || kv_block >= n_blocks) return RA_ERR_INVALID_ARG;
+  g.causal = causal != 0;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, D, Hq, g.L, B) || !make_map(&mk, k, D, Hkv, g.L, B) || !make_map(&mv, v, D, Hkv, g.L, B))
+    return RA_ERR_CUDA;
+  AttnArgs a = base_args(g);
+  a.nq = 1;
+  a.nkv = 1;
+  a.q_blocks[0] = static_cast<signed char>(q_block);
+  a.kv_list[0][0] = static_cast<signed char>(kv_block);
+  a.q_bmul = 1;
+  a.q_rmul = 0;
+  a.kv_bmul = 1;
+  a.kv_rmul = 0;
+  a.mode = kModePartial;
+  a.acc_out = block_out;
+  a.acc_lse = block_lse;
+  a.acc_brows = g.L;
+  a.acc_rmul = 0;
+  return launch_attn(D, a, mq, mk, mv, static_cast<cudaStream_t>(stream));
+}
+
+ra_status ra_merge_partial(float* out, float* lse, const float* block_out, const float* block_lse, int64_t rows,
+                           int D, void* stream) {
+  if (rows < 0 || D <= 0) return RA_ERR_INVALID_ARG;
+  if (D % 4 != 0 || D > 128 || 32 % (D / 4) != 0) return RA_ERR_UNSUPPORTED;
+  if (rows == 0) return RA_OK;
+  if (!out || !lse || !block_out || !block_lse) return RA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(block_out) || (reinterpret_cast<uintptr_t>(lse) & 3) ||
+      (reinterpret_cast<uintptr_t>(block_lse) & 3))
+    return RA_ERR_INVALID_ARG;
+  return launch_merge(out, lse, block_out, block_lse, rows, D, static_cast<cudaStream_t>(stream));
+}
+
+ra_status ra_merge_partials(const float* const* outs, const float* const* lses, int k, float* out, float* lse,
+                            int64_t rows, int D, void* stream) {
+  if (rows < 0 || D <= 0 || k < 1 || !outs || !lses) return RA_ERR_INVALID_ARG;
+  if (k > kMaxMergeInputs) return RA_ERR_UNSUPPORTED;
+  if (D % 4 != 0 || D > 128 || 32 % (D / 4) != 0) return RA_ERR_UNSUPPORTED;
+  if (rows == 0) return RA_OK;
+  if (!out || !lse || !aligned16(out) || (reinterpret_cast<uintptr_t>(lse) & 3)) return RA_ERR_INVALID_ARG;
+  MergeList ml;
+  memset(&ml, 0, sizeof(ml));
+  for (int j = 0; j < k; ++j) {
+    if (!outs[j] || !lses[j] || !aligned16(outs[j]) || (reinterpret_cast<uintptr_t>(lses[j]) & 3))
+      return RA_ERR_INVALID_ARG;
+    ml.outs[j] = outs[j];
+    ml.lses[j] = lses[j];
+  }
+  const long long nvec = rows * (D / 4);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  merge_partials_kernel<<<grid_for(nvec, kMergeThreads), kMergeThreads, 0, st>>>(ml, k, out, lse, rows, D / 4);
+  return cuda_status(cudaGetLastError());
+}
+
+ra_status ra_zigzag_permute(const void* src, void* dst, int B, int S, int H, int D, int elem_bytes, int n_blocks,
+                            int inverse, void* stream) {
+  if (!src || !dst || B < 1 || S < 1 || H < 1 || D < 1 || n_blocks < 1) return RA_ERR_INVALID_ARG;
+  if (elem_bytes != 2 && elem_bytes != 4) return RA_ERR_INVALID_ARG;
+  if (S % (2 * n_blocks) != 0) return RA_ERR_INVALID_ARG;
+  if (inverse != 0 && inverse != 1) return RA_ERR_INVALID_ARG;
+  if (src == dst) return RA_ERR_INVALID_ARG;
+  const long long row_bytes = static_cast<long long>(H) * D * elem_bytes;
+  const char* s0 = static_cast<const char*>(src);
+  const char* d0 = static_cast<const char*>(dst);
+  const long long tot = static_cast<long long>(B) * S * row_bytes;
+  if (s0 < d0 + tot && d0 < s0 + tot) return RA_ERR_INVALID_ARG;  // overlap
+  if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & (elem_bytes - 1))
+    return RA_ERR_INVALID_ARG;
+  PermGeom pg;
+  pg.S = S;
+  pg.n = n_blocks;
+  pg.L = S / n_blocks;
+  pg.c = S / (2 * n_blocks);
+  pg.zigzag = 1;
+  return launch_permute_bytes(src, dst, B, pg, row_bytes, inverse, static_cast<cudaStream_t>(stream));
+}
+
+size_t ra_ring_attention_workspace(int B, int S, int Hq, int D, int n_blocks, int gqa_groups, ra_partition partition,
+                                   ra_dtype in_dtype, const ra_options* opts) {
+  if (gqa_groups < 1 || Hq % gqa_groups != 0) return static_cast<size_t>(-1);
+  Geom g;
+  if (check_geom(B, S, n_blocks, Hq, Hq / gqa_groups, D, partition, &g) != RA_OK) return static_cast<size_t>(-1);
+  if (in_dtype != RA_F32 && in_dtype != RA_BF16) return static_cast<size_t>(-1);
+  if (!valid_opts(opts)) return static_cast<size_t>(-1);
+  return make_plan(g, in_dtype, opts).total;
+}
+
+ra_status ra_ring_attention(const void* q, const void* k, const void* v, ra_dtype in_dtype, int B, int S, int Hq,
+                            int D, int n_blocks, int causal, ra_partition partition, int gqa_groups, void* out,
+                            ra_dtype out_dtype, float* lse, void* workspace, size_t workspace_bytes,
+                            const ra_options* opts, void* stream) {
+  if (gqa_groups < 1 || Hq < 1 || Hq % gqa_groups != 0) return RA_ERR_INVALID_ARG;
+  Geom g;
+  ra_status s = check_geom(B, S, n_blocks, Hq, Hq / gqa_groups, D, partition, &g);
+  if (s != RA_OK) return s;
+  g.causal = causal != 0;
+  if (in_dtype != RA_F32 && in_dtype != RA_BF16) return RA_ERR_INVALID_ARG;
+  if (out_dtype != RA_F32 && out_dtype != RA_BF16) return RA_ERR_INVALID_ARG;
+  if (!valid_opts(opts)) return RA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out || !lse) return RA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return RA_ERR_INVALID_ARG;
+  const Plan p = make_plan(g, in_dtype, opts);
+  if (p.total > 0) {
+    if (!workspace || workspace_bytes < p.total) return RA_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return RA_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  const PermGeom pg = perm_geom(g);
+  const ra_order order = opts ? opts->order : RA_ORDER_RING;
+
+  // a2: partition (and fp32 -> bf16 rounding) of the inputs into block order
+  const void* qb = q;
+  const void* kb = k;
+  const void* vb = v;
+  if (p.copy_inputs) {
+    struct { const void* src; size_t off; int H; } mv[3] = {{q, p.q, g.Hq}, {k, p.k, g.Hkv}, {v, p.v, g.Hkv}};
+    for (auto& m : mv) {
+      const long long row_elems = static_cast<long long>(m.H) * D;
+      if (in_dtype == RA_BF16) {
+        s = launch_permute_bytes(m.src, ws + m.off, B, pg, row_elems * 2, 0, st);
+      } else {
+        const long long rows = static_cast<long long>(B) * S;
+        permute_cast_kernel<float, __nv_bfloat16><<<grid_for(rows * row_elems / 8, 256), 256, 0, st>>>(
+            static_cast<const float*>(m.src), reinterpret_cast<__nv_bfloat16*>(ws + m.off), B, pg, row_elems, 0);
+        s = cuda_status(cudaGetLastError());
+      }
+      if (s != RA_OK) return s;
+    }
+    qb = ws + p.q;
+    kb = ws + p.k;
+    vb = ws + p.v;
+  }
+
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, qb, D, g.Hq, g.L, B * g.n) || !make_map(&mk, kb, D, g.Hkv, g.L, B * g.n) ||
+      !make_map(&mv, vb, D, g.Hkv, g.L, B * g.n))
+    return RA_ERR_CUDA;
+
+  // a7: the order in which each query block meets the KV blocks
+  int kv_order[kMaxBlocks][kMaxBlocks];
+  for (int r = 0; r < g.n; ++r)
+    for (int t = 0; t < g.n; ++t)
+      kv_order[r][t] = order == RA_ORDER_RING ? ((r - t) % g.n + g.n) % g.n : (r + t) % g.n;
+
+  AttnArgs a = base_args(g);
+  a.nq = g.n;
+  for (int r = 0; r < g.n; ++r) a.q_blocks[r] = static_cast<signed char>(r);
+  a.q_bmul = g.n;
+  a.q_rmul = 1;
+  a.kv_bmul = g.n;
+  a.kv_rmul = 1;
+
+  if (p.sched == RA_SCHED_PERSISTENT) {
+    // a3-a6 in one launch: the running state is carried across block boundaries
+    a.nkv = g.n;
+    for (int r = 0; r < g.n; ++r)
+      for (int t = 0; t < g.n; ++t) a.kv_list[r][t] = static_cast<signed char>(kv_order[r][t]);
+    a.mode = kModeFinal;
+    a.out = out;
+    a.lse = lse;
+    a.out_bf16 = out_dtype == RA_BF16;
+    if (opts && opts->attn_event_begin) cudaEventRecord(static_cast<cudaEvent_t>(opts->attn_event_begin), st);
+    s = launch_attn(D, a, mq, mk, mv, st);
+    if (s == RA_OK && opts && opts->attn_event_end) cudaEventRecord(static_cast<cudaEvent_t>(opts->attn_event_end), st);
+    return s;
+  }
+
+  float* acc_out = reinterpret_cast<float*>(ws + p.acc_out);
+  float* acc_lse = reinterpret_cast<float*>(ws + p.acc_lse);
+  const long long rows = static_cast<long long>(B) * S * g.Hq;
+  a.nkv = 1;
+  a.acc_brows = S;
+  a.acc_rmul = 1;
+  if (opts && opts->attn_event_begin) cudaEventRecord(static_cast<cudaEvent_t>(opts->attn_event_begin), st);
+  for (int step = 0; step < g.n; ++step) {
+    for (int r = 0; r < g.n; ++r) a.kv_list[r][0] = static_cast<signed char>(kv_order[r][step]);
+    if (step == 0) {
+      a.mode = kModePartial;
+      a.acc_out = acc_out;
+      a.acc_lse = acc_lse;
+    } else if (p.sched == RA_SCHED_EPILOGUE_FUSED) {
+      a.mode = kModeMerge;
+      a.acc_out = acc_out;
+      a.acc_lse = acc_lse;
+    } else {
+      a.mode = kModePartial;
+      a.acc_out = reinterpret_cast<float*>(ws + p.part_out);
+      a.acc_lse = reinterpret_cast<float*>(ws + p.part_lse);
+    }
+    s = launch_attn(D, a, mq, mk, mv, st);
+    if (s != RA_OK) return s;
+    if (step > 0 && p.sched == RA_SCHED_UNFUSED) {
+      s = launch_merge(acc_out, acc_lse, a.acc_out, a.acc_lse, rows, D, st);
+      if (s != RA_OK) return s;
+    }
+  }
+  if (opts && opts->attn_event_end) cudaEventRecord(static_cast<cudaEvent_t>(opts->attn_event_end), st);
+  // a8: back to original token order, with the cast of out
+  const long long row_elems = static_cast<long long>(g.Hq) * D;
+  if (out_dtype == RA_BF16) {
+    permute_cast_kernel<float, __nv_bfloat16><<<grid_for(static_cast<long long>(B) * S * row_elems / 8, 256), 256, 0, st>>>(
+        acc_out, static_cast<__nv_bfloat16*>(out), B, pg, row_elems, 1);
+    s = cuda_status(cudaGetLastError());
+  } else {
+    s = launch_permute_bytes(acc_out, out, B, pg, row_elems * 4, 1, st);
+  }
+  if (s != RA_OK) return s;
+  return launch_permute_bytes(acc_lse, lse, B, pg, static_cast<long long>(g.Hq) * 4, 1, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,199 @@
+/*
+ * ra.h - exact blockwise (ring) attention on one NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libra_b200.so.  Plain pointers and sizes only; every pointer named
+ * "device" is a CUDA device address, every buffer is owned by the caller, and
+ * the library allocates no memory.  Calls are asynchronous on `stream`
+ * (a cudaStream_t passed as void*; NULL = the legacy default stream).  Argument
+ * validation is synchronous: an invalid call returns an error status before
+ * anything is launched and leaves every buffer untouched.  Errors that only a
+ * kernel can see (a bounded wait that ran out, an index out of range) are
+ * recorded in a device status word that ra_get_device_status() reads.
+ *
+ * Sources, by page title and section:
+ *  [TR]  TokenRing review (pith.science, arXiv 2412.20501).
+ *        "What carries the argument": the update rule that stitches partial
+ *        outputs, out <- out - sigma(block_lse - lse) * (out - block_out),
+ *        lse <- lse - ln sigma(lse - block_lse).
+ *        "Core claim" / "Referee Report, Summary": Q, K, V split along the
+ *        token dimension; a flash-attention kernel returns (block_out,
+ *        block_lse) per query block and key/value block.
+ *        "If this is right": zigzag causal partition; grouped-query attention.
+ *        "major comments, Algorithm 1 (section 3.2)": TokenRing step index.
+ *  [RA]  Anthology of the SOTA, SOTA-181 (Liu et al. 2023, ring attention):
+ *        each device keeps its query block and passes key/value blocks
+ *        around the ring; exact attention.
+ *
+ * Layouts (token-major, row-major, no padding):
+ *   q, out      [B, S, Hq,  D]     k, v   [B, S, Hkv, D]     lse [B, S, Hq]
+ * with Hq = Hkv * gqa_groups; query head h reads KV head h / gqa_groups.
+ * The softmax scale is 1/sqrt(D); lse is a natural logarithm.
+ * Supported: D in {64, 128}; bf16 attention inputs (fp32 inputs to
+ * ra_ring_attention are rounded to bf16, round-to-nearest-even, on entry).
+ * All device pointers must be 16-byte aligned.
+ */
+#ifndef RA_B200_H
+#define RA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RA_OK = 0,
+  RA_ERR_INVALID_ARG = 1,   /* bad shape, null or misaligned pointer, bad enum  */
+  RA_ERR_UNSUPPORTED = 2,   /* valid but outside what this build implements      */
+  RA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than the query says  */
+  RA_ERR_CUDA = 4,          /* a CUDA runtime / driver call failed               */
+  RA_ERR_TIMEOUT = 5,       /* device: a bounded wait ran out (kernel returned)  */
+  RA_ERR_DEVICE_BOUNDS = 6  /* device: an index check failed (access skipped)    */
+} ra_status;
+
+typedef enum { RA_F32 = 0, RA_BF16 = 1 } ra_dtype;
+
+/* [TR] "If this is right" (zigzag) and "Referee Report, Summary" (contiguous).
+ * Contiguous: block r = tokens [r*L, (r+1)*L), L = S / n_blocks.
+ * Zigzag: chunk size c = S / (2 n_blocks); block r = chunk r then chunk
+ * 2 n_blocks - 1 - r.  Requires S % (2 n_blocks) == 0. */
+typedef enum { RA_PART_CONTIGUOUS = 0, RA_PART_ZIGZAG = 1 } ra_partition;
+
+/* Order in which each query block meets the KV blocks.
+ * Ring [RA]: at step s = 0..n-1 query block r meets KV block (r - s) mod n.
+ * TokenRing [TR, Algorithm 1]: at step = 1..n KV block j meets query block
+ * (j - step + 1) mod n.  The result is the same up to rounding. */
+typedef enum { RA_ORDER_RING = 0, RA_ORDER_TOKENRING = 1 } ra_order;
+
+/* How ra_ring_attention runs the schedule on one GPU.
+ *  UNFUSED:          per ring step one ra_block_attn-style launch over all n
+ *                    (q block, kv block) pairs of the step, writing fp32
+ *                    partials, then one merge launch (ra_merge_partial).
+ *  EPILOGUE_FUSED:   the same launches, the attention epilogue applies the
+ *                    merge rule to the running (out, lse) in HBM itself.
+ *  PERSISTENT:       one launch; each CTA owns a (query tile, head) and walks
+ *                    the KV blocks in schedule order, carrying the running
+ *                    softmax state on chip across block boundaries; output is
+ *                    written once, in original token order.
+ *  AUTO:             PERSISTENT. */
+typedef enum {
+  RA_SCHED_AUTO = 0,
+  RA_SCHED_UNFUSED = 1,
+  RA_SCHED_EPILOGUE_FUSED = 2,
+  RA_SCHED_PERSISTENT = 3
+} ra_sched;
+
+typedef struct {
+  ra_order order;  /* default RA_ORDER_RING  */
+  ra_sched sched;  /* default RA_SCHED_AUTO  */
+  /* Optional cudaEvent_t handles (NULL = unused), recorded on `stream` right
+   * before the first and right after the last block-attention launch of the
+   * call, so a caller can time the attention kernels inside the full call. */
+  void* attn_event_begin;
+  void* attn_event_end;
+} ra_options;
+
+/*
+ * ra_block_attn - one query block against one key/value block.
+ * [TR] "What carries the argument" / "Core claim": the flash-attention kernel
+ * that returns (block_out, block_lse) for one block pair.
+ *
+ *  q          device, bf16, [B, L, Hq, D]: the rows of query block q_block
+ *             (block-local, in partition order; L = S / n_blocks).
+ *  k, v       device, bf16, [B, L, Hkv, D]: the rows of KV block kv_block.
+ *  in_dtype   must be RA_BF16 (else RA_ERR_UNSUPPORTED).
+ *  B, S       batch and full sequence length; n_blocks blocks of L tokens.
+ *  q_block, kv_block   block indices in [0, n_blocks); with `partition` they
+ *             give every row's original token position, used by the mask.
+ *  Hq, Hkv, D head counts (Hq % Hkv == 0) and head dim (64 or 128).
+ *  causal     nonzero: key j visible to query i iff pos(j) <= pos(i).
+ *  block_out  device, fp32, [B, L, Hq, D], written (softmax-normalised).
+ *  block_lse  device, fp32, [B, L, Hq], written.  A row that sees no key of
+ *             this block gets block_lse = -inf and block_out = 0.
+ */
+ra_status ra_block_attn(const void* q, const void* k, const void* v, ra_dtype in_dtype,
+                        int B, int S, int n_blocks, int q_block, int kv_block,
+                        int Hq, int Hkv, int D, int causal, ra_partition partition,
+                        float* block_out, float* block_lse, void* stream);
+
+/*
+ * ra_merge_partial - one application of the update rule, in place, fp32.
+ * [TR] "What carries the argument":
+ *     out <- out - sigma(block_lse - lse) * (out - block_out)
+ *     lse <- lse - ln sigma(lse - block_lse)
+ *  out, lse              device fp32 [rows, D] / [rows], read and written.
+ *  block_out, block_lse  device fp32 [rows, D] / [rows], read only.
+ *  rows, D               rows >= 0 (0 is a no-op), D > 0 and D % 4 == 0.
+ * lse = -inf marks an empty partial: merging an empty block_lse is a no-op;
+ * merging into an empty lse copies the partial.
+ */
+ra_status ra_merge_partial(float* out, float* lse, const float* block_out,
+                           const float* block_lse, int64_t rows, int D, void* stream);
+
+/*
+ * ra_merge_partials - k partials folded into one result in a single pass
+ * (the same rule applied k-1 times, left to right, on chip).
+ *  outs, lses    host arrays of k device pointers: fp32 [rows, D] / [rows].
+ *  out, lse      device fp32 [rows, D] / [rows], written (may alias outs[0],
+ *                lses[0]).  1 <= k <= 16.
+ */
+ra_status ra_merge_partials(const float* const* outs, const float* const* lses, int k,
+                            float* out, float* lse, int64_t rows, int D, void* stream);
+
+/*
+ * ra_ring_attention - the whole method: partition, schedule, block attention,
+ * merge, and the final cast / return to original token order.
+ *  q, k, v       device, in_dtype (RA_BF16 or RA_F32), original token order.
+ *  B, S, Hq, D   shapes; Hkv = Hq / gqa_groups.
+ *  n_blocks      ring size n >= 1, <= 16; S % n == 0 (contiguous) or
+ *                S % (2n) == 0 (zigzag).
+ *  causal        nonzero for causal attention over original positions.
+ *  out           device, out_dtype (RA_F32 or RA_BF16; bf16 is rounded to
+ *                nearest even from the fp32 result), [B, S, Hq, D].
+ *  lse           device fp32 [B, S, Hq].
+ *  workspace     device scratch of at least ra_ring_attention_workspace()
+ *                bytes (may be NULL when that is 0), 256-byte aligned.
+ *  opts          NULL for defaults.
+ */
+ra_status ra_ring_attention(const void* q, const void* k, const void* v, ra_dtype in_dtype,
+                            int B, int S, int Hq, int D, int n_blocks, int causal,
+                            ra_partition partition, int gqa_groups,
+                            void* out, ra_dtype out_dtype, float* lse,
+                            void* workspace, size_t workspace_bytes,
+                            const ra_options* opts, void* stream);
+
+/* Bytes of workspace ra_ring_attention needs for these arguments; 0 when
+ * none is needed; (size_t)-1 when the arguments are invalid. */
+size_t ra_ring_attention_workspace(int B, int S, int Hq, int D, int n_blocks, int gqa_groups,
+                                   ra_partition partition, ra_dtype in_dtype,
+                                   const ra_options* opts);
+
+/*
+ * ra_zigzag_permute - reorder token rows between original order and the
+ * partition's block order ([TR] "If this is right", zigzag partition).
+ *  src, dst      device [B, S, H, D] of elem_bytes each (2 or 4); no overlap.
+ *  inverse = 0:  dst[b, p] = src[b, perm[p]]   (original -> block order)
+ *  inverse = 1:  dst[b, perm[p]] = src[b, p]   (block order -> original)
+ * with perm[r*L + t] = r*c + t for t < c, (2n-1-r)*c + (t - c) otherwise.
+ * A pure copy: bit-exact.
+ */
+ra_status ra_zigzag_permute(const void* src, void* dst, int B, int S, int H, int D,
+                            int elem_bytes, int n_blocks, int inverse, void* stream);
+
+/* Reads and clears the device status word (synchronises `stream`).  Returns
+ * RA_OK, RA_ERR_TIMEOUT or RA_ERR_DEVICE_BOUNDS, or RA_ERR_CUDA when the read
+ * itself fails. */
+ra_status ra_get_device_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* ra_status_string(ra_status s);
+
+/* Library version string. */
+const char* ra_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RA_B200_H */

@@ -71,28 +71,40 @@ def full_attention(q, k, v, causal: bool, gqa_groups: int = 1, row_chunk: int = 
     return out, lse
 
 
-def attention_rows(q, k, v, rows, causal: bool, gqa_groups: int = 1):
-    """Exact attention for selected query rows only, one row at a time.
+def attention_rows(q, k, v, rows, causal: bool, gqa_groups: int = 1, batch: int = 32):
+    """Exact attention for selected query rows only.
 
     rows: iterable of (b, i, h).  Returns (out [R, D], lse [R]) in fp64.
     Used where the full oracle is too large: each sampled row is computed
-    against every key it may see.
+    against every key it may see.  ``batch`` bounds how many rows are
+    evaluated together (memory only; the result does not depend on it).
     """
     rows = list(rows)
     D = q.shape[-1]
     scale = softmax_scale(D)
     out = np.zeros((len(rows), D), dtype=np.float64)
     lse = np.zeros((len(rows),), dtype=np.float64)
+    # Rows that share (batch, KV head) are evaluated together against that
+    # head's keys (a matrix product instead of one matrix-vector product per
+    # row); each row still sees every key it may see, in one softmax.
+    groups = {}
     for r, (b, i, h) in enumerate(rows):
-        g = h // gqa_groups
-        jmax = i + 1 if causal else q.shape[1]
-        qi = _f64(q[b, i, h, :])
-        kk = _f64(k[b, :jmax, g, :])
-        vv = _f64(v[b, :jmax, g, :])
-        s = (kk @ qi) * scale
-        m = s.max()
-        e = np.exp(s - m)
-        tot = e.sum()
-        lse[r] = m + math.log(tot)
-        out[r] = (e / tot) @ vv
+        groups.setdefault((b, h // gqa_groups), []).append(r)
+    for (b, g), idx in groups.items():
+        jall = max(rows[r][1] for r in idx) + 1 if causal else q.shape[1]
+        kk = _f64(k[b, :jall, g, :])
+        vv = _f64(v[b, :jall, g, :])
+        for s0 in range(0, len(idx), batch):
+            sel = idx[s0:s0 + batch]
+            ii = np.array([rows[r][1] for r in sel])
+            jmax = int(ii.max()) + 1 if causal else q.shape[1]
+            qq = np.stack([_f64(q[b, rows[r][1], rows[r][2], :]) for r in sel])
+            s = (qq @ kk[:jmax].T) * scale
+            if causal:
+                s = np.where(np.arange(jmax)[None, :] <= ii[:, None], s, -np.inf)
+            m = s.max(axis=1, keepdims=True)
+            e = np.exp(s - m)
+            tot = e.sum(axis=1, keepdims=True)
+            lse[sel] = (m + np.log(tot))[:, 0]
+            out[sel] = (e / tot) @ vv[:jmax]
     return out, lse

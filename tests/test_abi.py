@@ -1,0 +1,122 @@
+"""The C-ABI library: loads, exports every symbol include/ra.h declares, and
+rejects invalid arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ra.h")
+
+
+@pytest.fixture(scope="module")
+def ra():
+    from blockwise_exact_attention_block_b200 import build
+    build.build()
+    import blockwise_exact_attention_block_b200 as mod
+    return mod
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ra_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ["ra_block_attn", "ra_merge_partial", "ra_ring_attention", "ra_ring_attention_workspace",
+              "ra_zigzag_permute", "ra_get_device_status", "ra_status_string"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(ra):
+    out = subprocess.run(["nm", "-D", "--defined-only", ra.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (ra_\w+)", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    assert set(ra.EXPORTED) <= exported
+
+
+def test_status_strings(ra):
+    assert ra.ra_status_string(0) == "RA_OK"
+    assert ra.ra_status_string(3) == "RA_ERR_WORKSPACE"
+    assert ra.ra_status_string(99) == "RA_ERR_UNKNOWN"
+    assert "sm_100a" in ra.ra_version()
+
+
+FAKE = 1 << 20  # an aligned, non-null address; never dereferenced on these paths
+
+
+def ring(ra, **kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, in_dtype=ra.RA_BF16, B=1, S=4096, Hq=8, D=128, n=4, causal=1,
+                part=ra.RA_PART_ZIGZAG, groups=1, out=FAKE, out_dtype=ra.RA_F32, lse=FAKE, ws=FAKE,
+                ws_bytes=1 << 40, opts=None, stream=None)
+    args.update(kw)
+    return ra._lib.ra_ring_attention(args["q"], args["k"], args["v"], args["in_dtype"], args["B"], args["S"],
+                                     args["Hq"], args["D"], args["n"], args["causal"], args["part"],
+                                     args["groups"], args["out"], args["out_dtype"], args["lse"], args["ws"],
+                                     args["ws_bytes"], args["opts"], args["stream"])
+
+
+def test_ring_attention_rejects_bad_arguments(ra):
+    E = ra
+    assert ring(ra, S=4100) == E.RA_ERR_INVALID_ARG            # S % (2n) != 0 under zigzag
+    assert ring(ra, S=4099, part=ra.RA_PART_CONTIGUOUS) == E.RA_ERR_INVALID_ARG
+    assert ring(ra, groups=3) == E.RA_ERR_INVALID_ARG          # Hq % groups != 0
+    assert ring(ra, D=96) == E.RA_ERR_UNSUPPORTED
+    assert ring(ra, n=17) == E.RA_ERR_UNSUPPORTED
+    assert ring(ra, n=0) == E.RA_ERR_INVALID_ARG
+    assert ring(ra, q=None) == E.RA_ERR_INVALID_ARG
+    assert ring(ra, out=FAKE + 4) == E.RA_ERR_INVALID_ARG      # misaligned
+    assert ring(ra, in_dtype=7) == E.RA_ERR_INVALID_ARG
+    assert ring(ra, part=5) == E.RA_ERR_INVALID_ARG
+    assert ring(ra, ws=None) == E.RA_ERR_WORKSPACE
+    assert ring(ra, ws_bytes=16) == E.RA_ERR_WORKSPACE
+    bad = ra.ra_options(9, 0, None, None)
+    assert ring(ra, opts=ctypes.byref(bad)) == E.RA_ERR_INVALID_ARG
+
+
+def test_block_attn_rejects_bad_arguments(ra):
+    f = ra._lib.ra_block_attn
+    ok = dict(q=FAKE, k=FAKE, v=FAKE, dt=ra.RA_BF16, B=1, S=1024, n=4, qb=0, kb=0, Hq=4, Hkv=2, D=128, causal=1,
+              part=ra.RA_PART_ZIGZAG, bo=FAKE, bl=FAKE)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["q"], a["k"], a["v"], a["dt"], a["B"], a["S"], a["n"], a["qb"], a["kb"], a["Hq"], a["Hkv"],
+                 a["D"], a["causal"], a["part"], a["bo"], a["bl"], None)
+
+    assert call(dt=ra.RA_F32) == ra.RA_ERR_UNSUPPORTED
+    assert call(qb=4) == ra.RA_ERR_INVALID_ARG
+    assert call(kb=-1) == ra.RA_ERR_INVALID_ARG
+    assert call(Hkv=3) == ra.RA_ERR_INVALID_ARG
+    assert call(bo=None) == ra.RA_ERR_INVALID_ARG
+    assert call(S=1028) == ra.RA_ERR_INVALID_ARG
+
+
+def test_merge_and_permute_reject_bad_arguments(ra):
+    m = ra._lib.ra_merge_partial
+    assert m(FAKE, FAKE, FAKE, FAKE, -1, 128, None) == ra.RA_ERR_INVALID_ARG
+    assert m(FAKE, FAKE, FAKE, FAKE, 0, 128, None) == ra.RA_OK          # empty: no-op
+    assert m(FAKE, FAKE, FAKE, FAKE, 10, 6, None) == ra.RA_ERR_UNSUPPORTED
+    assert m(FAKE + 8, FAKE, FAKE, FAKE, 10, 128, None) == ra.RA_ERR_INVALID_ARG
+    p = ra._lib.ra_zigzag_permute
+    assert p(FAKE, FAKE + (1 << 30), 1, 100, 2, 8, 2, 3, 0, None) == ra.RA_ERR_INVALID_ARG  # 100 % 6
+    assert p(FAKE, FAKE, 1, 96, 2, 8, 2, 3, 0, None) == ra.RA_ERR_INVALID_ARG               # in place
+    assert p(FAKE, FAKE + 64, 1, 96, 2, 8, 2, 3, 0, None) == ra.RA_ERR_INVALID_ARG          # overlap
+    assert p(FAKE, FAKE + (1 << 30), 1, 96, 2, 8, 3, 3, 0, None) == ra.RA_ERR_INVALID_ARG   # elem bytes
+
+
+def test_workspace_query(ra):
+    n = ra.ra_ring_attention_workspace(1, 24000, 32, 128, 4, 4, "zigzag")
+    # permuted bf16 copies of Q (32 heads) and K, V (8 heads each)
+    assert n >= 24000 * (32 + 8 + 8) * 128 * 2
+    assert ra.ra_ring_attention_workspace(1, 4096, 8, 128, 4, 1, "contiguous") == 0
+    n_unf = ra.ra_ring_attention_workspace(1, 4096, 8, 128, 4, 1, "contiguous", sched="unfused")
+    assert n_unf >= 2 * 4096 * 8 * (128 + 1) * 4
+    with pytest.raises(ra.RAError):
+        ra.ra_ring_attention_workspace(1, 4095, 8, 128, 4, 1, "zigzag")

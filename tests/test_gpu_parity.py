@@ -1,0 +1,242 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU fp64 oracle on
+the same seeded inputs.
+
+Tolerances (fixed for this method): bf16 attention inputs -> max-abs error
+<= 2e-2 and relative L2 error <= 1e-2, on out and on lse separately; the fp32
+merge kernels -> max-abs <= 1e-5 on out and |err| <= 1e-5 * max(1, |lse|) on
+lse, against the fp64 rule applied to the same fp32 partials; the zigzag
+permutation -> bit-exact.  Workloads too large for the full oracle are checked
+on sampled query rows, each computed exactly against every key it may see.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as F
+from oracle import blockwise as K
+from seeded_inputs import WORKLOADS, attention_inputs, merge_inputs, workload_inputs
+
+pytestmark = pytest.mark.gpu
+
+ATOL, RTOL_L2 = 2e-2, 1e-2
+MERGE_TOL = 1e-5
+
+
+def assert_close_bf16(got, ref, what):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    gi, ri = np.isneginf(got), np.isneginf(ref)
+    assert np.array_equal(gi, ri), f"{what}: -inf pattern differs"
+    fin = ~ri
+    if not fin.any():
+        return
+    err = np.abs(got[fin] - ref[fin])
+    mx = float(err.max())
+    rel = float(np.linalg.norm(got[fin] - ref[fin]) / max(np.linalg.norm(ref[fin]), 1e-30))
+    assert mx <= ATOL, f"{what}: max-abs {mx:.3e} > {ATOL}"
+    assert rel <= RTOL_L2, f"{what}: rel-L2 {rel:.3e} > {RTOL_L2}"
+
+
+def to_np(t):
+    return t.detach().float().cpu().numpy()
+
+
+# -------------------------------------------------------------- permutation
+
+@pytest.mark.parametrize("shape,n,dtype", [((1, 8, 1, 8), 2, torch.float32), ((2, 4096, 8, 128), 4, torch.bfloat16),
+                                           ((1, 24000, 4, 128), 4, torch.bfloat16), ((3, 96, 3, 2), 6, torch.float32),
+                                           ((1, 96, 3, 2), 3, torch.bfloat16)])
+def test_zigzag_permute_bit_exact(cuda_lib, shape, n, dtype):
+    ra = cuda_lib
+    g = torch.Generator().manual_seed(0)
+    x = torch.randn(shape, generator=g).to(dtype)
+    perm = K.zigzag_perm(shape[1], n)
+    d = ra.ra_zigzag_permute(x.cuda(), n, inverse=False)
+    ref = x[:, torch.from_numpy(perm)]
+    assert torch.equal(d.cpu(), ref)
+    back = ra.ra_zigzag_permute(d, n, inverse=True)
+    assert torch.equal(back.cpu(), x)
+
+
+# ---------------------------------------------------------------- merge rule
+
+def check_merge(got_o, got_l, ref_o, ref_l):
+    go, gl = to_np(got_o).astype(np.float64), to_np(got_l).astype(np.float64)
+    assert np.array_equal(np.isneginf(gl), np.isneginf(ref_l))
+    assert float(np.max(np.abs(go - ref_o))) <= MERGE_TOL
+    fin = np.isfinite(ref_l)
+    assert np.all(np.abs(gl[fin] - ref_l[fin]) <= MERGE_TOL * np.maximum(1.0, np.abs(ref_l[fin])))
+
+
+@pytest.mark.parametrize("T", [4096, 65536])
+def test_merge_partial_matches_oracle(cuda_lib, T):
+    ra = cuda_lib
+    outs, lses = merge_inputs(T, 2)
+    # empty partials on a few rows: the rule's -inf cases
+    lses[1][0, :4] = float("-inf")
+    lses[0][1, :4] = float("-inf")
+    lses[0][2, :2] = float("-inf")
+    lses[1][2, :2] = float("-inf")
+    ref_o, ref_l = K.merge_rule(outs[0].double().numpy(), lses[0].double().numpy(), outs[1].double().numpy(),
+                                lses[1].double().numpy())
+    o, l = outs[0].cuda(), lses[0].cuda()
+    ra.ra_merge_partial(o, l, outs[1].cuda(), lses[1].cuda())
+    check_merge(o, l, ref_o, ref_l)
+
+
+@pytest.mark.parametrize("k", [2, 4, 8, 16])
+def test_merge_partials_matches_oracle(cuda_lib, k):
+    ra = cuda_lib
+    outs, lses = merge_inputs(4096, k, seed=k)
+    ref_o, ref_l = K.merge_partials([o.double().numpy() for o in outs], [l.double().numpy() for l in lses])
+    go, gl = ra.ra_merge_partials([o.cuda() for o in outs], [l.cuda() for l in lses])
+    check_merge(go, gl, ref_o, ref_l)
+    # pairwise launches, folded left to right, give the same answer
+    o, l = outs[0].cuda(), lses[0].cuda()
+    for j in range(1, k):
+        ra.ra_merge_partial(o, l, outs[j].cuda(), lses[j].cuda())
+    check_merge(o, l, ref_o, ref_l)
+
+
+# ----------------------------------------------------------- block attention
+
+BLOCK_CASES = [
+    # B, S, n, Hq, Hkv, D, causal, partition
+    (2, 1200, 4, 4, 2, 128, True, "zigzag"),       # L=300: ragged tail, chunk (150) straddles a tile
+    (1, 1024, 4, 2, 2, 64, True, "contiguous"),
+    (1, 768, 2, 2, 1, 128, False, "contiguous"),
+]
+
+
+@pytest.mark.parametrize("case", BLOCK_CASES, ids=lambda c: f"B{c[0]}S{c[1]}n{c[2]}H{c[3]}/{c[4]}D{c[5]}{c[7]}{'C' if c[6] else ''}")
+def test_block_attn_every_pair(cuda_lib, case):
+    ra = cuda_lib
+    B, S, n, Hq, Hkv, D, causal, part = case
+    q, k, v = attention_inputs(B, S, Hq, Hkv, D, "bf16", seed=3)
+    perm = K.partition_perm(S, n, part)
+    L = S // n
+    pos = perm.reshape(n, L)
+    pt = torch.from_numpy(perm)
+    qp, kp, vp = q[:, pt], k[:, pt], v[:, pt]
+    for qb in range(n):
+        qblk = qp[:, qb * L:(qb + 1) * L].contiguous()
+        for kb in range(n):
+            kblk = kp[:, kb * L:(kb + 1) * L].contiguous()
+            vblk = vp[:, kb * L:(kb + 1) * L].contiguous()
+            bo, bl = ra.ra_block_attn(qblk.cuda(), kblk.cuda(), vblk.cuda(), S, n, qb, kb, causal, part)
+            ro, rl = K.block_partial(qblk, kblk, vblk, pos[qb], pos[kb], causal, Hq // Hkv)
+            assert_close_bf16(to_np(bo), ro, f"block_out q{qb} kv{kb}")
+            assert_close_bf16(to_np(bl), rl, f"block_lse q{qb} kv{kb}")
+
+
+# ----------------------------------------------------------- whole method
+
+SCHEDS = ["persistent", "fused", "unfused"]
+
+
+@pytest.mark.parametrize("order", ["ring", "tokenring"])
+@pytest.mark.parametrize("sched", SCHEDS)
+@pytest.mark.parametrize("case", [(2, 1200, 4, 4, 2, 128, True, "zigzag"), (1, 1024, 4, 2, 1, 64, True, "contiguous"),
+                                  (1, 640, 5, 2, 2, 128, False, "zigzag")],
+                         ids=lambda c: f"B{c[0]}S{c[1]}n{c[2]}D{c[5]}{c[7]}{'C' if c[6] else ''}")
+def test_ring_attention_matches_full_oracle(cuda_lib, case, sched, order):
+    ra = cuda_lib
+    B, S, n, Hq, Hkv, D, causal, part = case
+    q, k, v = attention_inputs(B, S, Hq, Hkv, D, "bf16", seed=4)
+    ro, rl = F.full_attention(q, k, v, causal, Hq // Hkv)
+    for out_dtype in (torch.float32, torch.bfloat16):
+        o, l = ra.ra_ring_attention(q.cuda(), k.cuda(), v.cuda(), n, causal, part, out_dtype=out_dtype,
+                                    order=order, sched=sched)
+        assert_close_bf16(to_np(o), ro, f"out {sched}/{order}/{out_dtype}")
+        assert_close_bf16(to_np(l), rl, f"lse {sched}/{order}/{out_dtype}")
+    assert ra.ra_get_device_status() == 0
+
+
+def test_tiny_workload(cuda_lib):
+    # fp32 inputs: the library rounds them to bf16 on entry; the attention is
+    # judged against the oracle on the same rounded values.
+    ra = cuda_lib
+    w = WORKLOADS["tiny"]
+    q, k, v = workload_inputs(w)
+    qr, kr, vr = (x.to(torch.bfloat16) for x in (q, k, v))
+    ro, rl = F.full_attention(qr, kr, vr, w.causal, w.gqa_groups)
+    for sched in SCHEDS:
+        o, l = ra.ra_ring_attention(q.cuda(), k.cuda(), v.cuda(), w.n_blocks, w.causal, w.partition, sched=sched)
+        assert_close_bf16(to_np(o), ro, f"tiny out {sched}")
+        assert_close_bf16(to_np(l), rl, f"tiny lse {sched}")
+
+
+@pytest.fixture(scope="module")
+def zigzag4k():
+    w = WORKLOADS["zigzag4k"]
+    q, k, v = workload_inputs(w)
+    ro, rl = F.full_attention(q, k, v, w.causal, w.gqa_groups)
+    return w, (q, k, v), (ro, rl)
+
+
+@pytest.mark.parametrize("sched", SCHEDS)
+@pytest.mark.parametrize("order", ["ring", "tokenring"])
+def test_zigzag4k_workload_full_oracle(cuda_lib, zigzag4k, sched, order):
+    ra = cuda_lib
+    w, (q, k, v), (ro, rl) = zigzag4k
+    o, l = ra.ra_ring_attention(q.cuda(), k.cuda(), v.cuda(), w.n_blocks, w.causal, w.partition, sched=sched,
+                                order=order)
+    assert_close_bf16(to_np(o), ro, "zigzag4k out")
+    assert_close_bf16(to_np(l), rl, "zigzag4k lse")
+
+
+def sample_rows(w, per_head=64, seed=0):
+    """Seeded random rows plus the first / last row of every zigzag chunk and
+    rows on 128-row tile boundaries of the blocks."""
+    rng = np.random.default_rng(seed)
+    perm = K.partition_perm(w.S, w.n_blocks, w.partition)
+    L = w.S // w.n_blocks
+    special = set()
+    c = w.S // (2 * w.n_blocks)
+    for ch in range(2 * w.n_blocks):
+        special.update([ch * c, ch * c + c - 1])
+    for r in rng.choice(w.n_blocks, size=min(4, w.n_blocks), replace=False):
+        for t in rng.choice(np.arange(128, L, 128), size=min(4, (L - 1) // 128), replace=False):
+            special.update([int(perm[r * L + t]), int(perm[r * L + t - 1])])
+    special.update([0, w.S - 1])
+    rows = []
+    for b in range(w.B):
+        for h in range(w.Hq):
+            pick = set(int(x) for x in rng.integers(0, w.S, per_head)) | special
+            rows.extend((b, i, h) for i in sorted(pick))
+    return rows
+
+
+def check_sampled(w, q, k, v, o, l, rows, what):
+    ro, rl = F.attention_rows(q, k, v, rows, w.causal, w.gqa_groups)
+    bi = torch.tensor([r[0] for r in rows])
+    ii = torch.tensor([r[1] for r in rows])
+    hi = torch.tensor([r[2] for r in rows])
+    go = o.float().cpu()[bi, ii, hi].numpy()
+    gl = l.cpu()[bi, ii, hi].numpy()
+    assert_close_bf16(go, ro, what + " out")
+    assert_close_bf16(gl, rl, what + " lse")
+
+
+@pytest.mark.parametrize("sched", SCHEDS)
+def test_gqa24k_workload_sampled_rows(cuda_lib, sched):
+    ra = cuda_lib
+    w = WORKLOADS["gqa24k"]
+    q, k, v = workload_inputs(w)
+    o, l = ra.ra_ring_attention(q.cuda(), k.cuda(), v.cuda(), w.n_blocks, w.causal, w.partition,
+                                out_dtype=torch.float32, sched=sched)
+    rows = sample_rows(w, per_head=16 if sched != "persistent" else 64)
+    check_sampled(w, q, k, v, o, l, rows, f"gqa24k {sched}")
+    assert ra.ra_get_device_status() == 0
+
+
+def test_long1m_workload_sampled_rows(cuda_lib):
+    ra = cuda_lib
+    w = WORKLOADS["long1m"]
+    q, k, v = workload_inputs(w)
+    o, l = ra.ra_ring_attention(q.cuda(), k.cuda(), v.cuda(), w.n_blocks, w.causal, w.partition,
+                                out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    rows = sample_rows(w, per_head=24)
+    check_sampled(w, q, k, v, o, l, rows, "long1m")
+    assert ra.ra_get_device_status() == 0
