@@ -166,13 +166,14 @@ class Clocks:
 # ---------------------------------------------------------------- our arm
 
 def launches_per_step(w, sched):
-    copy_inputs = w.partition == "zigzag" or w.in_dtype == "f32"
-    k = 3 if copy_inputs else 0
+    """Kernels of ours launched by one ra_ring_attention call."""
+    cast = 3 if w.in_dtype == "f32" else 0
     if sched in ("auto", "persistent"):
-        return k + 1
+        return cast + 1
+    out_cast = 1 if w.out_dtype == "bf16" else 0
     if sched == "fused":
-        return k + w.n_blocks + 2
-    return k + w.n_blocks + (w.n_blocks - 1) + 2
+        return cast + w.n_blocks + out_cast
+    return cast + w.n_blocks + (w.n_blocks - 1) + out_cast
 
 
 def run_ours(args):
@@ -199,7 +200,7 @@ def run_ours(args):
     out = torch.empty((w.B, w.S, w.Hq, w.D), dtype=odt, device=dev)
     lse = torch.empty((w.B, w.S, w.Hq), dtype=torch.float32, device=dev)
     need = ra.ra_ring_attention_workspace(w.B, w.S, w.Hq, w.D, w.n_blocks, w.gqa_groups, w.partition, q.dtype,
-                                          args.order, args.sched)
+                                          args.order, args.sched, odt)
     ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size

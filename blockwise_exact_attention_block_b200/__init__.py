@@ -58,7 +58,7 @@ _lib.ra_merge_partials.restype = _i
 _lib.ra_ring_attention.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _sz,
                                    ctypes.POINTER(ra_options), _vp]
 _lib.ra_ring_attention.restype = _i
-_lib.ra_ring_attention_workspace.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(ra_options)]
+_lib.ra_ring_attention_workspace.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(ra_options)]
 _lib.ra_ring_attention_workspace.restype = _sz
 _lib.ra_zigzag_permute.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
 _lib.ra_zigzag_permute.restype = _i
@@ -164,10 +164,11 @@ def ra_merge_partials(outs, lses, out=None, lse=None, stream=None):
 
 
 def ra_ring_attention_workspace(B, S, Hq, D, n_blocks, gqa_groups, partition="contiguous",
-                                in_dtype=torch.bfloat16, order="ring", sched="auto") -> int:
+                                in_dtype=torch.bfloat16, order="ring", sched="auto",
+                                out_dtype=torch.float32) -> int:
     o = _opts(order, sched)
     n = _lib.ra_ring_attention_workspace(B, S, Hq, D, n_blocks, gqa_groups, PARTITIONS[partition],
-                                         _dtype_code(in_dtype), ctypes.byref(o))
+                                         _dtype_code(in_dtype), _dtype_code(out_dtype), ctypes.byref(o))
     if n == ctypes.c_size_t(-1).value:
         raise RAError(RA_ERR_INVALID_ARG, "ra_ring_attention_workspace")
     return n
@@ -189,7 +190,8 @@ def ra_ring_attention(q, k, v, n_blocks: int, causal: bool, partition: str = "co
         out = torch.empty((B, S, Hq, D), dtype=out_dtype, device=q.device)
     if lse is None:
         lse = torch.empty((B, S, Hq), dtype=torch.float32, device=q.device)
-    need = ra_ring_attention_workspace(B, S, Hq, D, n_blocks, gqa_groups, partition, q.dtype, order, sched)
+    need = ra_ring_attention_workspace(B, S, Hq, D, n_blocks, gqa_groups, partition, q.dtype, order, sched,
+                                       out.dtype)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0

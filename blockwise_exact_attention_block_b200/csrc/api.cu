@@ -43,7 +43,8 @@ EncodeTiledFn encode_fn() {
 }
 
 // bf16 tensor viewed as [NB][L][H][D] (innermost last), box = 128 rows x 64
-// columns of one head, 128-byte swizzle.  Rows beyond L read as zero.
+// columns of one head, 128-byte swizzle.  Rows beyond L read as zero.  The
+// 4th coordinate is the batch index.
 bool make_map(CUtensorMap* m, const void* ptr, int D, int H, int L, int NB) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
@@ -104,17 +105,48 @@ AttnArgs base_args(const Geom& g) {
   memset(&a, 0, sizeof(a));
   a.B = g.B;
   a.S = g.S;
-  a.n = g.n;
-  a.L = g.L;
-  a.c = g.c;
   a.Hq = g.Hq;
   a.Hkv = g.Hkv;
   a.groups = g.groups;
-  a.zigzag = g.zigzag;
   a.causal = g.causal;
-  a.tiles_per_block = (g.L + kBM - 1) / kBM;
+  a.nseg = g.zigzag ? 2 : 1;
+  const int seg_len = g.zigzag ? g.c : g.L;
+  a.seg_tiles = (seg_len + kCtaRows - 1) / kCtaRows;
   a.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(g.D)));
   return a;
+}
+
+// Segments of block r: original positions, stored at the same rows (tensor
+// in original order) or at block-local rows 0.. (tensor holding block r only).
+void block_segments(const Geom& g, int r, bool block_local, Seg out[2]) {
+  if (!g.zigzag) {
+    out[0].pos = r * g.L;
+    out[0].len = g.L;
+    out[0].mem = block_local ? 0 : out[0].pos;
+    return;
+  }
+  out[0].pos = r * g.c;
+  out[1].pos = (2 * g.n - 1 - r) * g.c;
+  out[0].len = out[1].len = g.c;
+  out[0].mem = block_local ? 0 : out[0].pos;
+  out[1].mem = block_local ? g.c : out[1].pos;
+}
+
+// Query segments of the launch, heaviest (latest positions) first when causal.
+void order_segments(AttnArgs& a) {
+  const int m = a.nq * a.nseg;
+  for (int i = 0; i < m; ++i) a.seg_order[i] = static_cast<signed char>(i);
+  if (!a.causal) return;
+  for (int i = 1; i < m; ++i)
+    for (int j = i; j > 0; --j) {
+      const Seg& x = a.qseg[a.seg_order[j] / a.nseg][a.seg_order[j] % a.nseg];
+      const Seg& y = a.qseg[a.seg_order[j - 1] / a.nseg][a.seg_order[j - 1] % a.nseg];
+      if (x.pos > y.pos) {
+        const signed char t = a.seg_order[j];
+        a.seg_order[j] = a.seg_order[j - 1];
+        a.seg_order[j - 1] = t;
+      }
+    }
 }
 
 template <int D>
@@ -131,7 +163,7 @@ ra_status launch_attn_t(const AttnArgs& a, const CUtensorMap& mq, const CUtensor
     if (e != cudaSuccess) return RA_ERR_CUDA;
     attr_set[dev] = 1;
   }
-  const long long grid = static_cast<long long>(a.Hq) * a.B * a.nq * a.tiles_per_block;
+  const long long grid = static_cast<long long>(a.Hq) * a.B * a.nq * a.nseg * a.seg_tiles;
   if (grid <= 0) return RA_OK;
   if (grid > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
   attn_fwd_kernel<D, NST><<<static_cast<unsigned>(grid), kAttnThreads, SL::kBytes, st>>>(mq, mk, mv, a);
@@ -186,32 +218,27 @@ ra_status launch_permute_bytes(const void* src, void* dst, int B, const PermGeom
   return cuda_status(cudaGetLastError());
 }
 
-PermGeom perm_geom(const Geom& g) {
-  PermGeom p;
-  p.S = g.S;
-  p.L = g.L;
-  p.c = g.c;
-  p.n = g.n;
-  p.zigzag = g.zigzag;
-  return p;
-}
-
-// Workspace plan of ra_ring_attention; offsets in bytes.
+// Workspace plan of ra_ring_attention; offsets in bytes.  The partition
+// itself needs no copy (it is applied through the TMA coordinates); the
+// workspace holds only the bf16 rounding of fp32 inputs, the fp32 running
+// output when the output itself is bf16 (unfused / epilogue-fused), and the
+// per-step partials of the unfused schedule.
 struct Plan {
   ra_sched sched;
-  bool copy_inputs;
-  size_t q, k, v, acc_out, acc_lse, part_out, part_lse, total;
+  bool cast_inputs;
+  bool acc_in_ws;
+  size_t q, k, v, acc_out, part_out, part_lse, total;
 };
 
-Plan make_plan(const Geom& g, ra_dtype in_dtype, const ra_options* opts) {
+Plan make_plan(const Geom& g, ra_dtype in_dtype, ra_dtype out_dtype, const ra_options* opts) {
   Plan p;
   memset(&p, 0, sizeof(p));
   p.sched = opts ? opts->sched : RA_SCHED_AUTO;
   if (p.sched == RA_SCHED_AUTO) p.sched = RA_SCHED_PERSISTENT;
-  p.copy_inputs = g.zigzag || in_dtype == RA_F32;
+  p.cast_inputs = in_dtype == RA_F32;
   const size_t rows = static_cast<size_t>(g.B) * g.S;
   size_t off = 0;
-  if (p.copy_inputs) {
+  if (p.cast_inputs) {
     p.q = off;
     off = align256(off + rows * g.Hq * g.D * 2);
     p.k = off;
@@ -220,10 +247,11 @@ Plan make_plan(const Geom& g, ra_dtype in_dtype, const ra_options* opts) {
     off = align256(off + rows * g.Hkv * g.D * 2);
   }
   if (p.sched != RA_SCHED_PERSISTENT) {
-    p.acc_out = off;
-    off = align256(off + rows * g.Hq * g.D * 4);
-    p.acc_lse = off;
-    off = align256(off + rows * g.Hq * 4);
+    p.acc_in_ws = out_dtype != RA_F32;
+    if (p.acc_in_ws) {
+      p.acc_out = off;
+      off = align256(off + rows * g.Hq * g.D * 4);
+    }
     if (p.sched == RA_SCHED_UNFUSED) {
       p.part_out = off;
       off = align256(off + rows * g.Hq * g.D * 4);
@@ -293,17 +321,14 @@ ra_status ra_block_attn(const void* q, const void* k, const void* v, ra_dtype in
   AttnArgs a = base_args(g);
   a.nq = 1;
   a.nkv = 1;
-  a.q_blocks[0] = static_cast<signed char>(q_block);
+  block_segments(g, q_block, true, a.qseg[0]);
+  block_segments(g, kv_block, true, a.kvseg[kv_block]);
   a.kv_list[0][0] = static_cast<signed char>(kv_block);
-  a.q_bmul = 1;
-  a.q_rmul = 0;
-  a.kv_bmul = 1;
-  a.kv_rmul = 0;
+  order_segments(a);
   a.mode = kModePartial;
   a.acc_out = block_out;
   a.acc_lse = block_lse;
   a.acc_brows = g.L;
-  a.acc_rmul = 0;
   return launch_attn(D, a, mq, mk, mv, static_cast<cudaStream_t>(stream));
 }
 
@@ -364,13 +389,14 @@ ra_status ra_zigzag_permute(const void* src, void* dst, int B, int S, int H, int
 }
 
 size_t ra_ring_attention_workspace(int B, int S, int Hq, int D, int n_blocks, int gqa_groups, ra_partition partition,
-                                   ra_dtype in_dtype, const ra_options* opts) {
+                                   ra_dtype in_dtype, ra_dtype out_dtype, const ra_options* opts) {
   if (gqa_groups < 1 || Hq % gqa_groups != 0) return static_cast<size_t>(-1);
   Geom g;
   if (check_geom(B, S, n_blocks, Hq, Hq / gqa_groups, D, partition, &g) != RA_OK) return static_cast<size_t>(-1);
   if (in_dtype != RA_F32 && in_dtype != RA_BF16) return static_cast<size_t>(-1);
+  if (out_dtype != RA_F32 && out_dtype != RA_BF16) return static_cast<size_t>(-1);
   if (!valid_opts(opts)) return static_cast<size_t>(-1);
-  return make_plan(g, in_dtype, opts).total;
+  return make_plan(g, in_dtype, out_dtype, opts).total;
 }
 
 ra_status ra_ring_attention(const void* q, const void* k, const void* v, ra_dtype in_dtype, int B, int S, int Hq,
@@ -388,32 +414,32 @@ ra_status ra_ring_attention(const void* q, const void* k, const void* v, ra_dtyp
   if (!q || !k || !v || !out || !lse) return RA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
     return RA_ERR_INVALID_ARG;
-  const Plan p = make_plan(g, in_dtype, opts);
+  const Plan p = make_plan(g, in_dtype, out_dtype, opts);
   if (p.total > 0) {
     if (!workspace || workspace_bytes < p.total) return RA_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255) return RA_ERR_INVALID_ARG;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
-  const PermGeom pg = perm_geom(g);
   const ra_order order = opts ? opts->order : RA_ORDER_RING;
+  PermGeom ident;
+  memset(&ident, 0, sizeof(ident));
+  ident.S = S;
+  ident.L = g.L;
+  ident.n = g.n;
 
-  // a2: partition (and fp32 -> bf16 rounding) of the inputs into block order
+  // fp32 inputs are rounded to bf16 (nearest even) once, in original order
   const void* qb = q;
   const void* kb = k;
   const void* vb = v;
-  if (p.copy_inputs) {
+  if (p.cast_inputs) {
     struct { const void* src; size_t off; int H; } mv[3] = {{q, p.q, g.Hq}, {k, p.k, g.Hkv}, {v, p.v, g.Hkv}};
     for (auto& m : mv) {
       const long long row_elems = static_cast<long long>(m.H) * D;
-      if (in_dtype == RA_BF16) {
-        s = launch_permute_bytes(m.src, ws + m.off, B, pg, row_elems * 2, 0, st);
-      } else {
-        const long long rows = static_cast<long long>(B) * S;
-        permute_cast_kernel<float, __nv_bfloat16><<<grid_for(rows * row_elems / 8, 256), 256, 0, st>>>(
-            static_cast<const float*>(m.src), reinterpret_cast<__nv_bfloat16*>(ws + m.off), B, pg, row_elems, 0);
-        s = cuda_status(cudaGetLastError());
-      }
+      const long long rows = static_cast<long long>(B) * S;
+      permute_cast_kernel<float, __nv_bfloat16><<<grid_for(rows * row_elems / 8, 256), 256, 0, st>>>(
+          static_cast<const float*>(m.src), reinterpret_cast<__nv_bfloat16*>(ws + m.off), B, ident, row_elems, 0);
+      s = cuda_status(cudaGetLastError());
       if (s != RA_OK) return s;
     }
     qb = ws + p.q;
@@ -421,9 +447,9 @@ ra_status ra_ring_attention(const void* q, const void* k, const void* v, ra_dtyp
     vb = ws + p.v;
   }
 
+  // a2: the partition, as TMA coordinates into the tensors in original order
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, qb, D, g.Hq, g.L, B * g.n) || !make_map(&mk, kb, D, g.Hkv, g.L, B * g.n) ||
-      !make_map(&mv, vb, D, g.Hkv, g.L, B * g.n))
+  if (!make_map(&mq, qb, D, g.Hq, S, B) || !make_map(&mk, kb, D, g.Hkv, S, B) || !make_map(&mv, vb, D, g.Hkv, S, B))
     return RA_ERR_CUDA;
 
   // a7: the order in which each query block meets the KV blocks
@@ -434,11 +460,11 @@ ra_status ra_ring_attention(const void* q, const void* k, const void* v, ra_dtyp
 
   AttnArgs a = base_args(g);
   a.nq = g.n;
-  for (int r = 0; r < g.n; ++r) a.q_blocks[r] = static_cast<signed char>(r);
-  a.q_bmul = g.n;
-  a.q_rmul = 1;
-  a.kv_bmul = g.n;
-  a.kv_rmul = 1;
+  for (int r = 0; r < g.n; ++r) {
+    block_segments(g, r, false, a.qseg[r]);
+    block_segments(g, r, false, a.kvseg[r]);
+  }
+  order_segments(a);
 
   if (p.sched == RA_SCHED_PERSISTENT) {
     // a3-a6 in one launch: the running state is carried across block boundaries
@@ -455,12 +481,13 @@ ra_status ra_ring_attention(const void* q, const void* k, const void* v, ra_dtyp
     return s;
   }
 
-  float* acc_out = reinterpret_cast<float*>(ws + p.acc_out);
-  float* acc_lse = reinterpret_cast<float*>(ws + p.acc_lse);
+  // unfused / epilogue-fused: one launch per ring step over all n pairs of
+  // the step; the running (out, lse) is kept in fp32, in original order
+  float* acc_out = p.acc_in_ws ? reinterpret_cast<float*>(ws + p.acc_out) : static_cast<float*>(out);
+  float* acc_lse = lse;
   const long long rows = static_cast<long long>(B) * S * g.Hq;
   a.nkv = 1;
   a.acc_brows = S;
-  a.acc_rmul = 1;
   if (opts && opts->attn_event_begin) cudaEventRecord(static_cast<cudaEvent_t>(opts->attn_event_begin), st);
   for (int step = 0; step < g.n; ++step) {
     for (int r = 0; r < g.n; ++r) a.kv_list[r][0] = static_cast<signed char>(kv_order[r][step]);
@@ -485,17 +512,14 @@ ra_status ra_ring_attention(const void* q, const void* k, const void* v, ra_dtyp
     }
   }
   if (opts && opts->attn_event_end) cudaEventRecord(static_cast<cudaEvent_t>(opts->attn_event_end), st);
-  // a8: back to original token order, with the cast of out
-  const long long row_elems = static_cast<long long>(g.Hq) * D;
-  if (out_dtype == RA_BF16) {
+  // a8: the cast of out (fp32 -> bf16, nearest even); lse is already in place
+  if (p.acc_in_ws) {
+    const long long row_elems = static_cast<long long>(g.Hq) * D;
     permute_cast_kernel<float, __nv_bfloat16><<<grid_for(static_cast<long long>(B) * S * row_elems / 8, 256), 256, 0, st>>>(
-        acc_out, static_cast<__nv_bfloat16*>(out), B, pg, row_elems, 1);
+        acc_out, static_cast<__nv_bfloat16*>(out), B, ident, row_elems, 0);
     s = cuda_status(cudaGetLastError());
-  } else {
-    s = launch_permute_bytes(acc_out, out, B, pg, row_elems * 4, 1, st);
   }
-  if (s != RA_OK) return s;
-  return launch_permute_bytes(acc_lse, lse, B, pg, static_cast<long long>(g.Hq) * 4, 1, st);
+  return s;
 }
 
 }  // extern "C"

@@ -1,8 +1,9 @@
 // attn_fwd.cuh - block attention on the 5th-generation tensor cores (sm_100a).
 //
-// One CTA computes one 128-row query tile of one (batch, query head) against
-// a list of KV blocks (one block for ra_block_attn and the unfused schedule,
-// every block in schedule order for the persistent schedule).
+// One CTA computes 256 consecutive query rows (two 128-row tiles, A and B) of
+// one (batch, query head) against a list of KV blocks (one block for
+// ra_block_attn and the unfused schedule; every block, in schedule order, for
+// the persistent schedule).  Both tiles share every K/V tile load.
 //
 // TokenRing review (pith.science, arXiv 2412.20501), "What carries the
 // argument" / "Core claim": the flash-attention kernel that yields, for one
@@ -10,15 +11,18 @@
 // the per-row block_lse; "If this is right": grouped-query attention and the
 // zigzag causal partition; Anthology of the SOTA, SOTA-181: exact attention.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax: thread i owns query row i of the tile (TMEM lane i).
-//   warp 4     TMA producer: Q once, then K and V tiles into an NST-deep ring.
-//   warp 5     TMEM allocator and MMA issuer (one thread):
-//                S_j  = Q K_j^T       (SS MMA, fp32 into TMEM, two buffers)
-//                O   += P_j V_j       (TS MMA, P_j bf16 in TMEM over S_j)
-// Tensor memory (512 columns): S buffers at columns [0,128) and [128,256);
-// P_j is written as packed bf16 into the first 64 columns of its S buffer;
-// the O accumulator lives at columns [256, 256 + D).
+// Warp roles (320 threads):
+//   warps 0-3  softmax of tile A: thread i owns row i of A (TMEM lane i)
+//   warps 4-7  softmax of tile B (same lanes, its own TMEM columns)
+//   warp 8     TMA producer: Q (A and B) once, then K and V into an NST ring
+//   warp 9     TMEM allocator and MMA issuer (one thread):
+//                S_X = Q_X K^T   (SS MMA, fp32 in TMEM)
+//                O_X += P_X V    (TS MMA, P_X bf16 in TMEM over S_X)
+//              issued in the order PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so
+//              the tensor core works on one tile while the other tile's
+//              softmax runs.
+// Tensor memory (512 columns): S_A/P_A [0,128), S_B/P_B [128,256),
+// O_A [256,256+D), O_B [384,384+D).
 //
 // Online softmax in fp32 with base-2 exponentials (scores pre-scaled by
 // log2(e)/sqrt(D)).  The running maximum used for the exponentials is only
@@ -26,11 +30,14 @@
 // O is rescaled in TMEM rarely; the final out = O / l and
 // lse = ln 2 * (m + log2 l) are exact for any such choice of m.
 //
-// Causal masking uses original token positions.  Inside one block positions
-// increase with the block-local row index (both partitions), so the keys a
-// query may see form a prefix of each KV block: the tile loop stops at the
-// last tile the tile's last row can see, and only tiles cut by a row's prefix
-// are masked element-wise.
+// The partition is an index map, not a data movement: every block is one
+// (contiguous) or two (zigzag) segments of consecutive original positions,
+// and tiles never straddle a segment, so each 128-row tile is one TMA box read
+// straight from the caller's tensor.  Causal masking uses original positions;
+// inside a segment the keys a query may see form a prefix, so the KV loop
+// stops at the last tile the CTA's last row can see, tile A skips the KV tiles
+// none of its rows can see, and only tiles cut by a row's prefix are masked
+// element-wise.
 #pragma once
 
 #include "common.cuh"
@@ -40,9 +47,12 @@
 namespace ra {
 
 constexpr int kBM = 128;        // query rows per tile = TMEM lanes
+constexpr int kCtaRows = 256;   // two tiles per CTA
 constexpr int kBN = 128;        // keys per KV tile
 constexpr int kMaxBlocks = 16;  // ring size limit
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 
 enum AttnMode : int {
   kModePartial = 0,  // write (block_out, block_lse) into acc rows
@@ -50,28 +60,34 @@ enum AttnMode : int {
   kModeFinal = 2     // write (out, lse) at original token positions
 };
 
+// A run of consecutive original positions [pos, pos + len) stored at rows
+// [mem, mem + len) of a tensor.
+struct Seg {
+  int mem, pos, len;
+};
+
 struct AttnArgs {
-  int B, S, n, L, c;      // batch, sequence, ring size, block length, zigzag chunk
+  int B, S;               // batch, full sequence length
   int Hq, Hkv, groups;    // query heads, KV heads, Hq / Hkv
-  int zigzag, causal;
+  int causal;
   int nq;                 // query blocks covered by this launch
   int nkv;                // KV blocks each query block visits in this launch
-  int tiles_per_block;    // ceil(L / 128)
-  int q_bmul, q_rmul;     // TMA 4th coordinate of (batch b, block r) = b*bmul + r*rmul
-  int kv_bmul, kv_rmul;
+  int nseg;               // segments per block: 1 (contiguous) or 2 (zigzag)
+  int seg_tiles;          // ceil(segment length / 256): CTAs per query segment
   float scale_log2;       // log2(e) / sqrt(D)
   int mode;               // AttnMode
-  // kModePartial / kModeMerge: row = b * acc_brows + r * acc_rmul * L + t
+  // kModePartial / kModeMerge: row = b * acc_brows + memory row of the query
   float* acc_out;
   float* acc_lse;
   long long acc_brows;
-  int acc_rmul;
-  // kModeFinal: row = b * S + pos (original order)
+  // kModeFinal: row = b * S + original position of the query
   void* out;
   float* lse;
   int out_bf16;
-  signed char q_blocks[kMaxBlocks];
-  signed char kv_list[kMaxBlocks][kMaxBlocks];  // kv_list[i][s]: s-th KV block of query block i
+  Seg qseg[kMaxBlocks][2];                      // segments of the i-th query block of the launch
+  Seg kvseg[kMaxBlocks][2];                     // segments of KV block r
+  signed char kv_list[kMaxBlocks][kMaxBlocks];  // kv_list[i][s]: s-th KV block met by query block i
+  signed char seg_order[2 * kMaxBlocks];        // (i * nseg + e) of the query segments, heaviest first
 };
 
 template <int D, int NST>
@@ -79,32 +95,28 @@ struct AttnSmem {
   static constexpr int kBox = kBM * 64 * 2;  // one TMA box: 128 rows x 64 bf16 (128 B) = 16 KB
   static constexpr int kNBox = D / 64;
   static constexpr int kTile = kBox * kNBox;
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTile;
+  static constexpr int kQ = 0;                // Q_A, Q_B
+  static constexpr int kK = kQ + 2 * kTile;
   static constexpr int kV = kK + NST * kTile;
   static constexpr int kBar = kV + NST * kTile;
-  // barriers: Q, Kfull[NST], Vfull[NST], Kempty[NST], Vempty[NST], Sfull[2], Pfull[2], Odone, End
-  static constexpr int kNBar = 1 + 4 * NST + 2 + 2 + 1 + 1;
+  // barriers: Q, Kfull[NST], Vfull[NST], Kempty[NST], Vempty[NST], Sfull[2], Pfull[2], Odone[2], End
+  static constexpr int kNBar = 1 + 4 * NST + 2 + 2 + 2 + 1;
   static constexpr int kTmemSlot = kBar + kNBar * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4 + 1024;  // + slack to align the base to 1024
   static_assert(kBytes <= 232448, "shared memory budget");
 };
 
-__device__ __forceinline__ int block_pos(const AttnArgs& a, int r, int t) {
-  if (!a.zigzag) return r * a.L + t;
-  return t < a.c ? r * a.c + t : (2 * a.n - 1 - r) * a.c + (t - a.c);
+// Keys of a KV segment visible to a query at original position qpos: a
+// prefix of the segment.  qpos < 0 marks a padding row.
+__device__ __forceinline__ int visible_count(const AttnArgs& a, const Seg& kv, int qpos) {
+  if (qpos < 0) return 0;
+  if (!a.causal) return kv.len;
+  return min(max(qpos - kv.pos + 1, 0), kv.len);
 }
 
-// Number of keys of KV block kvb visible to a query at original position qpos
-// (they form a prefix of the block).  qpos < 0 marks a padding row.
-__device__ __forceinline__ int visible_count(const AttnArgs& a, int kvb, int qpos) {
-  if (qpos < 0) return 0;
-  if (!a.causal) return a.L;
-  if (!a.zigzag) return min(max(qpos - kvb * a.L + 1, 0), a.L);
-  const int c1 = min(max(qpos - kvb * a.c + 1, 0), a.c);
-  const int c2 = min(max(qpos - (2 * a.n - 1 - kvb) * a.c + 1, 0), a.c);
-  return c1 + c2;
+__device__ __forceinline__ int tiles_for(const AttnArgs& a, const Seg& kv, int qpos) {
+  return (visible_count(a, kv, qpos) + kBN - 1) / kBN;
 }
 
 // Bounded wait that ignores the abort flag, used only to drain work that is
@@ -118,6 +130,11 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
     }
   }
 }
+
+// Position of the CTA's g-th KV tile as (KV block index s, segment e, tile t).
+struct KvCursor {
+  int s, e, t, nt;
+};
 
 template <int D, int NST>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -133,29 +150,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int lane = threadIdx.x & 31;
 
   // ---- tile decode: heads fastest (heads of one KV group share K/V in L2),
-  // heaviest tiles first.
+  // then batch, then query tiles in decreasing position (heaviest first).
   int idx = blockIdx.x;
   const int h = idx % a.Hq;
   idx /= a.Hq;
   const int b = idx % a.B;
   idx /= a.B;
-  int qi, qt;
-  if (a.zigzag) {
-    qt = a.tiles_per_block - 1 - idx / a.nq;
-    qi = a.nq - 1 - idx % a.nq;
-  } else {
-    qi = a.nq - 1 - idx / a.tiles_per_block;
-    qt = a.tiles_per_block - 1 - idx % a.tiles_per_block;
-  }
-  const int r = a.q_blocks[qi];
+  const int so = a.seg_order[idx / a.seg_tiles];
+  const int qt = a.seg_tiles - 1 - idx % a.seg_tiles;
+  const int qi = so / a.nseg;
+  const Seg qs = a.qseg[qi][so % a.nseg];
   const int hk = h / a.groups;
-  const int t0 = qt * kBM;
-  const int q_rows = min(kBM, a.L - t0);
-  const int last_pos = block_pos(a, r, t0 + q_rows - 1);
+  const int t0 = qt * kCtaRows;  // CTA row offset inside the query segment
+  int rows[2], last[2];
+  for (int x = 0; x < 2; ++x) {
+    rows[x] = min(max(qs.len - t0 - x * kBM, 0), kBM);
+    last[x] = rows[x] > 0 ? qs.pos + t0 + x * kBM + rows[x] - 1 : -1;
+  }
+  const int last_u = max(last[0], last[1]);  // the CTA's last row: its KV range covers both tiles
+  auto seg_of = [&](int s_, int e_) -> const Seg& { return a.kvseg[a.kv_list[qi][s_]][e_]; };
 
   int total = 0;
   for (int s = 0; s < a.nkv; ++s)
-    total += (visible_count(a, a.kv_list[qi][s], last_pos) + kBN - 1) / kBN;
+    for (int e = 0; e < a.nseg; ++e) total += tiles_for(a, seg_of(s, e), last_u);
 
   auto bar = [&](int i) -> uint32_t { return sb + SL::kBar + 8u * i; };
   const int BQ = 0;
@@ -163,60 +180,61 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   auto BVF = [&](int s) { return 1 + NST + s; };
   auto BKE = [&](int s) { return 1 + 2 * NST + s; };
   auto BVE = [&](int s) { return 1 + 3 * NST + s; };
-  auto BSF = [&](int i) { return 1 + 4 * NST + i; };
-  auto BPF = [&](int i) { return 3 + 4 * NST + i; };
-  const int BOD = 5 + 4 * NST;
-  const int BEND = 6 + 4 * NST;
+  auto BSF = [&](int x) { return 1 + 4 * NST + x; };
+  auto BPF = [&](int x) { return 3 + 4 * NST + x; };
+  auto BOD = [&](int x) { return 5 + 4 * NST + x; };
+  const int BEND = 7 + 4 * NST;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SL::kAbort);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < SL::kNBar; ++i) mbar_init(bar(i), 1);
-    mbar_init(bar(BPF(0)), 128);
-    mbar_init(bar(BPF(1)), 128);
+    mbar_init(bar(BPF(0)), kBM);
+    mbar_init(bar(BPF(1)), kBM);
     *abort_flag = grid_timed_out() ? 1 : 0;  // after a timeout elsewhere, do no work
     fence_mbar_init();
   }
-  if (warp == 5) tmem_alloc(sb + SL::kTmemSlot, 512);
+  if (warp == kMmaWarp) tmem_alloc(sb + SL::kTmemSlot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + SL::kTmemSlot);
   if (*abort_flag) total = 0;
-  const uint32_t tO = tmem + 256;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && total > 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_expect_tx(bar(BQ), SL::kTile);
-      for (int x = 0; x < SL::kNBox; ++x)
-        tma_load_4d(sb + SL::kQ + x * SL::kBox, &tmQ, x * 64, h, t0, b * a.q_bmul + r * a.q_rmul,
-                    bar(BQ));
+      mbar_expect_tx(bar(BQ), 2 * SL::kTile);
+      for (int x = 0; x < 2; ++x)
+        for (int bx = 0; bx < SL::kNBox; ++bx)
+          tma_load_4d(sb + SL::kQ + x * SL::kTile + bx * SL::kBox, &tmQ, bx * 64, h, qs.mem + t0 + x * kBM, b,
+                      bar(BQ));
       int g = 0;
       bool ok = true;
       int issued_k[NST], issued_v[NST];
       for (int s = 0; s < NST; ++s) issued_k[s] = issued_v[s] = -1;
       for (int s = 0; s < a.nkv && ok; ++s) {
-        const int kvb = a.kv_list[qi][s];
-        const int nt = (visible_count(a, kvb, last_pos) + kBN - 1) / kBN;
-        const int wc = b * a.kv_bmul + kvb * a.kv_rmul;
-        for (int t = 0; t < nt; ++t, ++g) {
-          const int st = g % NST;
-          const uint32_t ph = (g / NST) & 1;
-          if (!mbar_wait(bar(BKE(st)), ph ^ 1, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(bar(BKF(st)), SL::kTile);
-          for (int x = 0; x < SL::kNBox; ++x)
-            tma_load_4d(sb + SL::kK + st * SL::kTile + x * SL::kBox, &tmK, x * 64, hk, t * kBN, wc,
-                        bar(BKF(st)));
-          issued_k[st] = g;
-          if (!mbar_wait(bar(BVE(st)), ph ^ 1, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(bar(BVF(st)), SL::kTile);
-          for (int x = 0; x < SL::kNBox; ++x)
-            tma_load_4d(sb + SL::kV + st * SL::kTile + x * SL::kBox, &tmV, x * 64, hk, t * kBN, wc,
-                        bar(BVF(st)));
-          issued_v[st] = g;
+        for (int e = 0; e < a.nseg && ok; ++e) {
+          const Seg ks = seg_of(s, e);
+          const int nt = tiles_for(a, ks, last_u);
+          for (int t = 0; t < nt; ++t, ++g) {
+            const int st = g % NST;
+            const uint32_t ph = (g / NST) & 1;
+            if (!mbar_wait(bar(BKE(st)), ph ^ 1, abort_flag)) { ok = false; break; }
+            mbar_expect_tx(bar(BKF(st)), SL::kTile);
+            for (int bx = 0; bx < SL::kNBox; ++bx)
+              tma_load_4d(sb + SL::kK + st * SL::kTile + bx * SL::kBox, &tmK, bx * 64, hk, ks.mem + t * kBN, b,
+                          bar(BKF(st)));
+            issued_k[st] = g;
+            if (!mbar_wait(bar(BVE(st)), ph ^ 1, abort_flag)) { ok = false; break; }
+            mbar_expect_tx(bar(BVF(st)), SL::kTile);
+            for (int bx = 0; bx < SL::kNBox; ++bx)
+              tma_load_4d(sb + SL::kV + st * SL::kTile + bx * SL::kBox, &tmV, bx * 64, hk, ks.mem + t * kBN, b,
+                          bar(BVF(st)));
+            issued_v[st] = g;
+          }
         }
       }
       if (!ok) {  // let every copy already issued land before shared memory is released
@@ -227,49 +245,89 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------- MMA issue
     if (lane == 0 && total > 0) {
       constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, D, true);
-      auto issue_s = [&](int g) {
-        const int st = g % NST;
-        const uint32_t dst = tmem + (g & 1) * 128;
+      auto issue_s = [&](int x, int st) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
-          const uint64_t ad = smem_desc_sw128(sb + SL::kQ + off, 16, 1024);
+          const uint64_t ad = smem_desc_sw128(sb + SL::kQ + x * SL::kTile + off, 16, 1024);
           const uint64_t bd = smem_desc_sw128(sb + SL::kK + st * SL::kTile + off, 16, 1024);
-          mma_ss(dst, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + x * 128, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(BSF(g & 1)));
-        tc_commit(bar(BKE(st)));
+        tc_commit(bar(BSF(x)));
       };
+      auto issue_pv = [&](int x, int st, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t bd = smem_desc_sw128(sb + SL::kV + st * SL::kTile + kk * 2048, SL::kBox, 1024);
+          mma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, bd, kIdescO, (acc || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(bar(BOD(x)));
+      };
+      // moves the cursor to the next KV tile that exists
+      auto advance = [&](KvCursor& k) {
+        ++k.t;
+        while (k.t >= k.nt && k.s < a.nkv) {
+          k.t = 0;
+          if (++k.e == a.nseg) {
+            k.e = 0;
+            ++k.s;
+          }
+          k.nt = k.s < a.nkv ? tiles_for(a, seg_of(k.s, k.e), last_u) : 0;
+        }
+      };
+      auto active = [&](const KvCursor& k, int x) { return k.t < tiles_for(a, seg_of(k.s, k.e), last[x]); };
+
+      KvCursor cur = {0, 0, -1, tiles_for(a, seg_of(0, 0), last_u)};
+      advance(cur);  // first existing tile (total > 0, so there is one)
+      bool act[2] = {active(cur, 0), active(cur, 1)};
+      int cnt[2] = {0, 0};  // P V products issued per tile
       bool ok = mbar_wait(bar(BQ), 0, abort_flag);
       if (ok) ok = mbar_wait(bar(BKF(0)), 0, abort_flag);
       if (ok) {
         tc_fence_after();
-        issue_s(0);
+        for (int x = 0; x < 2; ++x)
+          if (act[x]) issue_s(x, 0);
+        tc_commit(bar(BKE(0)));
       }
       for (int g = 0; ok && g < total; ++g) {
-        if (g + 1 < total) {
-          const int st1 = (g + 1) % NST;
-          if (!mbar_wait(bar(BKF(st1)), ((g + 1) / NST) & 1, abort_flag)) break;
-          tc_fence_after();
-          issue_s(g + 1);
-        }
-        if (!mbar_wait(bar(BPF(g & 1)), (g >> 1) & 1, abort_flag)) break;
         const int st = g % NST;
-        if (!mbar_wait(bar(BVF(st)), (g / NST) & 1, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t pcol = tmem + (g & 1) * 128;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bd = smem_desc_sw128(sb + SL::kV + st * SL::kTile + kk * 2048, SL::kBox, 1024);
-          mma_ts(tO, pcol + kk * 8, bd, kIdescO, (g > 0 || kk > 0) ? 1u : 0u);
+        const bool has_next = g + 1 < total;
+        KvCursor nxt = cur;
+        bool act1[2] = {false, false};
+        if (has_next) {
+          advance(nxt);
+          act1[0] = active(nxt, 0);
+          act1[1] = active(nxt, 1);
         }
-        tc_commit(bar(BOD));
+        if (!mbar_wait(bar(BVF(st)), (g / NST) & 1, abort_flag)) break;
+        bool k_ready = false;
+        for (int x = 0; x < 2; ++x) {
+          if (act[x]) {
+            if (!mbar_wait(bar(BPF(x)), cnt[x] & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(x, st, cnt[x] > 0);
+            ++cnt[x];
+          }
+          if (act1[x]) {
+            if (!k_ready) {
+              if (!mbar_wait(bar(BKF((g + 1) % NST)), ((g + 1) / NST) & 1, abort_flag)) { ok = false; break; }
+              tc_fence_after();
+              k_ready = true;
+            }
+            issue_s(x, (g + 1) % NST);
+          }
+        }
+        if (!ok) break;
         tc_commit(bar(BVE(st)));
+        if (has_next) tc_commit(bar(BKE((g + 1) % NST)));
+        cur = nxt;
+        act[0] = act1[0];
+        act[1] = act1[1];
       }
       // nothing may still write tensor memory when it is released
       tc_commit(bar(BEND));
@@ -277,152 +335,160 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else {
     // ------------------------------------------------------------- softmax
-    const int row = threadIdx.x;  // 0..127
-    const int tl = t0 + row;
-    const bool valid = row < q_rows;
-    const int qpos = valid ? block_pos(a, r, tl) : -1;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const int x = warp >> 2;            // tile A (0) or B (1)
+    const int row = threadIdx.x & 127;  // row inside the tile = TMEM lane
+    const bool valid = row < rows[x];
+    const int qpos = valid ? qs.pos + t0 + x * kBM + row : -1;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + x * 128;
+    const uint32_t tO = tmem + lane_base + 256 + x * 128;
     const float sl2 = a.scale_log2;
     float m_use = -INFINITY;
     float l_sum = 0.f;
-    bool ok = true;
-    int g = 0;
-    for (int s = 0; s < a.nkv && ok; ++s) {
-      const int kvb = a.kv_list[qi][s];
-      const int nt = (visible_count(a, kvb, last_pos) + kBN - 1) / kBN;
-      const int lim = visible_count(a, kvb, qpos);
-      for (int t = 0; t < nt; ++t, ++g) {
-        ok = mbar_wait(bar(BSF(g & 1)), (g >> 1) & 1, abort_flag);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t sv[kBN];
-        tmem_ld128_wait(tmem + lane_base + (g & 1) * 128, sv);
-        const int cnt = lim - t * kBN;
-        float mx = -INFINITY;
-        if (cnt < kBN) {
-#pragma unroll
-          for (int c = 0; c < kBN; ++c) {
-            const float x = c < cnt ? __uint_as_float(sv[c]) : -INFINITY;
-            sv[c] = __float_as_uint(x);
-            mx = fmaxf(mx, x);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < kBN; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
-        }
-        const float mt = mx * sl2;
-        float alpha = 1.f;
-        bool resc = false;
-        if (mt > m_use + 8.f) {
-          if (m_use != -INFINITY) {
-            alpha = fast_exp2(m_use - mt);
-            resc = true;
-          }
-          m_use = mt;
-        }
-        const float base = (m_use == -INFINITY) ? 0.f : m_use;
-        float psum = 0.f;
-        uint32_t pk[kBN / 2];
-#pragma unroll
-        for (int c = 0; c < kBN; c += 2) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c]), sl2, -base));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), sl2, -base));
-          psum += p0 + p1;
-          pk[c / 2] = pack_bf16x2(p0, p1);
-        }
-        l_sum = l_sum * alpha + psum;
-        const uint32_t pdst = tmem + lane_base + (g & 1) * 128;
-        tmem_st32(pdst, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(pdst + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
-        tmem_wait_st();
-        if (g > 0) {
-          // O may only be touched once the previous P V product has landed.
-          ok = mbar_wait(bar(BOD), (g - 1) & 1, abort_flag);
+    bool ok = total > 0;
+    int c = 0;  // tiles processed by this tile's softmax
+    for (int s = 0; s < a.nkv && ok; ++s)
+      for (int e = 0; e < a.nseg && ok; ++e) {
+        const Seg ks = seg_of(s, e);
+        const int nt = tiles_for(a, ks, last[x]);  // this tile's prefix of the CTA's tiles
+        const int lim = visible_count(a, ks, qpos);
+        for (int t = 0; t < nt; ++t, ++c) {
+          ok = mbar_wait(bar(BSF(x)), c & 1, abort_flag);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
-          if (__any_sync(0xffffffffu, resc)) {
-            tc_fence_after();
-            uint32_t ov[D];
-            if constexpr (D == 128) tmem_ld128_wait(tO + lane_base, ov);
-            else tmem_ld64_wait(tO + lane_base, ov);
+          tc_fence_after();
+          uint32_t sv[kBN];
+          tmem_ld128_wait(tS, sv);
+          const int cnt = lim - t * kBN;
+          // row maximum with 8 independent chains (short dependency paths)
+          float mx8[8];
 #pragma unroll
-            for (int i = 0; i < D; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+          if (cnt < kBN) {
 #pragma unroll
-            for (int i = 0; i < D / 32; ++i)
-              tmem_st32(tO + lane_base + 32 * i, *reinterpret_cast<const uint32_t(*)[32]>(&ov[32 * i]));
-            tmem_wait_st();
+            for (int j = 0; j < kBN; ++j) {
+              const float v = j < cnt ? __uint_as_float(sv[j]) : -INFINITY;
+              sv[j] = __float_as_uint(v);
+              mx8[j & 7] = fmaxf(mx8[j & 7], v);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < kBN; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], __uint_as_float(sv[j]));
           }
+          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          const float mt = mx * sl2;
+          float alpha = 1.f;
+          bool resc = false;
+          if (mt > m_use + 8.f) {
+            if (m_use != -INFINITY) {
+              alpha = fast_exp2(m_use - mt);
+              resc = true;
+            }
+            m_use = mt;
+          }
+          const float base = (m_use == -INFINITY) ? 0.f : m_use;
+          float ps8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) ps8[i] = 0.f;
+#pragma unroll
+          for (int ch = 0; ch < kBN / 32; ++ch) {  // 32 scores -> 16 packed bf16 pairs per store
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const float p0 = fast_exp2(fmaf(__uint_as_float(sv[ch * 32 + j]), sl2, -base));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(sv[ch * 32 + j + 1]), sl2, -base));
+              ps8[(j >> 1) & 7] += p0 + p1;
+              pk[j / 2] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(tS + ch * 16, pk);
+          }
+          const float psum = ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
+          l_sum = l_sum * alpha + psum;
+          tmem_wait_st();
+          if (c > 0) {
+            // O may only be touched once the previous P V product has landed.
+            ok = mbar_wait(bar(BOD(x)), (c - 1) & 1, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            if (__any_sync(0xffffffffu, resc)) {
+              tc_fence_after();
+#pragma unroll
+              for (int q = 0; q < D / 32; ++q) {
+                uint32_t ov[32];
+                tmem_ld32_wait(tO + 32 * q, ov);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                tmem_st32(tO + 32 * q, ov);
+              }
+              tmem_wait_st();
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(bar(BPF(x)));
         }
-        tc_fence_before();
-        mbar_arrive(bar(BPF(g & 1)));
       }
-    }
 
     // ------------------------------------------------------------ epilogue
-    if (ok && total > 0) {
-      ok = mbar_wait(bar(BOD), (total - 1) & 1, abort_flag);
+    if (ok && c > 0) {
+      ok = mbar_wait(bar(BOD(x)), (c - 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
     }
-    if (ok) {
-      uint32_t ov[D];
-      if (total > 0) {
-        tc_fence_after();
-        if constexpr (D == 128) tmem_ld128_wait(tO + lane_base, ov);
-        else tmem_ld64_wait(tO + lane_base, ov);
-      }
+    if (ok || total == 0) {
       const bool has = l_sum > 0.f;
       const float inv = has ? 1.f / l_sum : 0.f;
       const float row_lse = has ? (m_use + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
+      if (c > 0) tc_fence_after();
+      long long o_off = 0;
+      float* lse_ptr = nullptr;
+      if (a.mode == kModeFinal) {
+        const long long orow = static_cast<long long>(b) * a.S + qpos;
+        o_off = (orow * a.Hq + h) * D;
+        lse_ptr = a.lse + orow * a.Hq + h;
+      } else {
+        const long long prow = static_cast<long long>(b) * a.acc_brows + qs.mem + t0 + x * kBM + row;
+        o_off = (prow * a.Hq + h) * D;
+        lse_ptr = a.acc_lse + prow * a.Hq + h;
+      }
+      MergeWeights mw;
+      mw.w = 1.f;
+      mw.lse = row_lse;
+      if (valid && a.mode == kModeMerge) mw = merge_weights(*lse_ptr, row_lse);
+      if (valid) *lse_ptr = mw.lse;
 #pragma unroll
-      for (int i = 0; i < D; ++i) ov[i] = __float_as_uint(has ? __uint_as_float(ov[i]) * inv : 0.f);
-
-      if (valid) {
-        if (a.mode == kModeFinal) {
-          const long long orow = static_cast<long long>(b) * a.S + qpos;
-          const long long o = (orow * a.Hq + h) * D;
-          a.lse[orow * a.Hq + h] = row_lse;
-          if (a.out_bf16) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + o);
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t ov[32];
+        if (c > 0) tmem_ld32_wait(tO + 32 * q, ov);  // c is uniform across the warp
 #pragma unroll
-            for (int i = 0; i < D / 8; ++i) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(ov[8 * i + 0]), __uint_as_float(ov[8 * i + 1]));
-              w.y = pack_bf16x2(__uint_as_float(ov[8 * i + 2]), __uint_as_float(ov[8 * i + 3]));
-              w.z = pack_bf16x2(__uint_as_float(ov[8 * i + 4]), __uint_as_float(ov[8 * i + 5]));
-              w.w = pack_bf16x2(__uint_as_float(ov[8 * i + 6]), __uint_as_float(ov[8 * i + 7]));
-              dst[i] = w;
-            }
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(a.out) + o);
+        for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(has ? __uint_as_float(ov[i]) * inv : 0.f);
+        if (!valid) continue;
+        if (a.mode == kModeFinal && a.out_bf16) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + o_off + 32 * q);
 #pragma unroll
-            for (int i = 0; i < D / 4; ++i)
-              dst[i] = make_uint4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
+          for (int i = 0; i < 4; ++i) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(ov[8 * i + 0]), __uint_as_float(ov[8 * i + 1]));
+            w.y = pack_bf16x2(__uint_as_float(ov[8 * i + 2]), __uint_as_float(ov[8 * i + 3]));
+            w.z = pack_bf16x2(__uint_as_float(ov[8 * i + 4]), __uint_as_float(ov[8 * i + 5]));
+            w.w = pack_bf16x2(__uint_as_float(ov[8 * i + 6]), __uint_as_float(ov[8 * i + 7]));
+            dst[i] = w;
           }
         } else {
-          const long long prow =
-              static_cast<long long>(b) * a.acc_brows + static_cast<long long>(r) * a.acc_rmul * a.L + tl;
-          float* dst = a.acc_out + (prow * a.Hq + h) * D;
-          float* dl = a.acc_lse + prow * a.Hq + h;
-          if (a.mode == kModePartial) {
-            *dl = row_lse;
+          float4* dst =
+              reinterpret_cast<float4*>((a.mode == kModeFinal ? static_cast<float*>(a.out) : a.acc_out) + o_off + 32 * q);
 #pragma unroll
-            for (int i = 0; i < D / 4; ++i)
-              reinterpret_cast<uint4*>(dst)[i] = make_uint4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
-          } else {
-            const MergeWeights mw = merge_weights(*dl, row_lse);
-            *dl = mw.lse;
-            if (mw.w != 0.f) {
-#pragma unroll
-              for (int i = 0; i < D / 4; ++i) {
-                float4 cur = reinterpret_cast<float4*>(dst)[i];
-                cur.x = merge_out(cur.x, __uint_as_float(ov[4 * i + 0]), mw.w);
-                cur.y = merge_out(cur.y, __uint_as_float(ov[4 * i + 1]), mw.w);
-                cur.z = merge_out(cur.z, __uint_as_float(ov[4 * i + 2]), mw.w);
-                cur.w = merge_out(cur.w, __uint_as_float(ov[4 * i + 3]), mw.w);
-                reinterpret_cast<float4*>(dst)[i] = cur;
-              }
+          for (int i = 0; i < 8; ++i) {
+            float4 v = make_float4(__uint_as_float(ov[4 * i]), __uint_as_float(ov[4 * i + 1]),
+                                   __uint_as_float(ov[4 * i + 2]), __uint_as_float(ov[4 * i + 3]));
+            if (a.mode == kModeMerge) {
+              if (mw.w == 0.f) continue;
+              const float4 old = dst[i];
+              v.x = merge_out(old.x, v.x, mw.w);
+              v.y = merge_out(old.y, v.y, mw.w);
+              v.z = merge_out(old.z, v.z, mw.w);
+              v.w = merge_out(old.w, v.w, mw.w);
             }
+            dst[i] = v;
           }
         }
       }
@@ -432,7 +498,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, 512);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace ra

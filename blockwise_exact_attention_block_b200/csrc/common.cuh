@@ -176,6 +176,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
       : "memory");
 }
 
+// Stores 16 consecutive 32-bit TMEM columns of this thread's lane (warp-collective).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      RA_S32(0), RA_S32(1), RA_S32(2), RA_S32(3), RA_S32(4), RA_S32(5), RA_S32(6), RA_S32(7),
+      RA_S32(8), RA_S32(9), RA_S32(10), RA_S32(11), RA_S32(12), RA_S32(13), RA_S32(14), RA_S32(15)
+      : "memory");
+}
+
 #undef RA_S32
 
 // Shared-memory matrix descriptor for a tile written by TMA with 128-byte

@@ -167,7 +167,7 @@ ra_status ra_ring_attention(const void* q, const void* k, const void* v, ra_dtyp
  * none is needed; (size_t)-1 when the arguments are invalid. */
 size_t ra_ring_attention_workspace(int B, int S, int Hq, int D, int n_blocks, int gqa_groups,
                                    ra_partition partition, ra_dtype in_dtype,
-                                   const ra_options* opts);
+                                   ra_dtype out_dtype, const ra_options* opts);
 
 /*
  * ra_zigzag_permute - reorder token rows between original order and the

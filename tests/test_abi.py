@@ -6,6 +6,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "ra.h")
@@ -73,8 +74,10 @@ def test_ring_attention_rejects_bad_arguments(ra):
     assert ring(ra, out=FAKE + 4) == E.RA_ERR_INVALID_ARG      # misaligned
     assert ring(ra, in_dtype=7) == E.RA_ERR_INVALID_ARG
     assert ring(ra, part=5) == E.RA_ERR_INVALID_ARG
-    assert ring(ra, ws=None) == E.RA_ERR_WORKSPACE
-    assert ring(ra, ws_bytes=16) == E.RA_ERR_WORKSPACE
+    assert ring(ra, ws=None, in_dtype=ra.RA_F32) == E.RA_ERR_WORKSPACE     # fp32 inputs are rounded in scratch
+    assert ring(ra, ws_bytes=16, in_dtype=ra.RA_F32) == E.RA_ERR_WORKSPACE
+    unf = ra.ra_options(0, ra.RA_SCHED_UNFUSED, None, None)
+    assert ring(ra, ws=None, opts=ctypes.byref(unf)) == E.RA_ERR_WORKSPACE  # per-step partials
     bad = ra.ra_options(9, 0, None, None)
     assert ring(ra, opts=ctypes.byref(bad)) == E.RA_ERR_INVALID_ARG
 
@@ -112,11 +115,17 @@ def test_merge_and_permute_reject_bad_arguments(ra):
 
 
 def test_workspace_query(ra):
-    n = ra.ra_ring_attention_workspace(1, 24000, 32, 128, 4, 4, "zigzag")
-    # permuted bf16 copies of Q (32 heads) and K, V (8 heads each)
-    assert n >= 24000 * (32 + 8 + 8) * 128 * 2
+    # the partition is an index map: bf16 inputs need no scratch on the default path
+    assert ra.ra_ring_attention_workspace(1, 24000, 32, 128, 4, 4, "zigzag") == 0
     assert ra.ra_ring_attention_workspace(1, 4096, 8, 128, 4, 1, "contiguous") == 0
+    # fp32 inputs: bf16 copies of Q (32 heads) and K, V (8 heads each)
+    n = ra.ra_ring_attention_workspace(1, 24000, 32, 128, 4, 4, "zigzag", in_dtype=torch.float32)
+    assert n >= 24000 * (32 + 8 + 8) * 128 * 2
+    # unfused: fp32 partial out + lse; bf16 output adds the fp32 running output
     n_unf = ra.ra_ring_attention_workspace(1, 4096, 8, 128, 4, 1, "contiguous", sched="unfused")
-    assert n_unf >= 2 * 4096 * 8 * (128 + 1) * 4
+    assert n_unf >= 4096 * 8 * (128 + 1) * 4
+    n_unf16 = ra.ra_ring_attention_workspace(1, 4096, 8, 128, 4, 1, "contiguous", sched="unfused",
+                                             out_dtype=torch.bfloat16)
+    assert n_unf16 >= n_unf + 4096 * 8 * 128 * 4
     with pytest.raises(ra.RAError):
         ra.ra_ring_attention_workspace(1, 4095, 8, 128, 4, 1, "zigzag")
