@@ -48,6 +48,7 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     p.add_argument("--sched", default="auto", choices=["auto", "persistent", "fused", "unfused"])
     p.add_argument("--order", default="ring", choices=["ring", "tokenring"])
+    p.add_argument("--tiling", default="auto", choices=["auto", "row_pairs", "kv_split"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -70,7 +71,8 @@ def peaks():
 def workload_config(w, args, l2):
     return {"workload": w.name, "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "n_blocks": w.n_blocks,
             "causal": w.causal, "partition": w.partition, "in_dtype": w.in_dtype, "out_dtype": w.out_dtype,
-            "sched": args.sched, "order": args.order, "l2": l2, "parallelism": f"replicas{args.gpus}"}
+            "sched": args.sched, "order": args.order, "tiling": args.tiling, "l2": l2,
+            "parallelism": f"replicas{args.gpus}"}
 
 
 # ------------------------------------------------------------- CPU oracle
@@ -208,7 +210,8 @@ def run_ours(args):
 
     def step(events=None):
         ra.ra_ring_attention(q, k, v, w.n_blocks, w.causal, w.partition, w.gqa_groups, out=out, lse=lse,
-                             workspace=ws, order=args.order, sched=args.sched, attn_events=events)
+                             workspace=ws, order=args.order, sched=args.sched, attn_events=events,
+                             tiling=args.tiling)
 
     for _ in range(args.warmup):
         flush.zero_()

@@ -45,7 +45,10 @@ EXPORTED = ["ra_block_attn", "ra_merge_partial", "ra_merge_partials", "ra_ring_a
 
 class ra_options(ctypes.Structure):
     _fields_ = [("order", ctypes.c_int), ("sched", ctypes.c_int), ("attn_event_begin", ctypes.c_void_p),
-                ("attn_event_end", ctypes.c_void_p)]
+                ("attn_event_end", ctypes.c_void_p), ("tiling", ctypes.c_int)]
+
+
+TILINGS = {"auto": 0, "row_pairs": 1, "kv_split": 2}
 
 
 _vp, _i, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
@@ -111,8 +114,8 @@ def _dtype_code(dt: torch.dtype) -> int:
     raise ValueError(f"unsupported dtype {dt}")
 
 
-def _opts(order: str, sched: str, events=None) -> ra_options:
-    o = ra_options(ORDERS[order], SCHEDS[sched], None, None)
+def _opts(order: str, sched: str, events=None, tiling: str = "auto") -> ra_options:
+    o = ra_options(ORDERS[order], SCHEDS[sched], None, None, TILINGS[tiling])
     if events is not None:
         for ev in events:
             if ev.cuda_event == 0:  # torch creates the CUDA event on its first record
@@ -177,7 +180,7 @@ def ra_ring_attention_workspace(B, S, Hq, D, n_blocks, gqa_groups, partition="co
 def ra_ring_attention(q, k, v, n_blocks: int, causal: bool, partition: str = "contiguous",
                       gqa_groups: int | None = None, out=None, out_dtype=torch.float32, lse=None,
                       workspace=None, order: str = "ring", sched: str = "auto", stream=None,
-                      attn_events=None):
+                      attn_events=None, tiling: str = "auto"):
     """The whole method on one GPU.  Returns (out [B, S, Hq, D], lse fp32 [B, S, Hq]).
 
     attn_events: optional pair of torch.cuda.Event recorded around the
@@ -195,7 +198,7 @@ def ra_ring_attention(q, k, v, n_blocks: int, causal: bool, partition: str = "co
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    o = _opts(order, sched, attn_events)
+    o = _opts(order, sched, attn_events, tiling)
     _check(_lib.ra_ring_attention(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q.dtype), B, S, Hq, D, n_blocks,
                                   int(bool(causal)), PARTITIONS[partition], gqa_groups, _ptr(out),
                                   _dtype_code(out.dtype), _ptr(lse), _ptr(workspace), ws_bytes, ctypes.byref(o),

@@ -100,6 +100,19 @@ ra_status check_geom(int B, int S, int n, int Hq, int Hkv, int D, int partition,
   return RA_OK;
 }
 
+inline int seg_len_of(const Geom& g) { return g.zigzag ? g.c : g.L; }
+
+// Row pairs (256 query rows per CTA, shared K/V loads) unless that leaves
+// fewer than two CTAs per SM; then KV-split (128 rows per CTA, the KV tiles
+// halved between the two tiles and merged on chip), which doubles the CTA
+// count and halves the longest CTA.
+void choose_tiling(const Geom& g, AttnArgs& a, ra_tiling tiling) {
+  const int len = seg_len_of(g);
+  const long long pairs = static_cast<long long>(a.Hq) * a.B * a.nq * a.nseg * ((len + kCtaRows - 1) / kCtaRows);
+  a.kv_split = tiling == RA_TILING_KV_SPLIT || (tiling == RA_TILING_AUTO && pairs < 2LL * sm_count()) ? 1 : 0;
+  a.seg_tiles = (len + (a.kv_split ? kBM : kCtaRows) - 1) / (a.kv_split ? kBM : kCtaRows);
+}
+
 AttnArgs base_args(const Geom& g) {
   AttnArgs a;
   memset(&a, 0, sizeof(a));
@@ -110,8 +123,7 @@ AttnArgs base_args(const Geom& g) {
   a.groups = g.groups;
   a.causal = g.causal;
   a.nseg = g.zigzag ? 2 : 1;
-  const int seg_len = g.zigzag ? g.c : g.L;
-  a.seg_tiles = (seg_len + kCtaRows - 1) / kCtaRows;
+  a.seg_tiles = (seg_len_of(g) + kCtaRows - 1) / kCtaRows;
   a.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(g.D)));
   return a;
 }
@@ -266,6 +278,7 @@ Plan make_plan(const Geom& g, ra_dtype in_dtype, ra_dtype out_dtype, const ra_op
 bool valid_opts(const ra_options* o) {
   if (!o) return true;
   if (o->order != RA_ORDER_RING && o->order != RA_ORDER_TOKENRING) return false;
+  if (o->tiling < RA_TILING_AUTO || o->tiling > RA_TILING_KV_SPLIT) return false;
   return o->sched >= RA_SCHED_AUTO && o->sched <= RA_SCHED_PERSISTENT;
 }
 
@@ -325,6 +338,7 @@ ra_status ra_block_attn(const void* q, const void* k, const void* v, ra_dtype in
   block_segments(g, kv_block, true, a.kvseg[kv_block]);
   a.kv_list[0][0] = static_cast<signed char>(kv_block);
   order_segments(a);
+  choose_tiling(g, a, RA_TILING_AUTO);
   a.mode = kModePartial;
   a.acc_out = block_out;
   a.acc_lse = block_lse;
@@ -465,6 +479,7 @@ ra_status ra_ring_attention(const void* q, const void* k, const void* v, ra_dtyp
     block_segments(g, r, false, a.kvseg[r]);
   }
   order_segments(a);
+  choose_tiling(g, a, opts ? opts->tiling : RA_TILING_AUTO);
 
   if (p.sched == RA_SCHED_PERSISTENT) {
     // a3-a6 in one launch: the running state is carried across block boundaries

@@ -1,9 +1,13 @@
 // attn_fwd.cuh - block attention on the 5th-generation tensor cores (sm_100a).
 //
-// One CTA computes 256 consecutive query rows (two 128-row tiles, A and B) of
-// one (batch, query head) against a list of KV blocks (one block for
-// ra_block_attn and the unfused schedule; every block, in schedule order, for
-// the persistent schedule).  Both tiles share every K/V tile load.
+// One CTA runs two 128-row query tiles, A and B, of one (batch, query head)
+// against a list of KV blocks (one block for ra_block_attn and the unfused
+// schedule; every block, in schedule order, for the persistent schedule).
+// Row-pair mode: A and B are 256 consecutive query rows and share every K/V
+// tile load.  KV-split mode (grids too small to fill the GPU): A and B are
+// the same 128 rows; A takes the first half of the KV tiles, B the second
+// half, and the two partial results are stitched on chip with the merge rule
+// (the rule the method uses between blocks, applied inside one block).
 //
 // TokenRing review (pith.science, arXiv 2412.20501), "What carries the
 // argument" / "Core claim": the flash-attention kernel that yields, for one
@@ -73,7 +77,8 @@ struct AttnArgs {
   int nq;                 // query blocks covered by this launch
   int nkv;                // KV blocks each query block visits in this launch
   int nseg;               // segments per block: 1 (contiguous) or 2 (zigzag)
-  int seg_tiles;          // ceil(segment length / 256): CTAs per query segment
+  int seg_tiles;          // CTAs per query segment: ceil(len / 256), or ceil(len / 128) in KV-split mode
+  int kv_split;           // 1: KV-split mode (see the top of this file)
   float scale_log2;       // log2(e) / sqrt(D)
   int mode;               // AttnMode
   // kModePartial / kModeMerge: row = b * acc_brows + memory row of the query
@@ -161,11 +166,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int qi = so / a.nseg;
   const Seg qs = a.qseg[qi][so % a.nseg];
   const int hk = h / a.groups;
-  const int t0 = qt * kCtaRows;  // CTA row offset inside the query segment
-  int rows[2], last[2];
+  const bool split = a.kv_split != 0;
+  const int t0 = qt * (split ? kBM : kCtaRows);  // CTA row offset inside the query segment
+  int rows[2], last[2], row0[2];                 // per tile: valid rows, last position, first row
   for (int x = 0; x < 2; ++x) {
-    rows[x] = min(max(qs.len - t0 - x * kBM, 0), kBM);
-    last[x] = rows[x] > 0 ? qs.pos + t0 + x * kBM + rows[x] - 1 : -1;
+    row0[x] = t0 + (split ? 0 : x * kBM);
+    rows[x] = min(max(qs.len - row0[x], 0), kBM);
+    last[x] = rows[x] > 0 ? qs.pos + row0[x] + rows[x] - 1 : -1;
   }
   const int last_u = max(last[0], last[1]);  // the CTA's last row: its KV range covers both tiles
   auto seg_of = [&](int s_, int e_) -> const Seg& { return a.kvseg[a.kv_list[qi][s_]][e_]; };
@@ -173,6 +180,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   int total = 0;
   for (int s = 0; s < a.nkv; ++s)
     for (int e = 0; e < a.nseg; ++e) total += tiles_for(a, seg_of(s, e), last_u);
+  // Tile x's share of the CTA's KV tiles.  u = index in the CTA's sequence,
+  // t = index inside the segment.  KV-split: A takes [0, half), B [half, total).
+  const int half = (total + 1) / 2;
+  auto active = [&](int x, int u, int t, const Seg& ks) -> bool {
+    if (split) return x == 0 ? u < half : u >= half;
+    return t < tiles_for(a, ks, last[x]);
+  };
+  // The segment and in-segment tile of the CTA's u-th KV tile.
+  auto locate = [&](int u, int& s_, int& e_, int& t_) {
+    for (s_ = 0; s_ < a.nkv; ++s_)
+      for (e_ = 0; e_ < a.nseg; ++e_) {
+        const int nt = tiles_for(a, seg_of(s_, e_), last_u);
+        if (u < nt) {
+          t_ = u;
+          return;
+        }
+        u -= nt;
+      }
+    t_ = 0;
+  };
 
   auto bar = [&](int i) -> uint32_t { return sb + SL::kBar + 8u * i; };
   const int BQ = 0;
@@ -206,36 +233,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_expect_tx(bar(BQ), 2 * SL::kTile);
-      for (int x = 0; x < 2; ++x)
+      const int nqt = split ? 1 : 2;  // KV-split: both tiles read Q_A
+      mbar_expect_tx(bar(BQ), nqt * SL::kTile);
+      for (int x = 0; x < nqt; ++x)
         for (int bx = 0; bx < SL::kNBox; ++bx)
-          tma_load_4d(sb + SL::kQ + x * SL::kTile + bx * SL::kBox, &tmQ, bx * 64, h, qs.mem + t0 + x * kBM, b,
+          tma_load_4d(sb + SL::kQ + x * SL::kTile + bx * SL::kBox, &tmQ, bx * 64, h, qs.mem + row0[x], b,
                       bar(BQ));
       int g = 0;
       bool ok = true;
       int issued_k[NST], issued_v[NST];
       for (int s = 0; s < NST; ++s) issued_k[s] = issued_v[s] = -1;
-      for (int s = 0; s < a.nkv && ok; ++s) {
-        for (int e = 0; e < a.nseg && ok; ++e) {
-          const Seg ks = seg_of(s, e);
-          const int nt = tiles_for(a, ks, last_u);
-          for (int t = 0; t < nt; ++t, ++g) {
-            const int st = g % NST;
-            const uint32_t ph = (g / NST) & 1;
-            if (!mbar_wait(bar(BKE(st)), ph ^ 1, abort_flag)) { ok = false; break; }
-            mbar_expect_tx(bar(BKF(st)), SL::kTile);
-            for (int bx = 0; bx < SL::kNBox; ++bx)
-              tma_load_4d(sb + SL::kK + st * SL::kTile + bx * SL::kBox, &tmK, bx * 64, hk, ks.mem + t * kBN, b,
-                          bar(BKF(st)));
-            issued_k[st] = g;
-            if (!mbar_wait(bar(BVE(st)), ph ^ 1, abort_flag)) { ok = false; break; }
-            mbar_expect_tx(bar(BVF(st)), SL::kTile);
-            for (int bx = 0; bx < SL::kNBox; ++bx)
-              tma_load_4d(sb + SL::kV + st * SL::kTile + bx * SL::kBox, &tmV, bx * 64, hk, ks.mem + t * kBN, b,
-                          bar(BVF(st)));
-            issued_v[st] = g;
-          }
-        }
+      // load order: the CTA's sequence (row pairs), or A0, B0, A1, B1, ... (KV-split)
+      for (int g2 = 0; g2 < total && ok; ++g2) {
+        int s, e, t;
+        locate(split ? ((g2 & 1) ? half + (g2 >> 1) : (g2 >> 1)) : g2, s, e, t);
+        const Seg ks = seg_of(s, e);
+        const int st = g % NST;
+        const uint32_t ph = (g / NST) & 1;
+        if (!mbar_wait(bar(BKE(st)), ph ^ 1, abort_flag)) { ok = false; break; }
+        mbar_expect_tx(bar(BKF(st)), SL::kTile);
+        for (int bx = 0; bx < SL::kNBox; ++bx)
+          tma_load_4d(sb + SL::kK + st * SL::kTile + bx * SL::kBox, &tmK, bx * 64, hk, ks.mem + t * kBN, b,
+                      bar(BKF(st)));
+        issued_k[st] = g;
+        if (!mbar_wait(bar(BVE(st)), ph ^ 1, abort_flag)) { ok = false; break; }
+        mbar_expect_tx(bar(BVF(st)), SL::kTile);
+        for (int bx = 0; bx < SL::kNBox; ++bx)
+          tma_load_4d(sb + SL::kV + st * SL::kTile + bx * SL::kBox, &tmV, bx * 64, hk, ks.mem + t * kBN, b,
+                      bar(BVF(st)));
+        issued_v[st] = g;
+        ++g;
       }
       if (!ok) {  // let every copy already issued land before shared memory is released
         mbar_drain(bar(BQ), 0);
@@ -250,11 +277,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (lane == 0 && total > 0) {
       constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, D, true);
+      const int qslot1 = split ? 0 : 1;  // Q tile of B
       auto issue_s = [&](int x, int st) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
-          const uint64_t ad = smem_desc_sw128(sb + SL::kQ + x * SL::kTile + off, 16, 1024);
+          const uint64_t ad = smem_desc_sw128(sb + SL::kQ + (x ? qslot1 : 0) * SL::kTile + off, 16, 1024);
           const uint64_t bd = smem_desc_sw128(sb + SL::kK + st * SL::kTile + off, 16, 1024);
           mma_ss(tmem + x * 128, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
         }
@@ -280,11 +308,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           k.nt = k.s < a.nkv ? tiles_for(a, seg_of(k.s, k.e), last_u) : 0;
         }
       };
-      auto active = [&](const KvCursor& k, int x) { return k.t < tiles_for(a, seg_of(k.s, k.e), last[x]); };
+      auto active_at = [&](const KvCursor& k, int x) { return k.t < tiles_for(a, seg_of(k.s, k.e), last[x]); };
 
+      if (split) {
+        // KV-split: tile x's i-th KV tile is load 2i + x (A has half, B total - half tiles)
+        const int n_of[2] = {half, total - half};
+        bool okk = mbar_wait(bar(BQ), 0, abort_flag);
+        for (int x = 0; x < 2 && okk; ++x) {
+          if (n_of[x] == 0) continue;
+          okk = mbar_wait(bar(BKF(x % NST)), (x / NST) & 1, abort_flag);
+          if (!okk) break;
+          tc_fence_after();
+          issue_s(x, x % NST);
+          tc_commit(bar(BKE(x % NST)));
+        }
+        for (int j = 0; j < half && okk; ++j) {
+          for (int x = 0; x < 2; ++x) {
+            if (j >= n_of[x]) continue;
+            const int ld = 2 * j + x, st = ld % NST;
+            if (!mbar_wait(bar(BVF(st)), (ld / NST) & 1, abort_flag)) { okk = false; break; }
+            if (!mbar_wait(bar(BPF(x)), j & 1, abort_flag)) { okk = false; break; }
+            tc_fence_after();
+            issue_pv(x, st, j > 0);
+            tc_commit(bar(BVE(st)));
+            if (j + 1 < n_of[x]) {
+              const int ld1 = ld + 2, st1 = ld1 % NST;
+              if (!mbar_wait(bar(BKF(st1)), (ld1 / NST) & 1, abort_flag)) { okk = false; break; }
+              tc_fence_after();
+              issue_s(x, st1);
+              tc_commit(bar(BKE(st1)));
+            }
+          }
+        }
+        tc_commit(bar(BEND));
+        mbar_drain(bar(BEND), 0);
+      } else {
       KvCursor cur = {0, 0, -1, tiles_for(a, seg_of(0, 0), last_u)};
       advance(cur);  // first existing tile (total > 0, so there is one)
-      bool act[2] = {active(cur, 0), active(cur, 1)};
+      bool act[2] = {active_at(cur, 0), active_at(cur, 1)};
       int cnt[2] = {0, 0};  // P V products issued per tile
       bool ok = mbar_wait(bar(BQ), 0, abort_flag);
       if (ok) ok = mbar_wait(bar(BKF(0)), 0, abort_flag);
@@ -301,8 +362,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         bool act1[2] = {false, false};
         if (has_next) {
           advance(nxt);
-          act1[0] = active(nxt, 0);
-          act1[1] = active(nxt, 1);
+          act1[0] = active_at(nxt, 0);
+          act1[1] = active_at(nxt, 1);
         }
         if (!mbar_wait(bar(BVF(st)), (g / NST) & 1, abort_flag)) break;
         bool k_ready = false;
@@ -332,13 +393,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // nothing may still write tensor memory when it is released
       tc_commit(bar(BEND));
       mbar_drain(bar(BEND), 0);
+      }
     }
   } else {
     // ------------------------------------------------------------- softmax
     const int x = warp >> 2;            // tile A (0) or B (1)
     const int row = threadIdx.x & 127;  // row inside the tile = TMEM lane
     const bool valid = row < rows[x];
-    const int qpos = valid ? qs.pos + t0 + x * kBM + row : -1;
+    const int qpos = valid ? qs.pos + row0[x] + row : -1;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + x * 128;
     const uint32_t tO = tmem + lane_base + 256 + x * 128;
@@ -347,12 +409,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float l_sum = 0.f;
     bool ok = total > 0;
     int c = 0;  // tiles processed by this tile's softmax
+    int u = 0;  // position in the CTA's KV sequence
     for (int s = 0; s < a.nkv && ok; ++s)
       for (int e = 0; e < a.nseg && ok; ++e) {
         const Seg ks = seg_of(s, e);
-        const int nt = tiles_for(a, ks, last[x]);  // this tile's prefix of the CTA's tiles
+        const int nt = tiles_for(a, ks, last_u);
         const int lim = visible_count(a, ks, qpos);
-        for (int t = 0; t < nt; ++t, ++c) {
+        for (int t = 0; t < nt; ++t, ++u) {
+          if (!active(x, u, t, ks)) continue;
           ok = mbar_wait(bar(BSF(x)), c & 1, abort_flag);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
@@ -426,6 +490,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           tc_fence_before();
           mbar_arrive(bar(BPF(x)));
+          ++c;
         }
       }
 
@@ -434,10 +499,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ok = mbar_wait(bar(BOD(x)), (c - 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
     }
-    if (ok || total == 0) {
+    if (split) {
+      // Stitch B's partial into A's with the merge rule.  B writes its
+      // normalised row and lse to shared memory (the K/V ring is idle once
+      // both tiles' last P V product has landed), then A merges.
+      float* xo = reinterpret_cast<float*>(smem + SL::kK);  // [128][D + 4]
+      float* xl = xo + kBM * (D + 4);                        // [128]
+      named_barrier_sync(1, 256);  // both tiles' MMAs are complete
+      fence_proxy_async_smem();
+      if (x == 1) {
+        const bool has = ok && l_sum > 0.f;
+        const float inv = has ? 1.f / l_sum : 0.f;
+        xl[row] = has ? (m_use + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
+        if (c > 0) tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t ov[32];
+          if (ok && c > 0) tmem_ld32_wait(tO + 32 * q, ov);
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(xo + row * (D + 4) + 32 * q + i) =
+                make_float4(has ? __uint_as_float(ov[i]) * inv : 0.f, has ? __uint_as_float(ov[i + 1]) * inv : 0.f,
+                            has ? __uint_as_float(ov[i + 2]) * inv : 0.f, has ? __uint_as_float(ov[i + 3]) * inv : 0.f);
+        }
+      }
+      named_barrier_sync(1, 256);
+    }
+    // rows are written by every tile in row-pair mode, by A alone in KV-split mode
+    if ((ok || total == 0) && !(split && x == 1)) {
       const bool has = l_sum > 0.f;
       const float inv = has ? 1.f / l_sum : 0.f;
-      const float row_lse = has ? (m_use + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
+      float row_lse = has ? (m_use + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
+      MergeWeights mwb;  // KV-split: weight of B's partial in this row
+      mwb.w = 0.f;
+      if (split) {
+        mwb = merge_weights(row_lse, reinterpret_cast<float*>(smem + SL::kK)[kBM * (D + 4) + row]);
+        row_lse = mwb.lse;
+      }
       if (c > 0) tc_fence_after();
       long long o_off = 0;
       float* lse_ptr = nullptr;
@@ -446,7 +544,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         o_off = (orow * a.Hq + h) * D;
         lse_ptr = a.lse + orow * a.Hq + h;
       } else {
-        const long long prow = static_cast<long long>(b) * a.acc_brows + qs.mem + t0 + x * kBM + row;
+        const long long prow = static_cast<long long>(b) * a.acc_brows + qs.mem + row0[x] + row;
         o_off = (prow * a.Hq + h) * D;
         lse_ptr = a.acc_lse + prow * a.Hq + h;
       }
@@ -461,6 +559,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (c > 0) tmem_ld32_wait(tO + 32 * q, ov);  // c is uniform across the warp
 #pragma unroll
         for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(has ? __uint_as_float(ov[i]) * inv : 0.f);
+        if (split && mwb.w != 0.f) {
+          const float* xb = reinterpret_cast<const float*>(smem + SL::kK) + row * (D + 4) + 32 * q;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(merge_out(__uint_as_float(ov[i]), xb[i], mwb.w));
+        }
         if (!valid) continue;
         if (a.mode == kModeFinal && a.out_bf16) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + o_off + 32 * q);

@@ -101,6 +101,18 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* m, 
       : "memory");
 }
 
+// Barrier over the first `count` threads' warps that execute it (id 1-15;
+// id 0 is __syncthreads).
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Orders this thread's earlier async-proxy (TMA / tensor core) shared-memory
+// accesses before its later generic ones.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // --------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tc_fence_before() {

@@ -84,6 +84,13 @@ typedef enum {
   RA_SCHED_PERSISTENT = 3
 } ra_sched;
 
+/* How the block-attention kernel splits work between CTAs.
+ *  ROW_PAIRS: 256 query rows per CTA (two 128-row tiles sharing K/V loads).
+ *  KV_SPLIT:  128 query rows per CTA; the CTA's KV tiles are halved between
+ *             its two tiles and the two partials merged on chip with the rule.
+ *  AUTO:      ROW_PAIRS unless that gives fewer than two CTAs per SM. */
+typedef enum { RA_TILING_AUTO = 0, RA_TILING_ROW_PAIRS = 1, RA_TILING_KV_SPLIT = 2 } ra_tiling;
+
 typedef struct {
   ra_order order;  /* default RA_ORDER_RING  */
   ra_sched sched;  /* default RA_SCHED_AUTO  */
@@ -92,6 +99,7 @@ typedef struct {
    * call, so a caller can time the attention kernels inside the full call. */
   void* attn_event_begin;
   void* attn_event_end;
+  ra_tiling tiling; /* default RA_TILING_AUTO */
 } ra_options;
 
 /*

@@ -76,10 +76,12 @@ def test_ring_attention_rejects_bad_arguments(ra):
     assert ring(ra, part=5) == E.RA_ERR_INVALID_ARG
     assert ring(ra, ws=None, in_dtype=ra.RA_F32) == E.RA_ERR_WORKSPACE     # fp32 inputs are rounded in scratch
     assert ring(ra, ws_bytes=16, in_dtype=ra.RA_F32) == E.RA_ERR_WORKSPACE
-    unf = ra.ra_options(0, ra.RA_SCHED_UNFUSED, None, None)
+    unf = ra.ra_options(0, ra.RA_SCHED_UNFUSED, None, None, 0)
     assert ring(ra, ws=None, opts=ctypes.byref(unf)) == E.RA_ERR_WORKSPACE  # per-step partials
-    bad = ra.ra_options(9, 0, None, None)
+    bad = ra.ra_options(9, 0, None, None, 0)
     assert ring(ra, opts=ctypes.byref(bad)) == E.RA_ERR_INVALID_ARG
+    bad_tiling = ra.ra_options(0, 0, None, None, 7)
+    assert ring(ra, opts=ctypes.byref(bad_tiling)) == E.RA_ERR_INVALID_ARG
 
 
 def test_block_attn_rejects_bad_arguments(ra):

@@ -134,21 +134,22 @@ def test_block_attn_every_pair(cuda_lib, case):
 SCHEDS = ["persistent", "fused", "unfused"]
 
 
+@pytest.mark.parametrize("tiling", ["row_pairs", "kv_split"])
 @pytest.mark.parametrize("order", ["ring", "tokenring"])
 @pytest.mark.parametrize("sched", SCHEDS)
 @pytest.mark.parametrize("case", [(2, 1200, 4, 4, 2, 128, True, "zigzag"), (1, 1024, 4, 2, 1, 64, True, "contiguous"),
-                                  (1, 640, 5, 2, 2, 128, False, "zigzag")],
+                                  (1, 640, 5, 2, 2, 128, False, "zigzag"), (1, 2304, 2, 2, 2, 128, True, "contiguous")],
                          ids=lambda c: f"B{c[0]}S{c[1]}n{c[2]}D{c[5]}{c[7]}{'C' if c[6] else ''}")
-def test_ring_attention_matches_full_oracle(cuda_lib, case, sched, order):
+def test_ring_attention_matches_full_oracle(cuda_lib, case, sched, order, tiling):
     ra = cuda_lib
     B, S, n, Hq, Hkv, D, causal, part = case
     q, k, v = attention_inputs(B, S, Hq, Hkv, D, "bf16", seed=4)
     ro, rl = F.full_attention(q, k, v, causal, Hq // Hkv)
     for out_dtype in (torch.float32, torch.bfloat16):
         o, l = ra.ra_ring_attention(q.cuda(), k.cuda(), v.cuda(), n, causal, part, out_dtype=out_dtype,
-                                    order=order, sched=sched)
-        assert_close_bf16(to_np(o), ro, f"out {sched}/{order}/{out_dtype}")
-        assert_close_bf16(to_np(l), rl, f"lse {sched}/{order}/{out_dtype}")
+                                    order=order, sched=sched, tiling=tiling)
+        assert_close_bf16(to_np(o), ro, f"out {sched}/{order}/{tiling}/{out_dtype}")
+        assert_close_bf16(to_np(l), rl, f"lse {sched}/{order}/{tiling}/{out_dtype}")
     assert ra.ra_get_device_status() == 0
 
 
@@ -174,13 +175,14 @@ def zigzag4k():
     return w, (q, k, v), (ro, rl)
 
 
+@pytest.mark.parametrize("tiling", ["auto", "row_pairs", "kv_split"])
 @pytest.mark.parametrize("sched", SCHEDS)
 @pytest.mark.parametrize("order", ["ring", "tokenring"])
-def test_zigzag4k_workload_full_oracle(cuda_lib, zigzag4k, sched, order):
+def test_zigzag4k_workload_full_oracle(cuda_lib, zigzag4k, sched, order, tiling):
     ra = cuda_lib
     w, (q, k, v), (ro, rl) = zigzag4k
     o, l = ra.ra_ring_attention(q.cuda(), k.cuda(), v.cuda(), w.n_blocks, w.causal, w.partition, sched=sched,
-                                order=order)
+                                order=order, tiling=tiling)
     assert_close_bf16(to_np(o), ro, "zigzag4k out")
     assert_close_bf16(to_np(l), rl, "zigzag4k lse")
 
