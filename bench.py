@@ -52,6 +52,11 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-merge", action="store_true")
+    p.add_argument("--merge-sweep", action="store_true",
+                   help="time the merge kernels over the whole token / partial sweep instead")
+    p.add_argument("--merge-T", type=int, nargs="*", default=None, help="token counts of the merge sweep")
+    p.add_argument("--merge-k", type=int, nargs="*", default=None, help="partial counts of the merge sweep")
     a = p.parse_args()
     if a.steps is None:
         a.steps = DEFAULT_STEPS[a.workload]
@@ -163,6 +168,69 @@ class Clocks:
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def kernel_sha():
+    import hashlib
+    h = hashlib.sha256()
+    src = os.path.join(ROOT, "blockwise_exact_attention_block_b200", "csrc")
+    for f in ["attn_fwd.cuh", "common.cuh", "tmem_ld.cuh", "merge_rule.cuh"]:
+        h.update(open(os.path.join(src, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def attn_traffic(workload):
+    """DRAM bytes per attention launch from the committed ncu capture, or None
+    when there is none for this workload or the kernel changed since."""
+    path = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path)).get(workload)
+    if not rec or rec.get("kernel_sha") != kernel_sha():
+        return None
+    return rec["dram_bytes_per_launch"]
+
+
+# ------------------------------------------------------------ merge kernels
+
+def bench_merge(ra, dev, T, k, reps, flush, kway=False):
+    """GB/s of merging k partials of [T, 32, 128] fp32 (+ lse [T, 32]).
+
+    Pairwise: k-1 ra_merge_partial calls, 12*D+12 bytes per row each.
+    k-way: one ra_merge_partials call, (k+1)*(4*D+4) bytes per row.
+    At most 4 distinct partial buffers are allocated and cycled (16 partials
+    of 16 GiB do not fit in HBM); the bytes moved per merge are unchanged."""
+    import torch
+    H, D = 32, 128
+    rows = T * H
+    nb = min(max(k - 1, 1), 4) if not kway else min(k, 4)
+    g = torch.Generator(device=dev).manual_seed(1)
+    out = torch.randn((T, H, D), device=dev, generator=g)
+    lse = torch.rand((T, H), device=dev, generator=g) * 20 - 5
+    bos = [torch.randn((T, H, D), device=dev, generator=g) for _ in range(nb)]
+    bls = [torch.rand((T, H), device=dev, generator=g) * 20 - 5 for _ in range(nb)]
+    stream = torch.cuda.current_stream(dev)
+    times = []
+    for rep in range(reps + 2):
+        if rows * (D + 1) * 4 * 2 < 4 * (256 << 20):
+            flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        if kway:
+            ra.ra_merge_partials([out] + [bos[j % nb] for j in range(k - 1)],
+                                 [lse] + [bls[j % nb] for j in range(k - 1)], out=out, lse=lse)
+        else:
+            for j in range(k - 1):
+                ra.ra_merge_partial(out, lse, bos[j % nb], bls[j % nb])
+        e1.record(stream)
+        e1.synchronize()
+        if rep >= 2:
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    nbytes = rows * ((k + 1) * (4 * D + 4) if kway else (k - 1) * (12 * D + 12))
+    del out, lse, bos, bls
+    torch.cuda.empty_cache()
+    return nbytes / (ms * 1e-3) / 1e9, ms
 
 
 # ---------------------------------------------------------------- our arm
@@ -290,10 +358,7 @@ def run_ours(args):
     sustained = attn_mean > 100.0
     peak = pk["bf16_tflops_sustained" if sustained else "bf16_tflops"]
     achieved = w.flops / (attn_mean * 1e-3) / 1e12
-    prof = os.path.join(ROOT, "profiles", f"attn_fwd_{w.name}.json")
-    traffic = None
-    if os.path.exists(prof):
-        traffic = json.load(open(prof)).get("dram_bytes_per_launch")
+    traffic = attn_traffic(w.name)
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": traffic, "kernel": "attn_fwd_kernel",
             "peak_source": f"{pk_kind} {'sustained' if sustained else 'burst'} bf16 dense"}
@@ -302,6 +367,13 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v_, cores, sample, _ = oracle_sample(w)
         cpu = {"value": v_, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+    merge = None
+    if not args.no_merge:
+        gbs, mms = bench_merge(ra, dev, 1048576, 2, 10, flush)
+        merge = {"kernel": "merge_partial_kernel", "tokens": 1048576, "heads": 32, "D": 128, "partials": 2,
+                 "GB/s": gbs, "ms": mms, "peak_GB/s": pk["hbm_gbs"], "frac": gbs / pk["hbm_gbs"],
+                 "bytes_per_row": 12 * 128 + 12}
 
     value = w.flops * world * K / (total_ms * 1e-3) / 1e12
     line = {"metric": "causal-adj attention TFLOP/s (% of dense bf16 peak)", "value": value, "unit": "TFLOP/s",
@@ -312,6 +384,7 @@ def run_ours(args):
                                                f"L2 {l2_bytes >> 20} MiB)"),
             "pct_of_peak": 100.0 * value / peak, "attn_kernel_ms": attn_mean, "roofline": roof,
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "gpu_launches": K * launches_per_step(w, args.sched),
+            "merge": merge,
             "device_status": ra.ra_status_string(status)}
     if rank == 0:
         print(json.dumps(line))
@@ -321,10 +394,43 @@ def run_ours(args):
     return 0 if status == 0 else 1
 
 
+def run_merge_sweep(args):
+    import torch
+    import blockwise_exact_attention_block_b200 as ra
+    from seeded_inputs import MERGE_PARTIALS, MERGE_TOKENS
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    pk, pk_kind = peaks()
+    sweep = []
+    Ts = args.merge_T or MERGE_TOKENS
+    ks = args.merge_k or MERGE_PARTIALS
+    for T in Ts:
+        for k in ks:
+            reps = 10 if T <= 262144 else 3
+            pw, pw_ms = bench_merge(ra, dev, T, k, reps, flush)
+            kw, kw_ms = bench_merge(ra, dev, T, k, reps, flush, kway=True)
+            sweep.append({"T": T, "k": k, "pairwise_GB/s": pw, "pairwise_ms": pw_ms, "kway_GB/s": kw, "kway_ms": kw_ms})
+    top = max(sweep, key=lambda r: (r["T"], -r["k"]))
+    line = {"metric": "merge GB/s (% of HBM peak)", "value": top["pairwise_GB/s"], "unit": "GB/s", "n_gpus": 1,
+            "steps": None, "warmup": 2, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic (device randn / rand)",
+            "config": {"workload": "merge sweep [T,32,128] fp32", "T": Ts, "k": ks,
+                       "headline": {"T": top["T"], "k": top["k"]}},
+            "roofline": {"bound": "hbm", "achieved": top["pairwise_GB/s"], "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": top["pairwise_GB/s"] / pk["hbm_gbs"], "traffic": None,
+                         "peak_source": f"{pk_kind} copy bandwidth"},
+            "sweep": sweep}
+    print(json.dumps(line))
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.merge_sweep:
+        return run_merge_sweep(args)
     return run_ours(args)
 
 
