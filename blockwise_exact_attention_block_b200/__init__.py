@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_PKG, "libra_b200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m blockwise_exact_attention_block_b200.build`")
+        f"{LIB_PATH} is missing: build it with `python blockwise_exact_attention_block_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -40,7 +40,7 @@ SCHEDS = {"auto": RA_SCHED_AUTO, "unfused": RA_SCHED_UNFUSED, "fused": RA_SCHED_
 
 EXPORTED = ["ra_block_attn", "ra_merge_partial", "ra_merge_partials", "ra_ring_attention",
             "ra_ring_attention_workspace", "ra_zigzag_permute", "ra_get_device_status",
-            "ra_status_string", "ra_version"]
+            "ra_status_string", "ra_version", "ra_ring_attention_noalloc", "ra_noalloc_scratch_bytes"]
 
 
 class ra_options(ctypes.Structure):
@@ -63,6 +63,11 @@ _lib.ra_ring_attention.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i
 _lib.ra_ring_attention.restype = _i
 _lib.ra_ring_attention_workspace.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(ra_options)]
 _lib.ra_ring_attention_workspace.restype = _sz
+_lib.ra_ring_attention_noalloc.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _i, _vp,
+                                           ctypes.POINTER(ra_options), _vp]
+_lib.ra_ring_attention_noalloc.restype = _i
+_lib.ra_noalloc_scratch_bytes.argtypes = []
+_lib.ra_noalloc_scratch_bytes.restype = _sz
 _lib.ra_zigzag_permute.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
 _lib.ra_zigzag_permute.restype = _i
 _lib.ra_get_device_status.argtypes = [_vp]
@@ -204,6 +209,37 @@ def ra_ring_attention(q, k, v, n_blocks: int, causal: bool, partition: str = "co
                                   _dtype_code(out.dtype), _ptr(lse), _ptr(workspace), ws_bytes, ctypes.byref(o),
                                   _stream(stream)), "ra_ring_attention")
     return out, lse
+
+
+def ra_ring_attention_noalloc(q, k, v, n_blocks: int, causal: bool, partition: str = "contiguous",
+                              gqa_groups: int | None = None, out=None, out_dtype=torch.float32, lse=None,
+                              order: str = "ring", sched: str = "auto", stream=None, tiling: str = "auto"):
+    """ra_ring_attention with its scratch in the library's fixed device array.
+
+    For callers that may not allocate device memory at call time (their
+    framework owns the GPU's memory pool, or cudaMalloc's implicit device
+    synchronisation is not acceptable).  Pass `out` and `lse` to keep this
+    wrapper from allocating them.  Calls that need more than
+    ra_noalloc_scratch_bytes() of scratch raise RAError(RA_ERR_WORKSPACE);
+    calls that overlap on the GPU share the one scratch array and race."""
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if gqa_groups is None:
+        gqa_groups = Hq // Hkv
+    if out is None:
+        out = torch.empty((B, S, Hq, D), dtype=out_dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, S, Hq), dtype=torch.float32, device=q.device)
+    o = _opts(order, sched, None, tiling)
+    _check(_lib.ra_ring_attention_noalloc(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q.dtype), B, S, Hq, D, n_blocks,
+                                          int(bool(causal)), PARTITIONS[partition], gqa_groups, _ptr(out),
+                                          _dtype_code(out.dtype), _ptr(lse), ctypes.byref(o), _stream(stream)),
+           "ra_ring_attention_noalloc")
+    return out, lse
+
+
+def ra_noalloc_scratch_bytes() -> int:
+    return _lib.ra_noalloc_scratch_bytes()
 
 
 def ra_zigzag_permute(src, n_blocks: int, inverse: bool = False, dst=None, stream=None):

@@ -1,8 +1,11 @@
 """Build libra_b200.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m blockwise_exact_attention_block_b200.build [--verbose-ptxas]
+    python blockwise_exact_attention_block_b200/build.py [--verbose-ptxas]
 
-The library is one translation unit (csrc/api.cu) that includes every kernel.
+(run as a file: importing the package loads the library it builds)
+
+csrc/api.cu is the main translation unit (it includes every kernel);
+csrc/noalloc.cu adds the entry point whose scratch is a fixed device array.
 """
 from __future__ import annotations
 
@@ -13,7 +16,7 @@ import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
-SRC = os.path.join(PKG, "csrc", "api.cu")
+SRCS = [os.path.join(PKG, "csrc", "api.cu"), os.path.join(PKG, "csrc", "noalloc.cu")]
 OUT = os.path.join(PKG, "libra_b200.so")
 
 
@@ -41,7 +44,7 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
     if not force and up_to_date():
         return OUT
     cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
-           "-Xcompiler", "-fPIC", "-shared", "-I", os.path.join(ROOT, "include"), SRC, "-o", OUT + ".tmp"]
+           "-Xcompiler", "-fPIC", "-shared", "-I", os.path.join(ROOT, "include"), *SRCS, "-o", OUT + ".tmp"]
     if ptxas_verbose:
         cmd[1:1] = ["-Xptxas", "-v"]
     res = subprocess.run(cmd, capture_output=True, text=True)

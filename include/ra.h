@@ -189,6 +189,39 @@ size_t ra_ring_attention_workspace(int B, int S, int Hq, int D, int n_blocks, in
 ra_status ra_zigzag_permute(const void* src, void* dst, int B, int S, int H, int D,
                             int elem_bytes, int n_blocks, int inverse, void* stream);
 
+/*
+ * ra_ring_attention_noalloc - ra_ring_attention without a caller workspace;
+ * it allocates no memory at all.  (The pages have no counterpart: this is a
+ * deployment variant of the same call.)
+ *
+ * For callers that cannot allocate device memory at call time: code running
+ * after its framework has reserved the GPU's memory for its own pool, where a
+ * cudaMalloc fails or fragments that pool, and latency-bound callers that
+ * cannot accept the implicit device synchronisation of cudaMalloc/cudaFree.
+ * Arguments and results are those of ra_ring_attention minus the workspace.
+ * The scratch the call needs (ra_ring_attention_workspace) comes from one
+ * fixed device array of ra_noalloc_scratch_bytes() bytes (64 MiB) inside
+ * this library, held on every GPU that loads it until the process exits.
+ *  - Calls needing more scratch than that return RA_ERR_WORKSPACE before
+ *    anything runs (use ra_ring_attention with a workspace instead).  The
+ *    default path (bf16 inputs, persistent schedule) needs none.
+ *  - The first call on a device looks up the array's device address on the
+ *    current device (cudaGetSymbolAddress); make that first call before any
+ *    stream capture.  `stream` must belong to the current device.
+ *  - Every call on a device shares the one array and it keeps the last call's
+ *    contents; nothing in it needs to start at zero (every scratch byte the
+ *    call reads it first writes).  Calls whose work overlaps on the GPU (on
+ *    different streams, or from several host threads) race on it: order them.
+ */
+ra_status ra_ring_attention_noalloc(const void* q, const void* k, const void* v, ra_dtype in_dtype,
+                                    int B, int S, int Hq, int D, int n_blocks, int causal,
+                                    ra_partition partition, int gqa_groups,
+                                    void* out, ra_dtype out_dtype, float* lse,
+                                    const ra_options* opts, void* stream);
+
+/* Size in bytes of the fixed scratch array behind ra_ring_attention_noalloc. */
+size_t ra_noalloc_scratch_bytes(void);
+
 /* Reads and clears the device status word (synchronises `stream`).  Returns
  * RA_OK, RA_ERR_TIMEOUT or RA_ERR_DEVICE_BOUNDS, or RA_ERR_CUDA when the read
  * itself fails. */

@@ -14,8 +14,8 @@ HEADER = os.path.join(ROOT, "include", "ra.h")
 
 @pytest.fixture(scope="module")
 def ra():
-    from blockwise_exact_attention_block_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__._build_module().build()
     import blockwise_exact_attention_block_b200 as mod
     return mod
 
