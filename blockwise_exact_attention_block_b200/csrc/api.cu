@@ -161,16 +161,15 @@ void order_segments(AttnArgs& a) {
     }
 }
 
-template <int D>
+template <int D, bool SPLIT>
 ra_status launch_attn_t(const AttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                         cudaStream_t st) {
-  constexpr int NST = D == 128 ? 2 : 4;
-  using SL = AttnSmem<D, NST>;
+  using SL = AttnSmem<D, SPLIT>;
   static int attr_set[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, NST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          SL::kBytes);
     if (e != cudaSuccess) return RA_ERR_CUDA;
     attr_set[dev] = 1;
@@ -178,13 +177,15 @@ ra_status launch_attn_t(const AttnArgs& a, const CUtensorMap& mq, const CUtensor
   const long long grid = static_cast<long long>(a.Hq) * a.B * a.nq * a.nseg * a.seg_tiles;
   if (grid <= 0) return RA_OK;
   if (grid > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
-  attn_fwd_kernel<D, NST><<<static_cast<unsigned>(grid), kAttnThreads, SL::kBytes, st>>>(mq, mk, mv, a);
+  attn_fwd_kernel<D, SPLIT><<<static_cast<unsigned>(grid), kAttnThreads, SL::kBytes, st>>>(mq, mk, mv, a);
   return cuda_status(cudaGetLastError());
 }
 
 ra_status launch_attn(int D, const AttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mk,
                       const CUtensorMap& mv, cudaStream_t st) {
-  return D == 128 ? launch_attn_t<128>(a, mq, mk, mv, st) : launch_attn_t<64>(a, mq, mk, mv, st);
+  if (D == 128)
+    return a.kv_split ? launch_attn_t<128, true>(a, mq, mk, mv, st) : launch_attn_t<128, false>(a, mq, mk, mv, st);
+  return a.kv_split ? launch_attn_t<64, true>(a, mq, mk, mv, st) : launch_attn_t<64, false>(a, mq, mk, mv, st);
 }
 
 int grid_for(long long work, int per_block) {
@@ -282,9 +283,27 @@ bool valid_opts(const ra_options* o) {
   return o->sched >= RA_SCHED_AUTO && o->sched <= RA_SCHED_PERSISTENT;
 }
 
+__global__ void exp2_poly_selftest_kernel(const float* __restrict__ x, float* __restrict__ y, long long npairs) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < npairs;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float a, b;
+    f2_unpack(exp2_poly_x2(f2_pack(x[2 * i], x[2 * i + 1])), a, b);
+    y[2 * i] = a;
+    y[2 * i + 1] = b;
+  }
+}
+
 }  // namespace
 
 extern "C" {
+
+ra_status ra_selftest_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
+  if (n < 0 || (n & 1)) return RA_ERR_INVALID_ARG;
+  if (n == 0) return RA_OK;
+  if (!x || !y) return RA_ERR_INVALID_ARG;
+  exp2_poly_selftest_kernel<<<grid_for(n / 2, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n / 2);
+  return cuda_status(cudaGetLastError());
+}
 
 const char* ra_status_string(ra_status s) {
   switch (s) {

@@ -15,16 +15,21 @@
 // the per-row block_lse; "If this is right": grouped-query attention and the
 // zigzag causal partition; Anthology of the SOTA, SOTA-181: exact attention.
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax of tile A: thread i owns row i of A (TMEM lane i)
 //   warps 4-7  softmax of tile B (same lanes, its own TMEM columns)
-//   warp 8     TMA producer: Q (A and B) once, then K and V into an NST ring
+//   warp 8     TMA producer: Q once, then K and V tiles into their rings
 //   warp 9     TMEM allocator and MMA issuer (one thread):
 //                S_X = Q_X K^T   (SS MMA, fp32 in TMEM)
 //                O_X += P_X V    (TS MMA, P_X bf16 in TMEM over S_X)
 //              issued in the order PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so
 //              the tensor core works on one tile while the other tile's
 //              softmax runs.
+//   warps 10-11 idle (they complete the third warpgroup).
+// Registers: launched at 168 per thread (384 x 168 = 64512); the third
+// warpgroup gives most of its share to the softmax warpgroups
+// (2 x 128 x 216 + 128 x 72 = 64512), so the softmax keeps a whole score
+// row and its exponentials in registers.
 // Tensor memory (512 columns): S_A/P_A [0,128), S_B/P_B [128,256),
 // O_A [256,256+D), O_B [384,384+D).
 //
@@ -54,9 +59,23 @@ constexpr int kBM = 128;        // query rows per tile = TMEM lanes
 constexpr int kCtaRows = 256;   // two tiles per CTA
 constexpr int kBN = 128;        // keys per KV tile
 constexpr int kMaxBlocks = 16;  // ring size limit
-constexpr int kAttnThreads = 320;
+constexpr int kAttnThreads = 384;
+constexpr int kRegsLaunch = 168;  // per thread at launch (__launch_bounds__(384, 1))
+constexpr int kRegsSoftmax = 216;
+constexpr int kRegsOther = 72;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kAttnThreads * kRegsLaunch,
+              "register reallocation must fit in the launch allocation");
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+// Of every 8 exponential pairs in a full tile, this many run on the FMA pipe.
+#ifndef RA_EMU_PAIRS8
+#define RA_EMU_PAIRS8 0
+#endif
+constexpr int kEmuPairs8 = RA_EMU_PAIRS8;
+// 1: exponentials as ex2.approx.f16x2 (two per SFU instruction).
+#ifndef RA_EXP_F16X2
+#define RA_EXP_F16X2 0
+#endif
 
 enum AttnMode : int {
   kModePartial = 0,  // write (block_out, block_lse) into acc rows
@@ -95,17 +114,23 @@ struct AttnArgs {
   signed char seg_order[2 * kMaxBlocks];        // (i * nseg + e) of the query segments, heaviest first
 };
 
-template <int D, int NST>
+// Shared memory: the Q tiles (two for row pairs, one for KV-split), then a
+// ring of K tiles and a ring of V tiles sized to fill the 227 KB: K is
+// needed first (S = Q K^T), so its ring is at least as deep as V's.
+template <int D, bool SPLIT>
 struct AttnSmem {
   static constexpr int kBox = kBM * 64 * 2;  // one TMA box: 128 rows x 64 bf16 (128 B) = 16 KB
   static constexpr int kNBox = D / 64;
   static constexpr int kTile = kBox * kNBox;
-  static constexpr int kQ = 0;                // Q_A, Q_B
-  static constexpr int kK = kQ + 2 * kTile;
-  static constexpr int kV = kK + NST * kTile;
-  static constexpr int kBar = kV + NST * kTile;
-  // barriers: Q, Kfull[NST], Vfull[NST], Kempty[NST], Vempty[NST], Sfull[2], Pfull[2], Odone[2], End
-  static constexpr int kNBar = 1 + 4 * NST + 2 + 2 + 2 + 1;
+  static constexpr int kQTiles = SPLIT ? 1 : 2;
+  static constexpr int kNSK = D == 128 ? 3 : 6;
+  static constexpr int kNSV = D == 128 ? (SPLIT ? 3 : 2) : (SPLIT ? 6 : 4);
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kQTiles * kTile;
+  static constexpr int kV = kK + kNSK * kTile;
+  static constexpr int kBar = kV + kNSV * kTile;
+  // barriers: Q, Kfull[NSK], Kempty[NSK], Vfull[NSV], Vempty[NSV], Sfull[2], Pfull[2], Odone[2], End
+  static constexpr int kNBar = 1 + 2 * kNSK + 2 * kNSV + 2 + 2 + 2 + 1;
   static constexpr int kTmemSlot = kBar + kNBar * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4 + 1024;  // + slack to align the base to 1024
@@ -141,11 +166,13 @@ struct KvCursor {
   int s, e, t, nt;
 };
 
-template <int D, int NST>
+template <int D, bool SPLIT>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
-  using SL = AttnSmem<D, NST>;
+  using SL = AttnSmem<D, SPLIT>;
+  constexpr int NSK = SL::kNSK;
+  constexpr int NSV = SL::kNSV;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_u32 & 1023u)) & 1023u);
@@ -166,7 +193,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int qi = so / a.nseg;
   const Seg qs = a.qseg[qi][so % a.nseg];
   const int hk = h / a.groups;
-  const bool split = a.kv_split != 0;
+  constexpr bool split = SPLIT;
   const int t0 = qt * (split ? kBM : kCtaRows);  // CTA row offset inside the query segment
   int rows[2], last[2], row0[2];                 // per tile: valid rows, last position, first row
   for (int x = 0; x < 2; ++x) {
@@ -204,19 +231,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   auto bar = [&](int i) -> uint32_t { return sb + SL::kBar + 8u * i; };
   const int BQ = 0;
   auto BKF = [&](int s) { return 1 + s; };
-  auto BVF = [&](int s) { return 1 + NST + s; };
-  auto BKE = [&](int s) { return 1 + 2 * NST + s; };
-  auto BVE = [&](int s) { return 1 + 3 * NST + s; };
-  auto BSF = [&](int x) { return 1 + 4 * NST + x; };
-  auto BPF = [&](int x) { return 3 + 4 * NST + x; };
-  auto BOD = [&](int x) { return 5 + 4 * NST + x; };
-  const int BEND = 7 + 4 * NST;
+  auto BKE = [&](int s) { return 1 + NSK + s; };
+  auto BVF = [&](int s) { return 1 + 2 * NSK + s; };
+  auto BVE = [&](int s) { return 1 + 2 * NSK + NSV + s; };
+  auto BSF = [&](int x) { return 1 + 2 * NSK + 2 * NSV + x; };
+  auto BPF = [&](int x) { return 3 + 2 * NSK + 2 * NSV + x; };
+  auto BOD = [&](int x) { return 5 + 2 * NSK + 2 * NSV + x; };
+  const int BEND = 7 + 2 * NSK + 2 * NSV;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SL::kAbort);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < SL::kNBar; ++i) mbar_init(bar(i), 1);
-    mbar_init(bar(BPF(0)), kBM);
-    mbar_init(bar(BPF(1)), kBM);
+    mbar_init(bar(BPF(0)), kBM / 32);  // one arrival per softmax warp
+    mbar_init(bar(BPF(1)), kBM / 32);
     *abort_flag = grid_timed_out() ? 1 : 0;  // after a timeout elsewhere, do no work
     fence_mbar_init();
   }
@@ -227,6 +254,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + SL::kTmemSlot);
   if (*abort_flag) total = 0;
 
+  if (warp >= 8) {
+    // third warpgroup: TMA producer, MMA issuer, two idle warps
+    regs_dec<kRegsOther>();
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && total > 0) {
@@ -241,35 +271,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                       bar(BQ));
       int g = 0;
       bool ok = true;
-      int issued_k[NST], issued_v[NST];
-      for (int s = 0; s < NST; ++s) issued_k[s] = issued_v[s] = -1;
+      int issued_k[NSK], issued_v[NSV];
+      for (int s = 0; s < NSK; ++s) issued_k[s] = -1;
+      for (int s = 0; s < NSV; ++s) issued_v[s] = -1;
       // load order: the CTA's sequence (row pairs), or A0, B0, A1, B1, ... (KV-split)
       for (int g2 = 0; g2 < total && ok; ++g2) {
         int s, e, t;
         locate(split ? ((g2 & 1) ? half + (g2 >> 1) : (g2 >> 1)) : g2, s, e, t);
         const Seg ks = seg_of(s, e);
-        const int st = g % NST;
-        const uint32_t ph = (g / NST) & 1;
-        if (!mbar_wait(bar(BKE(st)), ph ^ 1, abort_flag)) { ok = false; break; }
-        mbar_expect_tx(bar(BKF(st)), SL::kTile);
+        const int sk = g % NSK, sv = g % NSV;
+        if (!mbar_wait(bar(BKE(sk)), ((g / NSK) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        mbar_expect_tx(bar(BKF(sk)), SL::kTile);
         for (int bx = 0; bx < SL::kNBox; ++bx)
-          tma_load_4d(sb + SL::kK + st * SL::kTile + bx * SL::kBox, &tmK, bx * 64, hk, ks.mem + t * kBN, b,
-                      bar(BKF(st)));
-        issued_k[st] = g;
-        if (!mbar_wait(bar(BVE(st)), ph ^ 1, abort_flag)) { ok = false; break; }
-        mbar_expect_tx(bar(BVF(st)), SL::kTile);
+          tma_load_4d(sb + SL::kK + sk * SL::kTile + bx * SL::kBox, &tmK, bx * 64, hk, ks.mem + t * kBN, b,
+                      bar(BKF(sk)));
+        issued_k[sk] = g;
+        if (!mbar_wait(bar(BVE(sv)), ((g / NSV) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        mbar_expect_tx(bar(BVF(sv)), SL::kTile);
         for (int bx = 0; bx < SL::kNBox; ++bx)
-          tma_load_4d(sb + SL::kV + st * SL::kTile + bx * SL::kBox, &tmV, bx * 64, hk, ks.mem + t * kBN, b,
-                      bar(BVF(st)));
-        issued_v[st] = g;
+          tma_load_4d(sb + SL::kV + sv * SL::kTile + bx * SL::kBox, &tmV, bx * 64, hk, ks.mem + t * kBN, b,
+                      bar(BVF(sv)));
+        issued_v[sv] = g;
         ++g;
       }
       if (!ok) {  // let every copy already issued land before shared memory is released
         mbar_drain(bar(BQ), 0);
-        for (int s = 0; s < NST; ++s) {
-          if (issued_k[s] >= 0) mbar_drain(bar(BKF(s)), (issued_k[s] / NST) & 1);
-          if (issued_v[s] >= 0) mbar_drain(bar(BVF(s)), (issued_v[s] / NST) & 1);
-        }
+        for (int s = 0; s < NSK; ++s)
+          if (issued_k[s] >= 0) mbar_drain(bar(BKF(s)), (issued_k[s] / NSK) & 1);
+        for (int s = 0; s < NSV; ++s)
+          if (issued_v[s] >= 0) mbar_drain(bar(BVF(s)), (issued_v[s] / NSV) & 1);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -316,24 +346,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         bool okk = mbar_wait(bar(BQ), 0, abort_flag);
         for (int x = 0; x < 2 && okk; ++x) {
           if (n_of[x] == 0) continue;
-          okk = mbar_wait(bar(BKF(x % NST)), (x / NST) & 1, abort_flag);
+          okk = mbar_wait(bar(BKF(x % NSK)), (x / NSK) & 1, abort_flag);
           if (!okk) break;
           tc_fence_after();
-          issue_s(x, x % NST);
-          tc_commit(bar(BKE(x % NST)));
+          issue_s(x, x % NSK);
+          tc_commit(bar(BKE(x % NSK)));
         }
         for (int j = 0; j < half && okk; ++j) {
           for (int x = 0; x < 2; ++x) {
             if (j >= n_of[x]) continue;
-            const int ld = 2 * j + x, st = ld % NST;
-            if (!mbar_wait(bar(BVF(st)), (ld / NST) & 1, abort_flag)) { okk = false; break; }
-            if (!mbar_wait(bar(BPF(x)), j & 1, abort_flag)) { okk = false; break; }
+            const int ld = 2 * j + x, st = ld % NSV;
+            if (!mbar_wait(bar(BVF(st)), (ld / NSV) & 1, abort_flag)) { okk = false; break; }
+            if (!mbar_wait_spin(bar(BPF(x)), j & 1, abort_flag)) { okk = false; break; }
             tc_fence_after();
             issue_pv(x, st, j > 0);
             tc_commit(bar(BVE(st)));
             if (j + 1 < n_of[x]) {
-              const int ld1 = ld + 2, st1 = ld1 % NST;
-              if (!mbar_wait(bar(BKF(st1)), (ld1 / NST) & 1, abort_flag)) { okk = false; break; }
+              const int ld1 = ld + 2, st1 = ld1 % NSK;
+              if (!mbar_wait(bar(BKF(st1)), (ld1 / NSK) & 1, abort_flag)) { okk = false; break; }
               tc_fence_after();
               issue_s(x, st1);
               tc_commit(bar(BKE(st1)));
@@ -356,7 +386,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_commit(bar(BKE(0)));
       }
       for (int g = 0; ok && g < total; ++g) {
-        const int st = g % NST;
+        const int st = g % NSV;                 // V stage of tile g
+        const int sk1 = (g + 1) % NSK;          // K stage of tile g + 1
         const bool has_next = g + 1 < total;
         KvCursor nxt = cur;
         bool act1[2] = {false, false};
@@ -365,27 +396,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           act1[0] = active_at(nxt, 0);
           act1[1] = active_at(nxt, 1);
         }
-        if (!mbar_wait(bar(BVF(st)), (g / NST) & 1, abort_flag)) break;
+        if (!mbar_wait(bar(BVF(st)), (g / NSV) & 1, abort_flag)) break;
         bool k_ready = false;
         for (int x = 0; x < 2; ++x) {
           if (act[x]) {
-            if (!mbar_wait(bar(BPF(x)), cnt[x] & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait_spin(bar(BPF(x)), cnt[x] & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             issue_pv(x, st, cnt[x] > 0);
             ++cnt[x];
           }
           if (act1[x]) {
             if (!k_ready) {
-              if (!mbar_wait(bar(BKF((g + 1) % NST)), ((g + 1) / NST) & 1, abort_flag)) { ok = false; break; }
+              if (!mbar_wait(bar(BKF(sk1)), ((g + 1) / NSK) & 1, abort_flag)) { ok = false; break; }
               tc_fence_after();
               k_ready = true;
             }
-            issue_s(x, (g + 1) % NST);
+            issue_s(x, sk1);
           }
         }
         if (!ok) break;
         tc_commit(bar(BVE(st)));
-        if (has_next) tc_commit(bar(BKE((g + 1) % NST)));
+        if (has_next) tc_commit(bar(BKE(sk1)));
         cur = nxt;
         act[0] = act1[0];
         act[1] = act1[1];
@@ -395,8 +426,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_drain(bar(BEND), 0);
       }
     }
+  }
   } else {
     // ------------------------------------------------------------- softmax
+    regs_inc<kRegsSoftmax>();
     const int x = warp >> 2;            // tile A (0) or B (1)
     const int row = threadIdx.x & 127;  // row inside the tile = TMEM lane
     const bool valid = row < rows[x];
@@ -424,23 +457,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           uint32_t sv[kBN];
           tmem_ld128_wait(tS, sv);
           const int cnt = lim - t * kBN;
-          // row maximum with 8 independent chains (short dependency paths)
-          float mx8[8];
+          const bool full = cnt >= kBN;
+          if (__any_sync(0xffffffffu, !full)) {  // warp-uniform: full tiles skip the masking code
 #pragma unroll
-          for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
-          if (cnt < kBN) {
-#pragma unroll
-            for (int j = 0; j < kBN; ++j) {
-              const float v = j < cnt ? __uint_as_float(sv[j]) : -INFINITY;
-              sv[j] = __float_as_uint(v);
-              mx8[j & 7] = fmaxf(mx8[j & 7], v);
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < kBN; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], __uint_as_float(sv[j]));
+            for (int j = 0; j < kBN; ++j) sv[j] = j < cnt ? sv[j] : __float_as_uint(-INFINITY);
           }
-          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          // row maximum: 3-input max, 8 independent chains of depth 8
+          float m8[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) m8[q] = fmaxf(__uint_as_float(sv[2 * q]), __uint_as_float(sv[2 * q + 1]));
+#pragma unroll
+          for (int j = 16; j < kBN; j += 16)
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              m8[q] = fmax3(m8[q], __uint_as_float(sv[j + 2 * q]), __uint_as_float(sv[j + 2 * q + 1]));
+          const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
           const float mt = mx * sl2;
           float alpha = 1.f;
           bool resc = false;
@@ -452,107 +483,130 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             m_use = mt;
           }
           const float base = (m_use == -INFINITY) ? 0.f : m_use;
-          float ps8[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) ps8[i] = 0.f;
+          const uint64_t sl2x2 = f2_pack(sl2, sl2);
+          const uint64_t nbase2 = f2_pack(-base, -base);
+          // Exponentials: the SFU does ex2 for most pairs; in tiles without
+          // masked entries (the whole warp), kEmuPairs of every 16 pairs run
+          // on the FMA pipe instead (exp2_poly_x2), splitting the load.
+          const bool emu = __all_sync(0xffffffffu, full);
+          uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
           for (int ch = 0; ch < kBN / 32; ++ch) {  // 32 scores -> 16 packed bf16 pairs per store
             uint32_t pk[16];
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const float p0 = fast_exp2(fmaf(__uint_as_float(sv[ch * 32 + j]), sl2, -base));
-              const float p1 = fast_exp2(fmaf(__uint_as_float(sv[ch * 32 + j + 1]), sl2, -base));
-              ps8[(j >> 1) & 7] += p0 + p1;
-              pk[j / 2] = pack_bf16x2(p0, p1);
+            for (int pp = 0; pp < 16; ++pp) {
+              const int j = ch * 32 + 2 * pp;
+              const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), sl2x2, nbase2);
+              uint64_t e2;
+              if (emu && (pp % 8) < kEmuPairs8) {
+                e2 = exp2_poly_x2(x2);
+              } else {
+                float x0, x1;
+                f2_unpack(x2, x0, x1);
+#if RA_EXP_F16X2
+                float q0, q1;
+                exp2_f16x2(x0, x1, q0, q1);
+                e2 = f2_pack(q0, q1);
+#else
+                e2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
+#endif
+              }
+              acc[pp & 3] = f2_add(acc[pp & 3], e2);
+              float p0, p1;
+              f2_unpack(e2, p0, p1);
+              pk[pp] = pack_bf16x2(p0, p1);
             }
             tmem_st16(tS + ch * 16, pk);
           }
-          const float psum = ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
-          l_sum = l_sum * alpha + psum;
+          const uint64_t acc2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+          float ps0, ps1;
+          f2_unpack(acc2, ps0, ps1);
+          l_sum = l_sum * alpha + (ps0 + ps1);
           tmem_wait_st();
-          if (c > 0) {
-            // O may only be touched once the previous P V product has landed.
-            ok = mbar_wait(bar(BOD(x)), (c - 1) & 1, abort_flag);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            if (__any_sync(0xffffffffu, resc)) {
-              tc_fence_after();
+          // O of this tile is stable here: S_X(c) was committed after the
+          // P V product of tile c-1, so its completion implies that one's.
+          if (c > 0 && __any_sync(0xffffffffu, resc)) {
+            tc_fence_after();
 #pragma unroll
-              for (int q = 0; q < D / 32; ++q) {
-                uint32_t ov[32];
-                tmem_ld32_wait(tO + 32 * q, ov);
+            for (int q = 0; q < D / 32; ++q) {
+              uint32_t ov[32];
+              tmem_ld32_wait(tO + 32 * q, ov);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                tmem_st32(tO + 32 * q, ov);
-              }
-              tmem_wait_st();
+              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+              tmem_st32(tO + 32 * q, ov);
             }
+            tmem_wait_st();
           }
           tc_fence_before();
-          mbar_arrive(bar(BPF(x)));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BPF(x)));
           ++c;
         }
       }
 
     // ------------------------------------------------------------ epilogue
+    // Each tile's rows are normalised (and, in KV-split mode, stitched with
+    // the other half by the merge rule) into a staging buffer in shared
+    // memory, then every warp writes its 32 rows to HBM as whole, coalesced
+    // rows.  The K/V rings hold the staging buffers: they are idle once the
+    // last P V product of both tiles has landed (the barrier below).
     if (ok && c > 0) {
       ok = mbar_wait(bar(BOD(x)), (c - 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
     }
-    if (split) {
-      // Stitch B's partial into A's with the merge rule.  B writes its
-      // normalised row and lse to shared memory (the K/V ring is idle once
-      // both tiles' last P V product has landed), then A merges.
-      float* xo = reinterpret_cast<float*>(smem + SL::kK);  // [128][D + 4]
-      float* xl = xo + kBM * (D + 4);                        // [128]
-      named_barrier_sync(1, 256);  // both tiles' MMAs are complete
-      fence_proxy_async_smem();
-      if (x == 1) {
-        const bool has = ok && l_sum > 0.f;
-        const float inv = has ? 1.f / l_sum : 0.f;
-        xl[row] = has ? (m_use + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
-        if (c > 0) tc_fence_after();
+    constexpr int kStride = D + 4;                       // floats per staged row (bank-conflict-free)
+    constexpr int kStageFloats = kBM * kStride + kBM;    // rows, then one float per row
+    static_assert(2 * kStageFloats * 4 <= SL::kBar - SL::kK, "staging buffers must fit in the K/V rings");
+    float* stage = reinterpret_cast<float*>(smem + SL::kK) + x * kStageFloats;
+    float* stage_w = stage + kBM * kStride;              // per-row lse (B, KV-split) or merge weight
+    named_barrier_sync(1, 256);  // both tiles' MMAs are complete: the rings are free
+    fence_proxy_async_smem();
+    if (split && x == 1) {
+      // B's normalised partial and its lse, for A to merge
+      const bool has = ok && l_sum > 0.f;
+      const float inv = has ? 1.f / l_sum : 0.f;
+      stage_w[row] = has ? (m_use + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
+      if (ok && c > 0) tc_fence_after();
 #pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
-          uint32_t ov[32];
-          if (ok && c > 0) tmem_ld32_wait(tO + 32 * q, ov);
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t ov[32];
+        if (ok && c > 0) tmem_ld32_wait(tO + 32 * q, ov);
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(xo + row * (D + 4) + 32 * q + i) =
-                make_float4(has ? __uint_as_float(ov[i]) * inv : 0.f, has ? __uint_as_float(ov[i + 1]) * inv : 0.f,
-                            has ? __uint_as_float(ov[i + 2]) * inv : 0.f, has ? __uint_as_float(ov[i + 3]) * inv : 0.f);
-        }
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(stage + row * kStride + 32 * q + i) =
+              make_float4(has ? __uint_as_float(ov[i]) * inv : 0.f, has ? __uint_as_float(ov[i + 1]) * inv : 0.f,
+                          has ? __uint_as_float(ov[i + 2]) * inv : 0.f, has ? __uint_as_float(ov[i + 3]) * inv : 0.f);
       }
-      named_barrier_sync(1, 256);
     }
+    if (split) named_barrier_sync(1, 256);
     // rows are written by every tile in row-pair mode, by A alone in KV-split mode
-    if ((ok || total == 0) && !(split && x == 1)) {
+    const bool writer = (ok || total == 0) && !(split && x == 1);
+    const long long row_base = a.mode == kModeFinal ? static_cast<long long>(b) * a.S + qs.pos + row0[x]
+                                                    : static_cast<long long>(b) * a.acc_brows + qs.mem + row0[x];
+    if (writer) {
       const bool has = l_sum > 0.f;
       const float inv = has ? 1.f / l_sum : 0.f;
       float row_lse = has ? (m_use + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
+      const float* bstage = stage + kStageFloats;  // B's region (KV-split)
       MergeWeights mwb;  // KV-split: weight of B's partial in this row
       mwb.w = 0.f;
       if (split) {
-        mwb = merge_weights(row_lse, reinterpret_cast<float*>(smem + SL::kK)[kBM * (D + 4) + row]);
+        mwb = merge_weights(row_lse, bstage[kBM * kStride + row]);
         row_lse = mwb.lse;
       }
-      if (c > 0) tc_fence_after();
-      long long o_off = 0;
-      float* lse_ptr = nullptr;
-      if (a.mode == kModeFinal) {
-        const long long orow = static_cast<long long>(b) * a.S + qpos;
-        o_off = (orow * a.Hq + h) * D;
-        lse_ptr = a.lse + orow * a.Hq + h;
-      } else {
-        const long long prow = static_cast<long long>(b) * a.acc_brows + qs.mem + row0[x] + row;
-        o_off = (prow * a.Hq + h) * D;
-        lse_ptr = a.acc_lse + prow * a.Hq + h;
+      float* lse_ptr = (a.mode == kModeFinal ? a.lse : a.acc_lse) + (row_base + row) * a.Hq + h;
+      float w = 1.f;
+      if (valid) {
+        if (a.mode == kModeMerge) {
+          const MergeWeights mw = merge_weights(*lse_ptr, row_lse);
+          *lse_ptr = mw.lse;
+          w = mw.w;
+        } else {
+          *lse_ptr = row_lse;
+        }
       }
-      MergeWeights mw;
-      mw.w = 1.f;
-      mw.lse = row_lse;
-      if (valid && a.mode == kModeMerge) mw = merge_weights(*lse_ptr, row_lse);
-      if (valid) *lse_ptr = mw.lse;
+      stage_w[row] = w;
+      if (c > 0) tc_fence_after();
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {
         uint32_t ov[32];
@@ -560,39 +614,53 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(has ? __uint_as_float(ov[i]) * inv : 0.f);
         if (split && mwb.w != 0.f) {
-          const float* xb = reinterpret_cast<const float*>(smem + SL::kK) + row * (D + 4) + 32 * q;
+          const float* xb = bstage + row * kStride + 32 * q;
 #pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(merge_out(__uint_as_float(ov[i]), xb[i], mwb.w));
         }
-        if (!valid) continue;
-        if (a.mode == kModeFinal && a.out_bf16) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + o_off + 32 * q);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(ov[8 * i + 0]), __uint_as_float(ov[8 * i + 1]));
-            w.y = pack_bf16x2(__uint_as_float(ov[8 * i + 2]), __uint_as_float(ov[8 * i + 3]));
-            w.z = pack_bf16x2(__uint_as_float(ov[8 * i + 4]), __uint_as_float(ov[8 * i + 5]));
-            w.w = pack_bf16x2(__uint_as_float(ov[8 * i + 6]), __uint_as_float(ov[8 * i + 7]));
-            dst[i] = w;
-          }
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(stage + row * kStride + 32 * q + i) =
+              make_float4(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1]), __uint_as_float(ov[i + 2]),
+                          __uint_as_float(ov[i + 3]));
+      }
+      __syncwarp();
+      // this warp's 32 rows, each written as one contiguous run
+      const int wr0 = (warp & 3) * 32;
+      const bool bf16_out = a.mode == kModeFinal && a.out_bf16;
+      constexpr int kLanesF32 = D / 4;   // float4 per row
+      constexpr int kLanesB16 = D / 8;   // 8 bf16 (16 B) per lane
+      const int lpr = bf16_out ? kLanesB16 : kLanesF32;
+      const int rpi = 32 / lpr;          // rows per warp instruction
+      const int ci = lane % lpr;
+      for (int r0 = 0; r0 < 32; r0 += rpi) {
+        const int r = wr0 + r0 + lane / lpr;
+        if (r >= rows[x]) continue;
+        const long long grow = (row_base + r) * a.Hq + h;
+        const float* src = stage + r * kStride;
+        if (bf16_out) {
+          const float4 lo = *reinterpret_cast<const float4*>(src + 8 * ci);
+          const float4 hi = *reinterpret_cast<const float4*>(src + 8 * ci + 4);
+          uint4 o;
+          o.x = pack_bf16x2(lo.x, lo.y);
+          o.y = pack_bf16x2(lo.z, lo.w);
+          o.z = pack_bf16x2(hi.x, hi.y);
+          o.w = pack_bf16x2(hi.z, hi.w);
+          reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + grow * D)[ci] = o;
         } else {
-          float4* dst =
-              reinterpret_cast<float4*>((a.mode == kModeFinal ? static_cast<float*>(a.out) : a.acc_out) + o_off + 32 * q);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float4 v = make_float4(__uint_as_float(ov[4 * i]), __uint_as_float(ov[4 * i + 1]),
-                                   __uint_as_float(ov[4 * i + 2]), __uint_as_float(ov[4 * i + 3]));
-            if (a.mode == kModeMerge) {
-              if (mw.w == 0.f) continue;
-              const float4 old = dst[i];
-              v.x = merge_out(old.x, v.x, mw.w);
-              v.y = merge_out(old.y, v.y, mw.w);
-              v.z = merge_out(old.z, v.z, mw.w);
-              v.w = merge_out(old.w, v.w, mw.w);
-            }
-            dst[i] = v;
+          float4 v = *reinterpret_cast<const float4*>(src + 4 * ci);
+          float4* dst = reinterpret_cast<float4*>((a.mode == kModeFinal ? static_cast<float*>(a.out) : a.acc_out) +
+                                                  grow * D) + ci;
+          if (a.mode == kModeMerge) {
+            const float wr = stage_w[r];
+            if (wr == 0.f) continue;
+            const float4 old = *dst;
+            v.x = merge_out(old.x, v.x, wr);
+            v.y = merge_out(old.y, v.y, wr);
+            v.z = merge_out(old.z, v.z, wr);
+            v.w = merge_out(old.w, v.w, wr);
           }
+          *dst = v;
         }
       }
     }

@@ -57,6 +57,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // True once any CTA has recorded a timeout: the rest of the grid then stops
 // waiting at once instead of each CTA running out its own limit.
 __device__ __forceinline__ bool grid_timed_out() {
@@ -80,6 +92,28 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       set_status(RA_ERR_TIMEOUT);
       *abort = 1;
       return false;
+    }
+  }
+}
+
+// Same contract as mbar_wait, but polls without letting the thread be
+// suspended, for the single MMA-issuing thread whose reaction time is on the
+// critical path.
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, volatile int* abort) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((it & 255) == 0) {
+      if (*abort || grid_timed_out()) {
+        *abort = 1;
+        return false;
+      }
+      if (clock64() - t0 > kWaitLimitCycles) {
+        set_status(RA_ERR_TIMEOUT);
+        *abort = 1;
+        return false;
+      }
     }
   }
 }
@@ -111,6 +145,16 @@ __device__ __forceinline__ void named_barrier_sync(int id, int count) {
 // accesses before its later generic ones.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Warpgroup-wide register reallocation (all 128 threads of the warpgroup).
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // --------------------------------------------------------------- tcgen05
@@ -228,6 +272,76 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// ------------------------------------------------------ packed fp32 pairs
+// Blackwell executes these as one instruction on two fp32 lanes.
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair of fp32 values, on the FMA and integer pipes (no SFU).
+// Range reduction: x = j + f with j the nearest integer (added to 1.5 * 2^23
+// so the rounding is done by the fp32 add itself) and f in [-0.5, 0.5];
+// 2^f from a degree-4 polynomial fitted here to minimise the relative error
+// on [-0.5, 0.5] (fit_exp2_poly.py; max relative error 2.7e-6 in fp32);
+// 2^j is added into the exponent field: with t = x + 1.5 * 2^23,
+// bits(result) = bits(p) + (bits(t) << 23) (mod 2^32).  Inputs are clamped
+// to [-125, 126] so the exponent never leaves the normal range.
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  x0 = fminf(fmaxf(x0, -125.f), 126.f);
+  x1 = fminf(fmaxf(x1, -125.f), 126.f);
+  const uint64_t xc = f2_pack(x0, x1);
+  const uint64_t t = f2_add(xc, f2_pack(kMagic, kMagic));
+  const uint64_t r = f2_add(t, f2_pack(-kMagic, -kMagic));       // nearest integers
+  const uint64_t f = f2_fma(r, f2_pack(-1.f, -1.f), xc);          // x - j, exact
+  uint64_t p = f2_fma(f, f2_pack(9.570068680e-03f, 9.570068680e-03f), f2_pack(5.591780692e-02f, 5.591780692e-02f));
+  p = f2_fma(p, f, f2_pack(2.402474433e-01f, 2.402474433e-01f));
+  p = f2_fma(p, f, f2_pack(6.931218505e-01f, 6.931218505e-01f));
+  p = f2_fma(p, f, f2_pack(9.999992847e-01f, 9.999992847e-01f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  const uint32_t r0 = __float_as_uint(p0) + (__float_as_uint(t0) << 23);
+  const uint32_t r1 = __float_as_uint(p1) + (__float_as_uint(t1) << 23);
+  return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
+}
+
+// 2^x for a pair on the SFU in half precision: both values are rounded to
+// fp16 (11-bit significand), exponentiated by one ex2.approx.f16x2, and
+// widened back to fp32.  Results below 2^-24 flush to 0; x = -inf gives 0.
+__device__ __forceinline__ void exp2_f16x2(float x0, float x1, float& p0, float& p1) {
+  uint32_t h2, e2;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h2) : "f"(x1), "f"(x0));
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(e2) : "r"(h2));
+  asm("{.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tcvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;}"
+      : "=f"(p0), "=f"(p1)
+      : "r"(e2));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
