@@ -48,7 +48,7 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     p.add_argument("--sched", default="auto", choices=["auto", "persistent", "fused", "unfused"])
     p.add_argument("--order", default="ring", choices=["ring", "tokenring"])
-    p.add_argument("--tiling", default="auto", choices=["auto", "row_pairs", "kv_split"])
+    p.add_argument("--tiling", default="auto", choices=["auto", "row_pairs", "kv_split", "cluster2"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")

@@ -49,7 +49,7 @@ class ra_options(ctypes.Structure):
                 ("attn_event_end", ctypes.c_void_p), ("tiling", ctypes.c_int)]
 
 
-TILINGS = {"auto": 0, "row_pairs": 1, "kv_split": 2}
+TILINGS = {"auto": 0, "row_pairs": 1, "kv_split": 2, "cluster2": 3}
 
 
 _vp, _i, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t

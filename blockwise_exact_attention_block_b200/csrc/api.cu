@@ -103,13 +103,16 @@ ra_status check_geom(int B, int S, int n, int Hq, int Hkv, int D, int partition,
 inline int seg_len_of(const Geom& g) { return g.zigzag ? g.c : g.L; }
 
 // Row pairs (256 query rows per CTA, shared K/V loads) unless that leaves
-// fewer than two CTAs per SM; then KV-split (128 rows per CTA, the KV tiles
-// halved between the two tiles and merged on chip), which doubles the CTA
-// count and halves the longest CTA.
+// fewer than two CTAs per SM; then KV-split (128 rows per CTA, the CTA's KV
+// tiles halved between its two warpgroups and merged on chip), which doubles
+// the CTA count and halves the longest CTA.  The two-CTA cluster split is
+// available on request (measured slower for the small grids that need it).
 void choose_tiling(const Geom& g, AttnArgs& a, ra_tiling tiling) {
   const int len = seg_len_of(g);
   const long long pairs = static_cast<long long>(a.Hq) * a.B * a.nq * a.nseg * ((len + kCtaRows - 1) / kCtaRows);
-  a.kv_split = tiling == RA_TILING_KV_SPLIT || (tiling == RA_TILING_AUTO && pairs < 2LL * sm_count()) ? 1 : 0;
+  if (tiling == RA_TILING_AUTO) tiling = pairs < 2LL * sm_count() ? RA_TILING_KV_SPLIT : RA_TILING_ROW_PAIRS;
+  a.kv_split = tiling == RA_TILING_KV_SPLIT ? 1 : 0;
+  a.cluster = tiling == RA_TILING_CLUSTER2 ? 2 : 1;
   a.seg_tiles = (len + (a.kv_split ? kBM : kCtaRows) - 1) / (a.kv_split ? kBM : kCtaRows);
 }
 
@@ -174,11 +177,27 @@ ra_status launch_attn_t(const AttnArgs& a, const CUtensorMap& mq, const CUtensor
     if (e != cudaSuccess) return RA_ERR_CUDA;
     attr_set[dev] = 1;
   }
-  const long long grid = static_cast<long long>(a.Hq) * a.B * a.nq * a.nseg * a.seg_tiles;
+  const long long grid = static_cast<long long>(a.Hq) * a.B * a.nq * a.nseg * a.seg_tiles * a.cluster;
   if (grid <= 0) return RA_OK;
   if (grid > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
-  attn_fwd_kernel<D, SPLIT><<<static_cast<unsigned>(grid), kAttnThreads, SL::kBytes, st>>>(mq, mk, mv, a);
-  return cuda_status(cudaGetLastError());
+  if (a.cluster == 1) {
+    attn_fwd_kernel<D, SPLIT><<<static_cast<unsigned>(grid), kAttnThreads, SL::kBytes, st>>>(mq, mk, mv, a);
+    return cuda_status(cudaGetLastError());
+  }
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kAttnThreads, 1, 1);
+  cfg.dynamicSmemBytes = SL::kBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(a.cluster);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, attn_fwd_kernel<D, SPLIT>, mq, mk, mv, a));
 }
 
 ra_status launch_attn(int D, const AttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mk,
@@ -279,7 +298,7 @@ Plan make_plan(const Geom& g, ra_dtype in_dtype, ra_dtype out_dtype, const ra_op
 bool valid_opts(const ra_options* o) {
   if (!o) return true;
   if (o->order != RA_ORDER_RING && o->order != RA_ORDER_TOKENRING) return false;
-  if (o->tiling < RA_TILING_AUTO || o->tiling > RA_TILING_KV_SPLIT) return false;
+  if (o->tiling < RA_TILING_AUTO || o->tiling > RA_TILING_CLUSTER2) return false;
   return o->sched >= RA_SCHED_AUTO && o->sched <= RA_SCHED_PERSISTENT;
 }
 

@@ -8,6 +8,10 @@
 // the same 128 rows; A takes the first half of the KV tiles, B the second
 // half, and the two partial results are stitched on chip with the merge rule
 // (the rule the method uses between blocks, applied inside one block).
+// Cluster mode (row pairs, still too few CTAs): two CTAs of a thread-block
+// cluster run the same 256 rows over the two halves of the KV tiles; each
+// stages its partial rows in shared memory, and CTA r finalises tile r by
+// reading the peer's partial through distributed shared memory and merging.
 //
 // TokenRing review (pith.science, arXiv 2412.20501), "What carries the
 // argument" / "Core claim": the flash-attention kernel that yields, for one
@@ -98,6 +102,7 @@ struct AttnArgs {
   int nseg;               // segments per block: 1 (contiguous) or 2 (zigzag)
   int seg_tiles;          // CTAs per query segment: ceil(len / 256), or ceil(len / 128) in KV-split mode
   int kv_split;           // 1: KV-split mode (see the top of this file)
+  int cluster;            // CTAs per cluster sharing one row pair (1 or 2; row pairs only)
   float scale_log2;       // log2(e) / sqrt(D)
   int mode;               // AttnMode
   // kModePartial / kModeMerge: row = b * acc_brows + memory row of the query
@@ -183,7 +188,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   // ---- tile decode: heads fastest (heads of one KV group share K/V in L2),
   // then batch, then query tiles in decreasing position (heaviest first).
-  int idx = blockIdx.x;
+  const int crank = a.cluster > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  int idx = blockIdx.x / a.cluster;
   const int h = idx % a.Hq;
   idx /= a.Hq;
   const int b = idx % a.B;
@@ -195,24 +201,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int hk = h / a.groups;
   constexpr bool split = SPLIT;
   const int t0 = qt * (split ? kBM : kCtaRows);  // CTA row offset inside the query segment
-  int rows[2], last[2], row0[2];                 // per tile: valid rows, last position, first row
-  for (int x = 0; x < 2; ++x) {
-    row0[x] = t0 + (split ? 0 : x * kBM);
-    rows[x] = min(max(qs.len - row0[x], 0), kBM);
-    last[x] = rows[x] > 0 ? qs.pos + row0[x] + rows[x] - 1 : -1;
-  }
-  const int last_u = max(last[0], last[1]);  // the CTA's last row: its KV range covers both tiles
+  // per tile X (A = 0, B = 1): first row in the segment, valid rows, last position
+  const int row0_a = t0, row0_b = t0 + (split ? 0 : kBM);
+  const int rows_a = min(max(qs.len - row0_a, 0), kBM), rows_b = min(max(qs.len - row0_b, 0), kBM);
+  const int last_a = rows_a > 0 ? qs.pos + row0_a + rows_a - 1 : -1;
+  const int last_b = rows_b > 0 ? qs.pos + row0_b + rows_b - 1 : -1;
+  const int last_u = max(last_a, last_b);  // the CTA's last row: its KV range covers both tiles
   auto seg_of = [&](int s_, int e_) -> const Seg& { return a.kvseg[a.kv_list[qi][s_]][e_]; };
 
   int total = 0;
   for (int s = 0; s < a.nkv; ++s)
     for (int e = 0; e < a.nseg; ++e) total += tiles_for(a, seg_of(s, e), last_u);
+  // this CTA's share [lo, hi) of the sequence (the cluster splits it in equal parts)
+  const int lo = crank * total / a.cluster;
+  const int hi = (crank + 1) * total / a.cluster;
+  int work = hi - lo;
   // Tile x's share of the CTA's KV tiles.  u = index in the CTA's sequence,
   // t = index inside the segment.  KV-split: A takes [0, half), B [half, total).
   const int half = (total + 1) / 2;
   auto active = [&](int x, int u, int t, const Seg& ks) -> bool {
     if (split) return x == 0 ? u < half : u >= half;
-    return t < tiles_for(a, ks, last[x]);
+    return u >= lo && u < hi && t < tiles_for(a, ks, x ? last_b : last_a);
   };
   // The segment and in-segment tile of the CTA's u-th KV tile.
   auto locate = [&](int u, int& s_, int& e_, int& t_) {
@@ -252,14 +261,79 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + SL::kTmemSlot);
-  if (*abort_flag) total = 0;
+  if (*abort_flag) work = 0;
+
+  // ---- staging buffers and the final row write (see the epilogue)
+  constexpr int kStride = D + 4;                        // floats per staged row (bank-conflict-free)
+  constexpr int kStageFloats = kBM * kStride + 2 * kBM; // rows, then per-row weight and lse
+  static_assert(2 * kStageFloats * 4 <= SL::kBar - SL::kK, "staging buffers must fit in the K/V rings");
+  auto stage_of = [&](int x) { return reinterpret_cast<float*>(smem + SL::kK) + x * kStageFloats; };
+  // Writes tile x's staged rows: the lse of each valid row (merged into the
+  // running state in epilogue-fused mode) and then, per warp, its 32 rows as
+  // contiguous runs.  Called by the 4 warps of tile x.
+  auto commit_rows = [&](int x) {
+    float* stage = stage_of(x);
+    float* stage_w = stage + kBM * kStride;
+    const float* stage_l = stage_w + kBM;
+    const int row = threadIdx.x & 127;
+    const int my_row0 = x ? row0_b : row0_a;
+    const int my_rows = x ? rows_b : rows_a;
+    const long long row_base = a.mode == kModeFinal ? static_cast<long long>(b) * a.S + qs.pos + my_row0
+                                                    : static_cast<long long>(b) * a.acc_brows + qs.mem + my_row0;
+    if (row < my_rows) {
+      float* lse_ptr = (a.mode == kModeFinal ? a.lse : a.acc_lse) + (row_base + row) * a.Hq + h;
+      if (a.mode == kModeMerge) {
+        const MergeWeights mw = merge_weights(*lse_ptr, stage_l[row]);
+        *lse_ptr = mw.lse;
+        stage_w[row] = mw.w;
+      } else {
+        *lse_ptr = stage_l[row];
+      }
+    }
+    __syncwarp();
+    const int wr0 = (warp & 3) * 32;
+    const bool bf16_out = a.mode == kModeFinal && a.out_bf16;
+    const int lpr = bf16_out ? D / 8 : D / 4;  // lanes per row: 16 B per lane
+    const int rpi = 32 / lpr;                  // rows per warp instruction
+    const int ci = lane % lpr;
+    for (int r0 = 0; r0 < 32; r0 += rpi) {
+      const int r = wr0 + r0 + lane / lpr;
+      if (r >= my_rows) continue;
+      const long long grow = (row_base + r) * a.Hq + h;
+      const float* src = stage + r * kStride;
+      if (bf16_out) {
+        const float4 lo4 = *reinterpret_cast<const float4*>(src + 8 * ci);
+        const float4 hi4 = *reinterpret_cast<const float4*>(src + 8 * ci + 4);
+        uint4 o;
+        o.x = pack_bf16x2(lo4.x, lo4.y);
+        o.y = pack_bf16x2(lo4.z, lo4.w);
+        o.z = pack_bf16x2(hi4.x, hi4.y);
+        o.w = pack_bf16x2(hi4.z, hi4.w);
+        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + grow * D)[ci] = o;
+      } else {
+        float4 v = *reinterpret_cast<const float4*>(src + 4 * ci);
+        float4* dst = reinterpret_cast<float4*>((a.mode == kModeFinal ? static_cast<float*>(a.out) : a.acc_out) +
+                                                grow * D) + ci;
+        if (a.mode == kModeMerge) {
+          const float wr = stage_w[r];
+          if (wr == 0.f) continue;
+          const float4 old = *dst;
+          v.x = merge_out(old.x, v.x, wr);
+          v.y = merge_out(old.y, v.y, wr);
+          v.z = merge_out(old.z, v.z, wr);
+          v.w = merge_out(old.w, v.w, wr);
+        }
+        *dst = v;
+      }
+    }
+  };
 
   if (warp >= 8) {
     // third warpgroup: TMA producer, MMA issuer, two idle warps
     regs_dec<kRegsOther>();
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && total > 0) {
+    if (lane == 0 && work > 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -267,7 +341,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_expect_tx(bar(BQ), nqt * SL::kTile);
       for (int x = 0; x < nqt; ++x)
         for (int bx = 0; bx < SL::kNBox; ++bx)
-          tma_load_4d(sb + SL::kQ + x * SL::kTile + bx * SL::kBox, &tmQ, bx * 64, h, qs.mem + row0[x], b,
+          tma_load_4d(sb + SL::kQ + x * SL::kTile + bx * SL::kBox, &tmQ, bx * 64, h, qs.mem + (x ? row0_b : row0_a), b,
                       bar(BQ));
       int g = 0;
       bool ok = true;
@@ -275,9 +349,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int s = 0; s < NSK; ++s) issued_k[s] = -1;
       for (int s = 0; s < NSV; ++s) issued_v[s] = -1;
       // load order: the CTA's sequence (row pairs), or A0, B0, A1, B1, ... (KV-split)
-      for (int g2 = 0; g2 < total && ok; ++g2) {
+      for (int g2 = 0; g2 < work && ok; ++g2) {
         int s, e, t;
-        locate(split ? ((g2 & 1) ? half + (g2 >> 1) : (g2 >> 1)) : g2, s, e, t);
+        locate(split ? ((g2 & 1) ? half + (g2 >> 1) : (g2 >> 1)) : lo + g2, s, e, t);
         const Seg ks = seg_of(s, e);
         const int sk = g % NSK, sv = g % NSV;
         if (!mbar_wait(bar(BKE(sk)), ((g / NSK) & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -304,7 +378,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------- MMA issue
-    if (lane == 0 && total > 0) {
+    if (lane == 0 && work > 0) {
       constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, D, true);
       const int qslot1 = split ? 0 : 1;  // Q tile of B
@@ -338,7 +412,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           k.nt = k.s < a.nkv ? tiles_for(a, seg_of(k.s, k.e), last_u) : 0;
         }
       };
-      auto active_at = [&](const KvCursor& k, int x) { return k.t < tiles_for(a, seg_of(k.s, k.e), last[x]); };
+      auto active_at = [&](const KvCursor& k, int x) {
+        return k.t < tiles_for(a, seg_of(k.s, k.e), x ? last_b : last_a);
+      };
 
       if (split) {
         // KV-split: tile x's i-th KV tile is load 2i + x (A has half, B total - half tiles)
@@ -373,8 +449,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_commit(bar(BEND));
         mbar_drain(bar(BEND), 0);
       } else {
-      KvCursor cur = {0, 0, -1, tiles_for(a, seg_of(0, 0), last_u)};
-      advance(cur);  // first existing tile (total > 0, so there is one)
+      KvCursor cur;
+      locate(lo, cur.s, cur.e, cur.t);  // this CTA's first tile (work > 0, so it exists)
+      cur.nt = tiles_for(a, seg_of(cur.s, cur.e), last_u);
       bool act[2] = {active_at(cur, 0), active_at(cur, 1)};
       int cnt[2] = {0, 0};  // P V products issued per tile
       bool ok = mbar_wait(bar(BQ), 0, abort_flag);
@@ -385,10 +462,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (act[x]) issue_s(x, 0);
         tc_commit(bar(BKE(0)));
       }
-      for (int g = 0; ok && g < total; ++g) {
+      for (int g = 0; ok && g < work; ++g) {
         const int st = g % NSV;                 // V stage of tile g
         const int sk1 = (g + 1) % NSK;          // K stage of tile g + 1
-        const bool has_next = g + 1 < total;
+        const bool has_next = g + 1 < work;
         KvCursor nxt = cur;
         bool act1[2] = {false, false};
         if (has_next) {
@@ -432,15 +509,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     regs_inc<kRegsSoftmax>();
     const int x = warp >> 2;            // tile A (0) or B (1)
     const int row = threadIdx.x & 127;  // row inside the tile = TMEM lane
-    const bool valid = row < rows[x];
-    const int qpos = valid ? qs.pos + row0[x] + row : -1;
+    const int my_row0 = x ? row0_b : row0_a;
+    const int my_rows = x ? rows_b : rows_a;
+    const bool valid = row < my_rows;
+    const int qpos = valid ? qs.pos + my_row0 + row : -1;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + x * 128;
     const uint32_t tO = tmem + lane_base + 256 + x * 128;
     const float sl2 = a.scale_log2;
     float m_use = -INFINITY;
     float l_sum = 0.f;
-    bool ok = total > 0;
+    bool ok = work > 0;
     int c = 0;  // tiles processed by this tile's softmax
     int u = 0;  // position in the CTA's KV sequence
     for (int s = 0; s < a.nkv && ok; ++s)
@@ -548,24 +627,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // Each tile's rows are normalised (and, in KV-split mode, stitched with
     // the other half by the merge rule) into a staging buffer in shared
     // memory, then every warp writes its 32 rows to HBM as whole, coalesced
-    // rows.  The K/V rings hold the staging buffers: they are idle once the
-    // last P V product of both tiles has landed (the barrier below).
+    // rows (commit_rows).  The K/V rings hold the staging buffers: they are
+    // idle once the last P V product of both tiles has landed (barrier below).
     if (ok && c > 0) {
       ok = mbar_wait(bar(BOD(x)), (c - 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
     }
-    constexpr int kStride = D + 4;                       // floats per staged row (bank-conflict-free)
-    constexpr int kStageFloats = kBM * kStride + kBM;    // rows, then one float per row
-    static_assert(2 * kStageFloats * 4 <= SL::kBar - SL::kK, "staging buffers must fit in the K/V rings");
-    float* stage = reinterpret_cast<float*>(smem + SL::kK) + x * kStageFloats;
-    float* stage_w = stage + kBM * kStride;              // per-row lse (B, KV-split) or merge weight
+    float* stage = stage_of(x);
+    float* stage_w = stage + kBM * kStride;  // per-row merge weight (epilogue-fused mode)
+    float* stage_l = stage_w + kBM;          // per-row lse of the staged partial
     named_barrier_sync(1, 256);  // both tiles' MMAs are complete: the rings are free
     fence_proxy_async_smem();
     if (split && x == 1) {
       // B's normalised partial and its lse, for A to merge
       const bool has = ok && l_sum > 0.f;
       const float inv = has ? 1.f / l_sum : 0.f;
-      stage_w[row] = has ? (m_use + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
+      stage_l[row] = has ? (m_use + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
       if (ok && c > 0) tc_fence_after();
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {
@@ -579,33 +656,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
     }
     if (split) named_barrier_sync(1, 256);
-    // rows are written by every tile in row-pair mode, by A alone in KV-split mode
-    const bool writer = (ok || total == 0) && !(split && x == 1);
-    const long long row_base = a.mode == kModeFinal ? static_cast<long long>(b) * a.S + qs.pos + row0[x]
-                                                    : static_cast<long long>(b) * a.acc_brows + qs.mem + row0[x];
+    // rows are staged by every tile in row-pair mode, by A alone in KV-split mode
+    const bool writer = (ok || work == 0) && !(split && x == 1);
     if (writer) {
       const bool has = l_sum > 0.f;
       const float inv = has ? 1.f / l_sum : 0.f;
       float row_lse = has ? (m_use + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
-      const float* bstage = stage + kStageFloats;  // B's region (KV-split)
+      const float* bstage = stage_of(1);  // B's region (KV-split)
       MergeWeights mwb;  // KV-split: weight of B's partial in this row
       mwb.w = 0.f;
       if (split) {
-        mwb = merge_weights(row_lse, bstage[kBM * kStride + row]);
+        mwb = merge_weights(row_lse, bstage[kBM * kStride + kBM + row]);
         row_lse = mwb.lse;
       }
-      float* lse_ptr = (a.mode == kModeFinal ? a.lse : a.acc_lse) + (row_base + row) * a.Hq + h;
-      float w = 1.f;
-      if (valid) {
-        if (a.mode == kModeMerge) {
-          const MergeWeights mw = merge_weights(*lse_ptr, row_lse);
-          *lse_ptr = mw.lse;
-          w = mw.w;
-        } else {
-          *lse_ptr = row_lse;
-        }
-      }
-      stage_w[row] = w;
+      stage_l[row] = row_lse;
       if (c > 0) tc_fence_after();
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {
@@ -624,46 +688,40 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               make_float4(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1]), __uint_as_float(ov[i + 2]),
                           __uint_as_float(ov[i + 3]));
       }
-      __syncwarp();
-      // this warp's 32 rows, each written as one contiguous run
-      const int wr0 = (warp & 3) * 32;
-      const bool bf16_out = a.mode == kModeFinal && a.out_bf16;
-      constexpr int kLanesF32 = D / 4;   // float4 per row
-      constexpr int kLanesB16 = D / 8;   // 8 bf16 (16 B) per lane
-      const int lpr = bf16_out ? kLanesB16 : kLanesF32;
-      const int rpi = 32 / lpr;          // rows per warp instruction
-      const int ci = lane % lpr;
-      for (int r0 = 0; r0 < 32; r0 += rpi) {
-        const int r = wr0 + r0 + lane / lpr;
-        if (r >= rows[x]) continue;
-        const long long grow = (row_base + r) * a.Hq + h;
-        const float* src = stage + r * kStride;
-        if (bf16_out) {
-          const float4 lo = *reinterpret_cast<const float4*>(src + 8 * ci);
-          const float4 hi = *reinterpret_cast<const float4*>(src + 8 * ci + 4);
-          uint4 o;
-          o.x = pack_bf16x2(lo.x, lo.y);
-          o.y = pack_bf16x2(lo.z, lo.w);
-          o.z = pack_bf16x2(hi.x, hi.y);
-          o.w = pack_bf16x2(hi.z, hi.w);
-          reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + grow * D)[ci] = o;
-        } else {
-          float4 v = *reinterpret_cast<const float4*>(src + 4 * ci);
-          float4* dst = reinterpret_cast<float4*>((a.mode == kModeFinal ? static_cast<float*>(a.out) : a.acc_out) +
-                                                  grow * D) + ci;
-          if (a.mode == kModeMerge) {
-            const float wr = stage_w[r];
-            if (wr == 0.f) continue;
-            const float4 old = *dst;
-            v.x = merge_out(old.x, v.x, wr);
-            v.y = merge_out(old.y, v.y, wr);
-            v.z = merge_out(old.z, v.z, wr);
-            v.w = merge_out(old.w, v.w, wr);
-          }
-          *dst = v;
+      if (a.cluster == 1) commit_rows(x);
+    }
+  }
+
+  if (a.cluster > 1) {
+    // Cluster mode: CTA r finalises tile r.  Its row = own partial merged
+    // with the peer CTA's partial of the same row (merge rule), read from the
+    // peer's staging buffer through distributed shared memory.
+    cluster_sync();  // both CTAs have staged both tiles
+    if (warp < 8 && (warp >> 2) == crank) {
+      const int x = crank;
+      const int row = threadIdx.x & 127;
+      float* stage = stage_of(x);
+      float* stage_l = stage + kBM * kStride + kBM;
+      const uint32_t peer = cluster_map(smem_u32(stage), static_cast<uint32_t>(crank ^ 1));
+      const float peer_lse = ld_cluster_f32(peer + 4u * (kBM * kStride + kBM + row));
+      const MergeWeights mw = merge_weights(stage_l[row], peer_lse);
+      stage_l[row] = mw.lse;
+      if (mw.w != 0.f) {
+        float* own = stage + row * kStride;
+#pragma unroll 8
+        for (int i = 0; i < D; i += 4) {
+          const float4 pv = ld_cluster_f4(peer + 4u * (row * kStride + i));
+          float4 ov = *reinterpret_cast<float4*>(own + i);
+          ov.x = merge_out(ov.x, pv.x, mw.w);
+          ov.y = merge_out(ov.y, pv.y, mw.w);
+          ov.z = merge_out(ov.z, pv.z, mw.w);
+          ov.w = merge_out(ov.w, pv.w, mw.w);
+          *reinterpret_cast<float4*>(own + i) = ov;
         }
       }
+      commit_rows(x);
     }
+    cluster_sync();  // the peer has finished reading this CTA's staging buffers
   }
 
   tc_fence_before();

@@ -88,8 +88,17 @@ typedef enum {
  *  ROW_PAIRS: 256 query rows per CTA (two 128-row tiles sharing K/V loads).
  *  KV_SPLIT:  128 query rows per CTA; the CTA's KV tiles are halved between
  *             its two tiles and the two partials merged on chip with the rule.
- *  AUTO:      ROW_PAIRS unless that gives fewer than two CTAs per SM. */
-typedef enum { RA_TILING_AUTO = 0, RA_TILING_ROW_PAIRS = 1, RA_TILING_KV_SPLIT = 2 } ra_tiling;
+ *  CLUSTER2:  row pairs, with the KV tiles of each 256 rows halved between
+ *             the two CTAs of a thread-block cluster; the partials are merged
+ *             with the rule through distributed shared memory.
+ *  AUTO:      ROW_PAIRS unless that gives fewer than two CTAs per SM, then
+ *             KV_SPLIT. */
+typedef enum {
+  RA_TILING_AUTO = 0,
+  RA_TILING_ROW_PAIRS = 1,
+  RA_TILING_KV_SPLIT = 2,
+  RA_TILING_CLUSTER2 = 3
+} ra_tiling;
 
 typedef struct {
   ra_order order;  /* default RA_ORDER_RING  */

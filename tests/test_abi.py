@@ -80,7 +80,7 @@ def test_ring_attention_rejects_bad_arguments(ra):
     assert ring(ra, ws=None, opts=ctypes.byref(unf)) == E.RA_ERR_WORKSPACE  # per-step partials
     bad = ra.ra_options(9, 0, None, None, 0)
     assert ring(ra, opts=ctypes.byref(bad)) == E.RA_ERR_INVALID_ARG
-    bad_tiling = ra.ra_options(0, 0, None, None, 7)
+    bad_tiling = ra.ra_options(0, 0, None, None, 9)
     assert ring(ra, opts=ctypes.byref(bad_tiling)) == E.RA_ERR_INVALID_ARG
 
 

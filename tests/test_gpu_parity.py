@@ -153,7 +153,7 @@ def test_block_attn_every_pair(cuda_lib, case):
 SCHEDS = ["persistent", "fused", "unfused"]
 
 
-@pytest.mark.parametrize("tiling", ["row_pairs", "kv_split"])
+@pytest.mark.parametrize("tiling", ["row_pairs", "kv_split", "cluster2"])
 @pytest.mark.parametrize("order", ["ring", "tokenring"])
 @pytest.mark.parametrize("sched", SCHEDS)
 @pytest.mark.parametrize("case", [(2, 1200, 4, 4, 2, 128, True, "zigzag"), (1, 1024, 4, 2, 1, 64, True, "contiguous"),
@@ -194,7 +194,7 @@ def zigzag4k():
     return w, (q, k, v), (ro, rl)
 
 
-@pytest.mark.parametrize("tiling", ["auto", "row_pairs", "kv_split"])
+@pytest.mark.parametrize("tiling", ["auto", "row_pairs", "kv_split", "cluster2"])
 @pytest.mark.parametrize("sched", SCHEDS)
 @pytest.mark.parametrize("order", ["ring", "tokenring"])
 def test_zigzag4k_workload_full_oracle(cuda_lib, zigzag4k, sched, order, tiling):
