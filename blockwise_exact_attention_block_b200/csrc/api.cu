@@ -164,15 +164,15 @@ void order_segments(AttnArgs& a) {
     }
 }
 
-template <int D, bool SPLIT>
+template <int D, int TILING>
 ra_status launch_attn_t(const AttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                         cudaStream_t st) {
-  using SL = AttnSmem<D, SPLIT>;
+  using SL = AttnSmem<D, TILING == kTileKvSplit>;
   static int attr_set[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, TILING>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          SL::kBytes);
     if (e != cudaSuccess) return RA_ERR_CUDA;
     attr_set[dev] = 1;
@@ -180,8 +180,8 @@ ra_status launch_attn_t(const AttnArgs& a, const CUtensorMap& mq, const CUtensor
   const long long grid = static_cast<long long>(a.Hq) * a.B * a.nq * a.nseg * a.seg_tiles * a.cluster;
   if (grid <= 0) return RA_OK;
   if (grid > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
-  if (a.cluster == 1) {
-    attn_fwd_kernel<D, SPLIT><<<static_cast<unsigned>(grid), kAttnThreads, SL::kBytes, st>>>(mq, mk, mv, a);
+  if (TILING != kTileCluster2) {
+    attn_fwd_kernel<D, TILING><<<static_cast<unsigned>(grid), kAttnThreads, SL::kBytes, st>>>(mq, mk, mv, a);
     return cuda_status(cudaGetLastError());
   }
   cudaLaunchConfig_t cfg;
@@ -192,19 +192,25 @@ ra_status launch_attn_t(const AttnArgs& a, const CUtensorMap& mq, const CUtensor
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(a.cluster);
+  attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, attn_fwd_kernel<D, SPLIT>, mq, mk, mv, a));
+  return cuda_status(cudaLaunchKernelEx(&cfg, attn_fwd_kernel<D, TILING>, mq, mk, mv, a));
+}
+
+template <int D>
+ra_status launch_attn_d(const AttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                        cudaStream_t st) {
+  if (a.kv_split) return launch_attn_t<D, kTileKvSplit>(a, mq, mk, mv, st);
+  if (a.cluster == 2) return launch_attn_t<D, kTileCluster2>(a, mq, mk, mv, st);
+  return launch_attn_t<D, kTileRowPairs>(a, mq, mk, mv, st);
 }
 
 ra_status launch_attn(int D, const AttnArgs& a, const CUtensorMap& mq, const CUtensorMap& mk,
                       const CUtensorMap& mv, cudaStream_t st) {
-  if (D == 128)
-    return a.kv_split ? launch_attn_t<128, true>(a, mq, mk, mv, st) : launch_attn_t<128, false>(a, mq, mk, mv, st);
-  return a.kv_split ? launch_attn_t<64, true>(a, mq, mk, mv, st) : launch_attn_t<64, false>(a, mq, mk, mv, st);
+  return D == 128 ? launch_attn_d<128>(a, mq, mk, mv, st) : launch_attn_d<64>(a, mq, mk, mv, st);
 }
 
 int grid_for(long long work, int per_block) {

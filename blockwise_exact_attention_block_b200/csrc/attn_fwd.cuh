@@ -102,7 +102,8 @@ struct AttnArgs {
   int nseg;               // segments per block: 1 (contiguous) or 2 (zigzag)
   int seg_tiles;          // CTAs per query segment: ceil(len / 256), or ceil(len / 128) in KV-split mode
   int kv_split;           // 1: KV-split mode (see the top of this file)
-  int cluster;            // CTAs per cluster sharing one row pair (1 or 2; row pairs only)
+  int cluster;            // CTAs per cluster sharing one row pair (1 or 2; row pairs only;
+                          // selects the kernel instantiation, see Tiling)
   float scale_log2;       // log2(e) / sqrt(D)
   int mode;               // AttnMode
   // kModePartial / kModeMerge: row = b * acc_brows + memory row of the query
@@ -171,10 +172,16 @@ struct KvCursor {
   int s, e, t, nt;
 };
 
-template <int D, bool SPLIT>
+// Tiling modes (compile-time: each kernel instantiation carries only its own
+// code).
+enum Tiling : int { kTileRowPairs = 0, kTileKvSplit = 1, kTileCluster2 = 2 };
+
+template <int D, int TILING>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
+  constexpr bool SPLIT = TILING == kTileKvSplit;
+  constexpr int kCl = TILING == kTileCluster2 ? 2 : 1;  // CTAs per cluster
   using SL = AttnSmem<D, SPLIT>;
   constexpr int NSK = SL::kNSK;
   constexpr int NSV = SL::kNSV;
@@ -188,8 +195,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   // ---- tile decode: heads fastest (heads of one KV group share K/V in L2),
   // then batch, then query tiles in decreasing position (heaviest first).
-  const int crank = a.cluster > 1 ? static_cast<int>(cluster_ctarank()) : 0;
-  int idx = blockIdx.x / a.cluster;
+  int crank = 0;
+  if constexpr (kCl > 1) crank = static_cast<int>(cluster_ctarank());
+  int idx = blockIdx.x / kCl;
   const int h = idx % a.Hq;
   idx /= a.Hq;
   const int b = idx % a.B;
@@ -213,8 +221,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   for (int s = 0; s < a.nkv; ++s)
     for (int e = 0; e < a.nseg; ++e) total += tiles_for(a, seg_of(s, e), last_u);
   // this CTA's share [lo, hi) of the sequence (the cluster splits it in equal parts)
-  const int lo = crank * total / a.cluster;
-  const int hi = (crank + 1) * total / a.cluster;
+  const int lo = kCl > 1 ? crank * total / kCl : 0;
+  const int hi = kCl > 1 ? (crank + 1) * total / kCl : total;
   int work = hi - lo;
   // Tile x's share of the CTA's KV tiles.  u = index in the CTA's sequence,
   // t = index inside the segment.  KV-split: A takes [0, half), B [half, total).
@@ -688,11 +696,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               make_float4(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1]), __uint_as_float(ov[i + 2]),
                           __uint_as_float(ov[i + 3]));
       }
-      if (a.cluster == 1) commit_rows(x);
+      if constexpr (kCl == 1) commit_rows(x);
     }
   }
 
-  if (a.cluster > 1) {
+  if constexpr (kCl > 1) {
     // Cluster mode: CTA r finalises tile r.  Its row = own partial merged
     // with the peer CTA's partial of the same row (merge rule), read from the
     // peer's staging buffer through distributed shared memory.
