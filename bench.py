@@ -191,6 +191,27 @@ def attn_traffic(workload):
     return rec["dram_bytes_per_launch"]
 
 
+# ------------------------------------------------------------- multi-rank
+
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest `value` over all ranks (the slowest rank's time); the
+    identity without an initialised process group.  Works with any backend:
+    the tensor lives on `device` (a CUDA device for NCCL, the CPU for gloo)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(flops_per_step: float, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s of `world` replicas that each ran `steps` steps, timed
+    by the slowest rank (weak scaling: every rank does the same work)."""
+    return flops_per_step * world * steps / (max_ms * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------ merge kernels
 
 def bench_merge(ra, dev, T, k, reps, flush, kway=False):
@@ -310,11 +331,7 @@ def run_ours(args):
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     attn_ms = [a.elapsed_time(b) for a, b in av]
-    total_ms = sum(step_ms)
-    tot = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
-    total_ms = float(tot.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     status = ra.ra_get_device_status()
 
     # end to end through the public call with host buffers: H2D of Q, K, V from
@@ -345,12 +362,10 @@ def run_ours(args):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
         h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
         d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
-        e2e = {"value": w.flops * world * Ke / (float(e_ms.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": replica_throughput(w.flops, world, Ke, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke}
 
     pk, pk_kind = peaks()
@@ -375,7 +390,7 @@ def run_ours(args):
                  "GB/s": gbs, "ms": mms, "peak_GB/s": pk["hbm_gbs"], "frac": gbs / pk["hbm_gbs"],
                  "bytes_per_row": 12 * 128 + 12}
 
-    value = w.flops * world * K / (total_ms * 1e-3) / 1e12
+    value = replica_throughput(w.flops, world, K, total_ms)
     line = {"metric": "causal-adj attention TFLOP/s (% of dense bf16 peak)", "value": value, "unit": "TFLOP/s",
             "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
