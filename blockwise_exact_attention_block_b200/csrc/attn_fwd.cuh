@@ -276,10 +276,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   constexpr int kStageFloats = kBM * kStride + 2 * kBM; // rows, then per-row weight and lse
   static_assert(2 * kStageFloats * 4 <= SL::kBar - SL::kK, "staging buffers must fit in the K/V rings");
   auto stage_of = [&](int x) { return reinterpret_cast<float*>(smem + SL::kK) + x * kStageFloats; };
-  // Writes tile x's staged rows: the lse of each valid row (merged into the
-  // running state in epilogue-fused mode) and then, per warp, its 32 rows as
-  // contiguous runs.  Called by the 4 warps of tile x.
-  auto commit_rows = [&](int x) {
+  // Final write of tile x's staged rows, in two parts.  commit_lse: each of
+  // the tile's threads writes the lse of its own row (merged into the running
+  // state in epilogue-fused mode, where it also records the row's weight).
+  // store_rows: warp wi of nw warps writes rows [wi*128/nw, (wi+1)*128/nw)
+  // as contiguous runs (16 bytes per lane).
+  auto commit_lse = [&](int x) {
     float* stage = stage_of(x);
     float* stage_w = stage + kBM * kStride;
     const float* stage_l = stage_w + kBM;
@@ -298,15 +300,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         *lse_ptr = stage_l[row];
       }
     }
-    __syncwarp();
-    const int wr0 = (warp & 3) * 32;
+  };
+  auto store_rows = [&](int x, int wi, int nw) {
+    const float* stage = stage_of(x);
+    const float* stage_w = stage + kBM * kStride;
+    const int my_row0 = x ? row0_b : row0_a;
+    const int my_rows = x ? rows_b : rows_a;
+    const long long row_base = a.mode == kModeFinal ? static_cast<long long>(b) * a.S + qs.pos + my_row0
+                                                    : static_cast<long long>(b) * a.acc_brows + qs.mem + my_row0;
+    const int per = kBM / nw;
+    const int wr0 = wi * per;
     const bool bf16_out = a.mode == kModeFinal && a.out_bf16;
     const int lpr = bf16_out ? D / 8 : D / 4;  // lanes per row: 16 B per lane
     const int rpi = 32 / lpr;                  // rows per warp instruction
     const int ci = lane % lpr;
-    for (int r0 = 0; r0 < 32; r0 += rpi) {
+    for (int r0 = 0; r0 < per; r0 += rpi) {
       const int r = wr0 + r0 + lane / lpr;
-      if (r >= my_rows) continue;
+      if (r >= my_rows || r0 + lane / lpr >= per) continue;
       const long long grow = (row_base + r) * a.Hq + h;
       const float* src = stage + r * kStride;
       if (bf16_out) {
@@ -651,17 +661,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const bool has = ok && l_sum > 0.f;
       const float inv = has ? 1.f / l_sum : 0.f;
       stage_l[row] = has ? (m_use + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
-      if (ok && c > 0) tc_fence_after();
-#pragma unroll
-      for (int q = 0; q < D / 32; ++q) {
-        uint32_t ov[32];
-        if (ok && c > 0) tmem_ld32_wait(tO + 32 * q, ov);
-#pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4*>(stage + row * kStride + 32 * q + i) =
-              make_float4(has ? __uint_as_float(ov[i]) * inv : 0.f, has ? __uint_as_float(ov[i + 1]) * inv : 0.f,
-                          has ? __uint_as_float(ov[i + 2]) * inv : 0.f, has ? __uint_as_float(ov[i + 3]) * inv : 0.f);
+      uint32_t ov[D];
+      if (ok && c > 0) {
+        tc_fence_after();
+        if constexpr (D == 128) tmem_ld128_wait(tO, ov);
+        else tmem_ld64_wait(tO, ov);
       }
+#pragma unroll
+      for (int i = 0; i < D; i += 4)
+        *reinterpret_cast<float4*>(stage + row * kStride + i) =
+            make_float4(has ? __uint_as_float(ov[i]) * inv : 0.f, has ? __uint_as_float(ov[i + 1]) * inv : 0.f,
+                        has ? __uint_as_float(ov[i + 2]) * inv : 0.f, has ? __uint_as_float(ov[i + 3]) * inv : 0.f);
     }
     if (split) named_barrier_sync(1, 256);
     // rows are staged by every tile in row-pair mode, by A alone in KV-split mode
@@ -678,25 +688,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         row_lse = mwb.lse;
       }
       stage_l[row] = row_lse;
-      if (c > 0) tc_fence_after();
-#pragma unroll
-      for (int q = 0; q < D / 32; ++q) {
-        uint32_t ov[32];
-        if (c > 0) tmem_ld32_wait(tO + 32 * q, ov);  // c is uniform across the warp
-#pragma unroll
-        for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(has ? __uint_as_float(ov[i]) * inv : 0.f);
-        if (split && mwb.w != 0.f) {
-          const float* xb = bstage + row * kStride + 32 * q;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(merge_out(__uint_as_float(ov[i]), xb[i], mwb.w));
-        }
-#pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4*>(stage + row * kStride + 32 * q + i) =
-              make_float4(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1]), __uint_as_float(ov[i + 2]),
-                          __uint_as_float(ov[i + 3]));
+      uint32_t ov[D];
+      if (c > 0) {  // c is uniform across the warp
+        tc_fence_after();
+        if constexpr (D == 128) tmem_ld128_wait(tO, ov);
+        else tmem_ld64_wait(tO, ov);
       }
-      if constexpr (kCl == 1) commit_rows(x);
+#pragma unroll
+      for (int i = 0; i < D; i += 4) {
+        float4 v = make_float4(has ? __uint_as_float(ov[i]) * inv : 0.f, has ? __uint_as_float(ov[i + 1]) * inv : 0.f,
+                               has ? __uint_as_float(ov[i + 2]) * inv : 0.f,
+                               has ? __uint_as_float(ov[i + 3]) * inv : 0.f);
+        if (split && mwb.w != 0.f) {
+          const float4 xb = *reinterpret_cast<const float4*>(bstage + row * kStride + i);
+          v.x = merge_out(v.x, xb.x, mwb.w);
+          v.y = merge_out(v.y, xb.y, mwb.w);
+          v.z = merge_out(v.z, xb.z, mwb.w);
+          v.w = merge_out(v.w, xb.w, mwb.w);
+        }
+        *reinterpret_cast<float4*>(stage + row * kStride + i) = v;
+      }
+      if constexpr (kCl == 1) {
+        commit_lse(x);
+        if (!split) {  // each warp stores the 32 rows it staged
+          __syncwarp();
+          store_rows(x, warp & 3, 4);
+        }
+      }
+    }
+    if (split) {
+      // KV-split: only A staged rows; all 8 warps store them (16 rows each)
+      named_barrier_sync(1, 256);
+      if (ok || work == 0) store_rows(0, warp, 8);
     }
   }
 
@@ -727,7 +750,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           *reinterpret_cast<float4*>(own + i) = ov;
         }
       }
-      commit_rows(x);
+      commit_lse(x);
+      __syncwarp();
+      store_rows(x, warp & 3, 4);
     }
     cluster_sync();  // the peer has finished reading this CTA's staging buffers
   }
