@@ -172,6 +172,62 @@ def test_ring_attention_matches_full_oracle(cuda_lib, case, sched, order, tiling
     assert ra.ra_get_device_status() == 0
 
 
+EDGE_CASES = [
+    # B, S, Hq, Hkv, D, n, causal, partition
+    (1, 256, 2, 2, 128, 1, True, "contiguous"),     # one block: plain attention
+    (1, 256, 2, 2, 128, 1, True, "zigzag"),         # one block, two chunks
+    (1, 512, 2, 1, 128, 16, True, "zigzag"),        # 16 blocks, chunks of 16 rows
+    (1, 32, 1, 1, 128, 16, True, "zigzag"),         # chunks of a single row
+    (3, 384, 6, 2, 64, 3, True, "zigzag"),          # batch 3, GQA 3, D=64, c=64
+    (2, 640, 4, 4, 128, 5, False, "contiguous"),    # non-causal, L=128
+    (1, 2000, 4, 1, 128, 4, True, "zigzag"),        # c=250: tiles straddle nothing, ragged tails
+    (1, 1000, 2, 2, 64, 2, False, "zigzag"),        # non-causal zigzag
+]
+
+
+@pytest.mark.parametrize("sched", SCHEDS)
+@pytest.mark.parametrize("case", EDGE_CASES, ids=lambda c: f"B{c[0]}S{c[1]}H{c[2]}/{c[3]}D{c[4]}n{c[5]}{c[7]}{'C' if c[6] else ''}")
+def test_ring_attention_edge_cases(cuda_lib, case, sched):
+    ra = cuda_lib
+    B, S, Hq, Hkv, D, n, causal, part = case
+    q, k, v = attention_inputs(B, S, Hq, Hkv, D, "bf16", seed=6)
+    ro, rl = F.full_attention(q, k, v, causal, Hq // Hkv)
+    for tiling in ("auto", "row_pairs", "kv_split", "cluster2"):
+        o, l = ra.ra_ring_attention(q.cuda(), k.cuda(), v.cuda(), n, causal, part, out_dtype=torch.float32,
+                                    sched=sched, tiling=tiling)
+        assert_close_bf16(to_np(o), ro, f"out {sched}/{tiling}")
+        assert_close_bf16(to_np(l), rl, f"lse {sched}/{tiling}")
+    assert ra.ra_get_device_status() == 0
+
+
+def test_block_attn_empty_and_full_pairs(cuda_lib):
+    # causal zigzag, n=4: pairs whose KV block lies wholly after (every row
+    # empty: lse = -inf, out = 0) or wholly before (no masking) the query block
+    ra = cuda_lib
+    B, S, n, Hq, Hkv, D = 1, 2048, 4, 2, 2, 128
+    q, k, v = attention_inputs(B, S, Hq, Hkv, D, "bf16", seed=8)
+    perm = K.zigzag_perm(S, n)
+    L = S // n
+    pos = perm.reshape(n, L)
+    pt = torch.from_numpy(perm)
+    qp, kp, vp = q[:, pt], k[:, pt], v[:, pt]
+    seen_empty = seen_full = False
+    for qb in range(n):
+        for kb in range(n):
+            qblk = qp[:, qb * L:(qb + 1) * L].contiguous()
+            kblk = kp[:, kb * L:(kb + 1) * L].contiguous()
+            vblk = vp[:, kb * L:(kb + 1) * L].contiguous()
+            bo, bl = ra.ra_block_attn(qblk.cuda(), kblk.cuda(), vblk.cuda(), S, n, qb, kb, True, "zigzag")
+            ro, rl = K.block_partial(qblk, kblk, vblk, pos[qb], pos[kb], True, 1)
+            empty_rows = np.isneginf(rl)
+            seen_empty |= bool(empty_rows.any())
+            seen_full |= bool((~empty_rows).all())
+            assert np.all(to_np(bo)[empty_rows] == 0.0)
+            assert_close_bf16(to_np(bo), ro, f"block_out q{qb} kv{kb}")
+            assert_close_bf16(to_np(bl), rl, f"block_lse q{qb} kv{kb}")
+    assert seen_empty and seen_full
+
+
 def test_tiny_workload(cuda_lib):
     # fp32 inputs: the library rounds them to bf16 on entry; the attention is
     # judged against the oracle on the same rounded values.
