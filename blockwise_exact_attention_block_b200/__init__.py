@@ -40,8 +40,7 @@ SCHEDS = {"auto": RA_SCHED_AUTO, "unfused": RA_SCHED_UNFUSED, "fused": RA_SCHED_
 
 EXPORTED = ["ra_block_attn", "ra_merge_partial", "ra_merge_partials", "ra_ring_attention",
             "ra_ring_attention_workspace", "ra_zigzag_permute", "ra_get_device_status",
-            "ra_status_string", "ra_version", "ra_ring_attention_noalloc", "ra_noalloc_scratch_bytes",
-            "ra_selftest_exp2_poly"]
+            "ra_status_string", "ra_version", "ra_ring_attention_noalloc", "ra_noalloc_scratch_bytes"]
 
 
 class ra_options(ctypes.Structure):
@@ -71,8 +70,6 @@ _lib.ra_noalloc_scratch_bytes.argtypes = []
 _lib.ra_noalloc_scratch_bytes.restype = _sz
 _lib.ra_zigzag_permute.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
 _lib.ra_zigzag_permute.restype = _i
-_lib.ra_selftest_exp2_poly.argtypes = [_vp, _vp, _i64, _vp]
-_lib.ra_selftest_exp2_poly.restype = _i
 _lib.ra_get_device_status.argtypes = [_vp]
 _lib.ra_get_device_status.restype = _i
 _lib.ra_status_string.argtypes = [_i]
@@ -253,13 +250,6 @@ def ra_zigzag_permute(src, n_blocks: int, inverse: bool = False, dst=None, strea
     _check(_lib.ra_zigzag_permute(_ptr(src), _ptr(dst), B, S, H, D, src.element_size(), n_blocks,
                                   int(bool(inverse)), _stream(stream)), "ra_zigzag_permute")
     return dst
-
-
-def ra_selftest_exp2_poly(x, stream=None):
-    """The kernel's FMA-pipe 2^x approximation applied to an fp32 CUDA tensor."""
-    y = torch.empty_like(x)
-    _check(_lib.ra_selftest_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "ra_selftest_exp2_poly")
-    return y
 
 
 def ra_get_device_status(stream=None) -> int:

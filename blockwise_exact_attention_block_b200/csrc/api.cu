@@ -308,27 +308,9 @@ bool valid_opts(const ra_options* o) {
   return o->sched >= RA_SCHED_AUTO && o->sched <= RA_SCHED_PERSISTENT;
 }
 
-__global__ void exp2_poly_selftest_kernel(const float* __restrict__ x, float* __restrict__ y, long long npairs) {
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < npairs;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    float a, b;
-    f2_unpack(exp2_poly_x2(f2_pack(x[2 * i], x[2 * i + 1])), a, b);
-    y[2 * i] = a;
-    y[2 * i + 1] = b;
-  }
-}
-
 }  // namespace
 
 extern "C" {
-
-ra_status ra_selftest_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
-  if (n < 0 || (n & 1)) return RA_ERR_INVALID_ARG;
-  if (n == 0) return RA_OK;
-  if (!x || !y) return RA_ERR_INVALID_ARG;
-  exp2_poly_selftest_kernel<<<grid_for(n / 2, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n / 2);
-  return cuda_status(cudaGetLastError());
-}
 
 const char* ra_status_string(ra_status s) {
   switch (s) {

@@ -71,11 +71,6 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kAttnThreads * kRegsL
               "register reallocation must fit in the launch allocation");
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-// Of every 8 exponential pairs in a full tile, this many run on the FMA pipe.
-#ifndef RA_EMU_PAIRS8
-#define RA_EMU_PAIRS8 0
-#endif
-constexpr int kEmuPairs8 = RA_EMU_PAIRS8;
 // 1: exponentials as ex2.approx.f16x2 (two per SFU instruction).
 #ifndef RA_EXP_F16X2
 #define RA_EXP_F16X2 0
@@ -582,10 +577,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const float base = (m_use == -INFINITY) ? 0.f : m_use;
           const uint64_t sl2x2 = f2_pack(sl2, sl2);
           const uint64_t nbase2 = f2_pack(-base, -base);
-          // Exponentials: the SFU does ex2 for most pairs; in tiles without
-          // masked entries (the whole warp), kEmuPairs of every 16 pairs run
-          // on the FMA pipe instead (exp2_poly_x2), splitting the load.
-          const bool emu = __all_sync(0xffffffffu, full);
+          // exponentials on the SFU (ex2.approx), two per pair of scores
           uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
           for (int ch = 0; ch < kBN / 32; ++ch) {  // 32 scores -> 16 packed bf16 pairs per store
@@ -594,20 +586,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             for (int pp = 0; pp < 16; ++pp) {
               const int j = ch * 32 + 2 * pp;
               const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), sl2x2, nbase2);
-              uint64_t e2;
-              if (emu && (pp % 8) < kEmuPairs8) {
-                e2 = exp2_poly_x2(x2);
-              } else {
-                float x0, x1;
-                f2_unpack(x2, x0, x1);
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
 #if RA_EXP_F16X2
-                float q0, q1;
-                exp2_f16x2(x0, x1, q0, q1);
-                e2 = f2_pack(q0, q1);
+              float q0, q1;
+              exp2_f16x2(x0, x1, q0, q1);
+              const uint64_t e2 = f2_pack(q0, q1);
 #else
-                e2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
+              const uint64_t e2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
 #endif
-              }
               acc[pp & 3] = f2_add(acc[pp & 3], e2);
               float p0, p1;
               f2_unpack(e2, p0, p1);

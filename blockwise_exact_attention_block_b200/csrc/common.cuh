@@ -338,36 +338,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// 2^x for a pair of fp32 values, on the FMA and integer pipes (no SFU).
-// Range reduction: x = j + f with j the nearest integer (added to 1.5 * 2^23
-// so the rounding is done by the fp32 add itself) and f in [-0.5, 0.5];
-// 2^f from a degree-4 polynomial fitted here to minimise the relative error
-// on [-0.5, 0.5] (fit_exp2_poly.py; max relative error 2.7e-6 in fp32);
-// 2^j is added into the exponent field: with t = x + 1.5 * 2^23,
-// bits(result) = bits(p) + (bits(t) << 23) (mod 2^32).  Inputs are clamped
-// to [-125, 126] so the exponent never leaves the normal range.
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  float x0, x1;
-  f2_unpack(x, x0, x1);
-  x0 = fminf(fmaxf(x0, -125.f), 126.f);
-  x1 = fminf(fmaxf(x1, -125.f), 126.f);
-  const uint64_t xc = f2_pack(x0, x1);
-  const uint64_t t = f2_add(xc, f2_pack(kMagic, kMagic));
-  const uint64_t r = f2_add(t, f2_pack(-kMagic, -kMagic));       // nearest integers
-  const uint64_t f = f2_fma(r, f2_pack(-1.f, -1.f), xc);          // x - j, exact
-  uint64_t p = f2_fma(f, f2_pack(9.570068680e-03f, 9.570068680e-03f), f2_pack(5.591780692e-02f, 5.591780692e-02f));
-  p = f2_fma(p, f, f2_pack(2.402474433e-01f, 2.402474433e-01f));
-  p = f2_fma(p, f, f2_pack(6.931218505e-01f, 6.931218505e-01f));
-  p = f2_fma(p, f, f2_pack(9.999992847e-01f, 9.999992847e-01f));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  const uint32_t r0 = __float_as_uint(p0) + (__float_as_uint(t0) << 23);
-  const uint32_t r1 = __float_as_uint(p1) + (__float_as_uint(t1) << 23);
-  return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
-}
-
 // 2^x for a pair on the SFU in half precision: both values are rounded to
 // fp16 (11-bit significand), exponentiated by one ex2.approx.f16x2, and
 // widened back to fp32.  Results below 2^-24 flush to 0; x = -inf gives 0.

@@ -231,13 +231,6 @@ ra_status ra_ring_attention_noalloc(const void* q, const void* k, const void* v,
 /* Size in bytes of the fixed scratch array behind ra_ring_attention_noalloc. */
 size_t ra_noalloc_scratch_bytes(void);
 
-/* Diagnostic: y[i] = the FMA-pipe 2^x approximation the attention kernel
- * uses for part of its exponentials, on device arrays x, y of n floats
- * (n even).  Exists so the approximation can be checked against the CUDA
- * exp2f results; relative error bound 3e-6 for x in [-125, 126] (inputs
- * outside are clamped to that range). */
-ra_status ra_selftest_exp2_poly(const float* x, float* y, int64_t n, void* stream);
-
 /* Reads and clears the device status word (synchronises `stream`).  Returns
  * RA_OK, RA_ERR_TIMEOUT or RA_ERR_DEVICE_BOUNDS, or RA_ERR_CUDA when the read
  * itself fails. */

@@ -58,25 +58,6 @@ def test_zigzag_permute_bit_exact(cuda_lib, shape, n, dtype):
     assert torch.equal(back.cpu(), x)
 
 
-# ------------------------------------------- FMA-pipe exponential (2^x)
-
-def test_exp2_poly_against_cuda_exp2(cuda_lib):
-    # the approximation the kernel uses for part of its exponentials, against
-    # CUDA's exp2f (torch.exp2 on the device) and its clamping range
-    ra = cuda_lib
-    g = torch.Generator(device="cuda").manual_seed(0)
-    x = torch.cat([torch.rand(1 << 20, device="cuda", generator=g) * 251.0 - 125.0,
-                   torch.rand(1 << 16, device="cuda", generator=g) * 30.0 - 30.0,
-                   torch.tensor([-125.0, -64.5, -1.5, -0.5, 0.0, 0.5, 1.0, 7.999, 8.0, 126.0], device="cuda")])
-    x = x[: x.numel() // 2 * 2].contiguous()
-    y = ra.ra_selftest_exp2_poly(x)
-    ref = torch.exp2(x.double())
-    rel = ((y.double() - ref).abs() / ref).max().item()
-    assert rel <= 3e-6, rel
-    lo = ra.ra_selftest_exp2_poly(torch.tensor([-1000.0, float("-inf")], device="cuda"))
-    assert torch.allclose(lo.double(), torch.full((2,), 2.0 ** -125, dtype=torch.float64, device="cuda"), rtol=3e-6)
-
-
 # ---------------------------------------------------------------- merge rule
 
 def check_merge(got_o, got_l, ref_o, ref_l):
