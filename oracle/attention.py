@@ -108,3 +108,36 @@ def attention_rows(q, k, v, rows, causal: bool, gqa_groups: int = 1, batch: int 
             lse[sel] = (m + np.log(tot))[:, 0]
             out[sel] = (e / tot) @ vv[:jmax]
     return out, lse
+
+
+def decode_attention(q, k, v, causal: bool, gqa_groups: int = 1):
+    """Attention of the last Tq tokens of a sequence over its Skv cached keys.
+
+    q: [B, Tq, Hq, D] holds the queries of tokens Skv - Tq .. Skv - 1;
+    k, v: [B, Skv, Hkv, D] the key/value cache of tokens 0 .. Skv - 1.
+    Query i (position Skv - Tq + i) sees key j iff j <= Skv - Tq + i when
+    causal, every key otherwise.  Returns (out [B, Tq, Hq, D], lse [B, Tq, Hq])
+    in fp64.  TokenRing review, "Reading between the lines": the decode-phase
+    KV-cache variant; the computation is plain softmax attention per query.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Tq, Hq, D = q.shape
+    Skv = k.shape[1]
+    if Tq > Skv:
+        raise ValueError("more queries than cached tokens")
+    scale = softmax_scale(D)
+    out = np.zeros((B, Tq, Hq, D), dtype=np.float64)
+    lse = np.zeros((B, Tq, Hq), dtype=np.float64)
+    pos = Skv - Tq + np.arange(Tq)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // gqa_groups
+            s = (q[b, :, h, :] @ k[b, :, g, :].T) * scale
+            if causal:
+                s = np.where(np.arange(Skv)[None, :] <= pos[:, None], s, -np.inf)
+            m = s.max(axis=1, keepdims=True)
+            e = np.exp(s - m)
+            tot = e.sum(axis=1, keepdims=True)
+            lse[b, :, h] = (m + np.log(tot))[:, 0]
+            out[b, :, h, :] = (e / tot) @ v[b, :, g, :]
+    return out, lse

@@ -242,3 +242,25 @@ def visible_pairs_per_block(S: int, n: int, partition: str) -> np.ndarray:
     """Number of causal (query, key) pairs whose query lies in each block."""
     pos = partition_perm(S, n, partition).reshape(n, S // n)
     return (pos + 1).sum(axis=1)
+
+
+def kv_splits(Skv: int, n_splits: int):
+    """Contiguous chunks of the KV cache: chunk i = [i*Lk, min((i+1)*Lk, Skv)),
+    Lk = ceil(Skv / n_splits); the last chunk may be shorter."""
+    Lk = -(-Skv // n_splits)
+    return [(i * Lk, min((i + 1) * Lk, Skv)) for i in range(n_splits) if i * Lk < Skv]
+
+
+def decode_blockwise(q, k, v, causal: bool, gqa_groups: int, n_splits: int):
+    """Decode attention by KV-cache chunks: one partial per chunk
+    (block_partial), folded with the merge rule (merge_partials).  Query i has
+    position Skv - Tq + i.  TokenRing review, "Reading between the lines"."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    Tq, Skv = q.shape[1], k.shape[1]
+    qpos = Skv - Tq + np.arange(Tq)
+    outs, lses = [], []
+    for (j0, j1) in kv_splits(Skv, n_splits):
+        bo, bl = block_partial(q, k[:, j0:j1], v[:, j0:j1], qpos, np.arange(j0, j1), causal, gqa_groups)
+        outs.append(bo)
+        lses.append(bl)
+    return merge_partials(outs, lses)

@@ -365,3 +365,43 @@ def test_causal_pin_catches_off_by_one_mask():
     shifted = np.concatenate([np.zeros_like(v[:, :1]), v[:, :-1]], axis=1)
     assert np.max(np.abs(out[0, 0, 0] - v[0, 0, 0])) < TOL
     assert np.max(np.abs(out[0, 0, 0] - shifted[0, 0, 0])) > 1e-6
+
+
+# --------------------------------------------------------- decode (KV cache)
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_decode_equals_last_rows_of_full_attention(causal):
+    # the decode queries are the last Tq tokens: same rows of full attention
+    B, S, Hq, Hkv, D, Tq = 2, 80, 4, 2, 16, 7
+    q, k, v = small(B, S, Hq, Hkv, D, seed=21)
+    fo, fl = F.full_attention(q, k, v, causal, 2, row_chunk=16)
+    do, dl = F.decode_attention(q[:, S - Tq:], k, v, causal, 2)
+    assert np.max(np.abs(do - fo[:, S - Tq:])) < TOL
+    assert np.max(np.abs(dl - fl[:, S - Tq:])) < TOL
+
+
+def test_decode_single_token_brute_force():
+    B, S, Hq, D = 1, 9, 2, 4
+    q, k, v = small(B, S, Hq, Hq, D, seed=23)
+    bo, bl = brute_attention(q, k, v, True, 1)
+    do, dl = F.decode_attention(q[:, -1:], k, v, True, 1)
+    assert np.max(np.abs(do[:, 0] - bo[:, -1])) < TOL
+    assert np.max(np.abs(dl[:, 0] - bl[:, -1])) < TOL
+
+
+@pytest.mark.parametrize("n_splits", [1, 2, 3, 7, 16])
+@pytest.mark.parametrize("causal", [False, True])
+def test_decode_blockwise_equals_decode(n_splits, causal):
+    B, S, Hq, Hkv, D, Tq = 1, 100, 4, 1, 8, 5
+    q, k, v = small(B, S, Hq, Hkv, D, seed=25)
+    ro, rl = F.decode_attention(q[:, -Tq:], k, v, causal, 4)
+    bo, bl = K.decode_blockwise(q[:, -Tq:], k, v, causal, 4, n_splits)
+    assert np.max(np.abs(bo - ro)) < TOL
+    assert np.max(np.abs(bl - rl)) < TOL
+
+
+def test_kv_splits_cover_the_cache():
+    for Skv, n in [(100, 3), (4096, 16), (7, 16), (10000, 7)]:
+        sp = K.kv_splits(Skv, n)
+        assert sp[0][0] == 0 and sp[-1][1] == Skv
+        assert all(a1 == b0 for (_, a1), (b0, _) in zip(sp, sp[1:]))
