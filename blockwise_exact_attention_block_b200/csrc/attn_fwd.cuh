@@ -63,6 +63,9 @@ constexpr int kBM = 128;        // query rows per tile = TMEM lanes
 constexpr int kCtaRows = 256;   // two tiles per CTA
 constexpr int kBN = 128;        // keys per KV tile
 constexpr int kMaxBlocks = 16;  // ring size limit
+// Largest row sum of a tile's exponentials accepted on the common softmax path
+// (every value is then <= 2^15).
+constexpr float kFastSumLimit = 32768.f;
 constexpr int kAttnThreads = 384;
 constexpr int kRegsLaunch = 168;  // per thread at launch (__launch_bounds__(384, 1))
 constexpr int kRegsSoftmax = 216;
@@ -162,9 +165,15 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   }
 }
 
-// Position of the CTA's g-th KV tile as (KV block index s, segment e, tile t).
-struct KvCursor {
-  int s, e, t, nt;
+// A walk over the CTA's KV tiles in schedule order: segment sg (KV block
+// s = sg / nseg of the CTA's list, segment e = sg % nseg) and tile t inside it,
+// with the segment itself and its tile counts for the CTA's last row (nt) and
+// the last rows of tiles A and B (na, nb).  The launch arguments are only read
+// when the walk enters a segment, so a step costs a few integer operations.
+struct KvWalk {
+  int sg, t;
+  int nt, na, nb;
+  Seg seg;
 };
 
 // Tiling modes (compile-time: each kernel instantiation carries only its own
@@ -222,22 +231,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // Tile x's share of the CTA's KV tiles.  u = index in the CTA's sequence,
   // t = index inside the segment.  KV-split: A takes [0, half), B [half, total).
   const int half = (total + 1) / 2;
-  auto active = [&](int x, int u, int t, const Seg& ks) -> bool {
-    if (split) return x == 0 ? u < half : u >= half;
-    return u >= lo && u < hi && t < tiles_for(a, ks, x ? last_b : last_a);
-  };
-  // The segment and in-segment tile of the CTA's u-th KV tile.
-  auto locate = [&](int u, int& s_, int& e_, int& t_) {
-    for (s_ = 0; s_ < a.nkv; ++s_)
-      for (e_ = 0; e_ < a.nseg; ++e_) {
-        const int nt = tiles_for(a, seg_of(s_, e_), last_u);
-        if (u < nt) {
-          t_ = u;
-          return;
-        }
-        u -= nt;
+  // Walk helpers (see KvWalk): enter the segment sg (skipping segments the
+  // CTA sees nothing of), start at the CTA's u-th tile, step to the next tile.
+  const int nsg = a.nkv * a.nseg;
+  auto enter = [&](KvWalk& k) {
+    for (; k.sg < nsg; ++k.sg) {
+      k.seg = a.kvseg[a.kv_list[qi][k.sg / a.nseg]][k.sg % a.nseg];
+      k.nt = tiles_for(a, k.seg, last_u);
+      if (k.nt > 0) {
+        k.na = tiles_for(a, k.seg, last_a);
+        k.nb = tiles_for(a, k.seg, last_b);
+        return;
       }
-    t_ = 0;
+    }
+    k.nt = k.na = k.nb = 0;
+  };
+  auto walk_from = [&](int u) -> KvWalk {
+    KvWalk k;
+    k.sg = 0;
+    enter(k);
+    while (k.nt > 0 && u >= k.nt) {
+      u -= k.nt;
+      ++k.sg;
+      enter(k);
+    }
+    k.t = u;
+    return k;
+  };
+  auto walk_next = [&](KvWalk& k) {
+    if (++k.t >= k.nt) {
+      k.t = 0;
+      ++k.sg;
+      enter(k);
+    }
   };
 
   auto bar = [&](int i) -> uint32_t { return sb + SL::kBar + 8u * i; };
@@ -358,14 +384,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                       bar(BQ));
       int g = 0;
       bool ok = true;
+      // row pairs: one walk over [lo, hi); KV-split: A's tiles [0, half) and B's
+      // [half, total), loaded alternately A0, B0, A1, B1, ...
+      KvWalk wa = walk_from(split ? 0 : lo);
+      KvWalk wb = walk_from(split ? half : total);
       int issued_k[NSK], issued_v[NSV];
       for (int s = 0; s < NSK; ++s) issued_k[s] = -1;
       for (int s = 0; s < NSV; ++s) issued_v[s] = -1;
       // load order: the CTA's sequence (row pairs), or A0, B0, A1, B1, ... (KV-split)
       for (int g2 = 0; g2 < work && ok; ++g2) {
-        int s, e, t;
-        locate(split ? ((g2 & 1) ? half + (g2 >> 1) : (g2 >> 1)) : lo + g2, s, e, t);
-        const Seg ks = seg_of(s, e);
+        const bool use_b = split && (g2 & 1);
+        const int t = use_b ? wb.t : wa.t;
+        const Seg ks = use_b ? wb.seg : wa.seg;
         const int sk = g % NSK, sv = g % NSV;
         if (!mbar_wait(bar(BKE(sk)), ((g / NSK) & 1) ^ 1, abort_flag)) { ok = false; break; }
         mbar_expect_tx(bar(BKF(sk)), SL::kTile);
@@ -380,6 +410,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                       bar(BVF(sv)));
         issued_v[sv] = g;
         ++g;
+        if (use_b) walk_next(wb);
+        else walk_next(wa);
       }
       if (!ok) {  // let every copy already issued land before shared memory is released
         mbar_drain(bar(BQ), 0);
@@ -412,21 +444,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           mma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, bd, kIdescO, (acc || kk > 0) ? 1u : 0u);
         }
         tc_commit(bar(BOD(x)));
-      };
-      // moves the cursor to the next KV tile that exists
-      auto advance = [&](KvCursor& k) {
-        ++k.t;
-        while (k.t >= k.nt && k.s < a.nkv) {
-          k.t = 0;
-          if (++k.e == a.nseg) {
-            k.e = 0;
-            ++k.s;
-          }
-          k.nt = k.s < a.nkv ? tiles_for(a, seg_of(k.s, k.e), last_u) : 0;
-        }
-      };
-      auto active_at = [&](const KvCursor& k, int x) {
-        return k.t < tiles_for(a, seg_of(k.s, k.e), x ? last_b : last_a);
       };
 
       if (split) {
@@ -462,10 +479,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_commit(bar(BEND));
         mbar_drain(bar(BEND), 0);
       } else {
-      KvCursor cur;
-      locate(lo, cur.s, cur.e, cur.t);  // this CTA's first tile (work > 0, so it exists)
-      cur.nt = tiles_for(a, seg_of(cur.s, cur.e), last_u);
-      bool act[2] = {active_at(cur, 0), active_at(cur, 1)};
+      KvWalk cur = walk_from(lo);  // this CTA's first tile (work > 0, so it exists)
+      bool act[2] = {cur.t < cur.na, cur.t < cur.nb};
       int cnt[2] = {0, 0};  // P V products issued per tile
       bool ok = mbar_wait(bar(BQ), 0, abort_flag);
       if (ok) ok = mbar_wait(bar(BKF(0)), 0, abort_flag);
@@ -479,12 +494,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int st = g % NSV;                 // V stage of tile g
         const int sk1 = (g + 1) % NSK;          // K stage of tile g + 1
         const bool has_next = g + 1 < work;
-        KvCursor nxt = cur;
+        KvWalk nxt = cur;
         bool act1[2] = {false, false};
         if (has_next) {
-          advance(nxt);
-          act1[0] = active_at(nxt, 0);
-          act1[1] = active_at(nxt, 1);
+          walk_next(nxt);
+          act1[0] = nxt.t < nxt.na;
+          act1[1] = nxt.t < nxt.nb;
         }
         if (!mbar_wait(bar(BVF(st)), (g / NSV) & 1, abort_flag)) break;
         bool k_ready = false;
@@ -530,103 +545,141 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t tS = tmem + lane_base + x * 128;
     const uint32_t tO = tmem + lane_base + 256 + x * 128;
     const float sl2 = a.scale_log2;
-    float m_use = -INFINITY;
+    // Padding rows (beyond the segment) see no key; a finite base keeps their
+    // warp on the common path (their exponentials are all 0).
+    float m_use = valid ? -INFINITY : 0.f;
     float l_sum = 0.f;
     bool ok = work > 0;
     int c = 0;  // tiles processed by this tile's softmax
-    int u = 0;  // position in the CTA's KV sequence
-    for (int s = 0; s < a.nkv && ok; ++s)
-      for (int e = 0; e < a.nseg && ok; ++e) {
-        const Seg ks = seg_of(s, e);
-        const int nt = tiles_for(a, ks, last_u);
-        const int lim = visible_count(a, ks, qpos);
-        for (int t = 0; t < nt; ++t, ++u) {
-          if (!active(x, u, t, ks)) continue;
-          ok = mbar_wait(bar(BSF(x)), c & 1, abort_flag);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          tc_fence_after();
-          uint32_t sv[kBN];
-          tmem_ld128_wait(tS, sv);
-          const int cnt = lim - t * kBN;
-          const bool full = cnt >= kBN;
-          if (__any_sync(0xffffffffu, !full)) {  // warp-uniform: full tiles skip the masking code
+    // This tile's KV tiles: row pairs, those of [lo, hi) its rows see;
+    // KV-split, A's [0, half) or B's [half, total) of the CTA's sequence.
+    KvWalk w = walk_from(split ? (x ? half : 0) : lo);
+    const int n_walk = split ? (x ? total - half : half) : work;
+    int lim_sg = -1, lim = 0;  // keys of the walk's segment this row sees
+    for (int i = 0; i < n_walk && ok; ++i, walk_next(w)) {
+      if (!split && w.t >= (x ? w.nb : w.na)) continue;
+      if (w.sg != lim_sg) {
+        lim_sg = w.sg;
+        lim = visible_count(a, w.seg, qpos);
+      }
+      const int t = w.t;
+      ok = mbar_wait(bar(BSF(x)), c & 1, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[kBN];
+      const int cnt = lim - t * kBN;
+      const bool masked = __any_sync(0xffffffffu, cnt < kBN);  // warp-uniform: full tiles skip the masking code
+      // S of this row from TMEM, with the keys it may not see set to -inf
+      auto load_s = [&]() {
+        tmem_ld128_wait(tS, sv);
+        if (masked) {
 #pragma unroll
-            for (int j = 0; j < kBN; ++j) sv[j] = j < cnt ? sv[j] : __float_as_uint(-INFINITY);
-          }
-          // row maximum: 3-input max, 8 independent chains of depth 8
-          float m8[8];
+          for (int j = 0; j < kBN; ++j) sv[j] = j < cnt ? sv[j] : __float_as_uint(-INFINITY);
+        }
+      };
+      load_s();
+      // P = 2^(scale * S - base) as packed bf16 pairs, on the SFU (ex2.approx),
+      // two per pair of scores, into pk (when given) or straight into the
+      // tile's TMEM columns (over S); returns the row sum of the fp32 values.
+      auto exps = [&](float base, uint32_t* pk_out) -> float {
+        const uint64_t sl2x2 = f2_pack(sl2, sl2);
+        const uint64_t nbase2 = f2_pack(-base, -base);
+        uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-          for (int q = 0; q < 8; ++q) m8[q] = fmaxf(__uint_as_float(sv[2 * q]), __uint_as_float(sv[2 * q + 1]));
+        for (int ch = 0; ch < kBN / 32; ++ch) {  // 32 scores -> 16 packed bf16 pairs per store
+          uint32_t pk_local[16];
+          uint32_t* pk = pk_out ? pk_out + ch * 16 : pk_local;
 #pragma unroll
-          for (int j = 16; j < kBN; j += 16)
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              m8[q] = fmax3(m8[q], __uint_as_float(sv[j + 2 * q]), __uint_as_float(sv[j + 2 * q + 1]));
-          const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-          const float mt = mx * sl2;
-          float alpha = 1.f;
-          bool resc = false;
-          if (mt > m_use + 8.f) {
-            if (m_use != -INFINITY) {
-              alpha = fast_exp2(m_use - mt);
-              resc = true;
-            }
-            m_use = mt;
-          }
-          const float base = (m_use == -INFINITY) ? 0.f : m_use;
-          const uint64_t sl2x2 = f2_pack(sl2, sl2);
-          const uint64_t nbase2 = f2_pack(-base, -base);
-          // exponentials on the SFU (ex2.approx), two per pair of scores
-          uint64_t acc[4] = {0, 0, 0, 0};
-#pragma unroll
-          for (int ch = 0; ch < kBN / 32; ++ch) {  // 32 scores -> 16 packed bf16 pairs per store
-            uint32_t pk[16];
-#pragma unroll
-            for (int pp = 0; pp < 16; ++pp) {
-              const int j = ch * 32 + 2 * pp;
-              const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), sl2x2, nbase2);
-              float x0, x1;
-              f2_unpack(x2, x0, x1);
+          for (int pp = 0; pp < 16; ++pp) {
+            const int j = ch * 32 + 2 * pp;
+            const uint64_t x2 =
+                f2_fma(f2_pack(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), sl2x2, nbase2);
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
 #if RA_EXP_F16X2
-              float q0, q1;
-              exp2_f16x2(x0, x1, q0, q1);
-              const uint64_t e2 = f2_pack(q0, q1);
+            float q0, q1;
+            exp2_f16x2(x0, x1, q0, q1);
+            const uint64_t e2 = f2_pack(q0, q1);
 #else
-              const uint64_t e2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
+            const uint64_t e2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
 #endif
-              acc[pp & 3] = f2_add(acc[pp & 3], e2);
-              float p0, p1;
-              f2_unpack(e2, p0, p1);
-              pk[pp] = pack_bf16x2(p0, p1);
-            }
-            tmem_st16(tS + ch * 16, pk);
+            acc[pp & 3] = f2_add(acc[pp & 3], e2);
+            float p0, p1;
+            f2_unpack(e2, p0, p1);
+            pk[pp] = pack_bf16x2(p0, p1);
           }
-          const uint64_t acc2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
-          float ps0, ps1;
-          f2_unpack(acc2, ps0, ps1);
-          l_sum = l_sum * alpha + (ps0 + ps1);
-          tmem_wait_st();
-          // O of this tile is stable here: S_X(c) was committed after the
-          // P V product of tile c-1, so its completion implies that one's.
-          if (c > 0 && __any_sync(0xffffffffu, resc)) {
-            tc_fence_after();
+          if (!pk_out) tmem_st16(tS + ch * 16, pk);
+        }
+        const uint64_t acc2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+        float ps0, ps1;
+        f2_unpack(acc2, ps0, ps1);
+        return ps0 + ps1;
+      };
+      // Common case: the exponentials against the running base m_use, with no
+      // tile maximum.  Kept when every value stays <= 2^15 (their sum does),
+      // which bf16 P and the fp32 sums hold exactly as well as values <= 1:
+      // out = O / l and lse = ln 2 * (m_use + log2 l) are exact for any base.
+      float psum = 0.f;
+      bool done = false;
+      if (__all_sync(0xffffffffu, m_use != -INFINITY)) {
+        uint32_t pk[kBN / 2];
+        psum = exps(m_use, pk);
+        done = __all_sync(0xffffffffu, psum <= kFastSumLimit);
+        if (done) {
 #pragma unroll
-            for (int q = 0; q < D / 32; ++q) {
-              uint32_t ov[32];
-              tmem_ld32_wait(tO + 32 * q, ov);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-              tmem_st32(tO + 32 * q, ov);
-            }
-            tmem_wait_st();
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(BPF(x)));
-          ++c;
+          for (int ch = 0; ch < kBN / 32; ++ch) tmem_st16(tS + ch * 16, pk + ch * 16);
+        } else {
+          load_s();  // S is still in TMEM: nothing was stored over it
         }
       }
+      // Otherwise (a row's first tile, or a score that rose more than about 8
+      // above the base): the tile maximum; the base is raised when the tile
+      // maximum exceeds it by more than 8, and the exponentials redone.
+      float alpha = 1.f;
+      bool resc = false;
+      if (!done) {
+        // row maximum: 3-input max, 8 independent chains of depth 8
+        float m8[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) m8[q] = fmaxf(__uint_as_float(sv[2 * q]), __uint_as_float(sv[2 * q + 1]));
+#pragma unroll
+        for (int j = 16; j < kBN; j += 16)
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            m8[q] = fmax3(m8[q], __uint_as_float(sv[j + 2 * q]), __uint_as_float(sv[j + 2 * q + 1]));
+        const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+        const float mt = mx * sl2;
+        if (mt > m_use + 8.f) {
+          if (m_use != -INFINITY) {
+            alpha = fast_exp2(m_use - mt);
+            resc = true;
+          }
+          m_use = mt;
+        }
+        psum = exps(m_use == -INFINITY ? 0.f : m_use, nullptr);
+      }
+      l_sum = l_sum * alpha + psum;
+      tmem_wait_st();
+      // O of this tile is stable here: S_X(c) was committed after the
+      // P V product of tile c-1, so its completion implies that one's.
+      if (c > 0 && __any_sync(0xffffffffu, resc)) {
+        tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t ov[32];
+          tmem_ld32_wait(tO + 32 * q, ov);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_st32(tO + 32 * q, ov);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BPF(x)));
+      ++c;
+    }
 
     // ------------------------------------------------------------ epilogue
     // Each tile's rows are normalised (and, in KV-split mode, stitched with
