@@ -137,7 +137,9 @@ struct AttnSmem {
   static constexpr int kNBar = 1 + 2 * kNSK + 2 * kNSV + 2 + 2 + 2 + 1;
   static constexpr int kTmemSlot = kBar + kNBar * 8;
   static constexpr int kAbort = kTmemSlot + 4;
-  static constexpr int kBytes = kAbort + 4 + 1024;  // + slack to align the base to 1024
+  static constexpr int kTotal = kAbort + 4;               // KV tiles of the CTA's sequence
+  static constexpr int kSegTab = (kTotal + 4 + 15) & ~15;  // SegTile[2 * kMaxBlocks]
+  static constexpr int kBytes = kSegTab + 2 * kMaxBlocks * 32 + 1024;  // + slack to align the base to 1024
   static_assert(kBytes <= 232448, "shared memory budget");
 };
 
@@ -165,15 +167,23 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   }
 }
 
+// One KV segment of the CTA's sequence with its tile counts for the CTA's
+// last row (nt) and the last rows of tiles A and B (na, nb); the kernel fills
+// a table of these in shared memory once, one segment per lane.
+struct SegTile {
+  Seg seg;
+  int nt, na, nb, pad[2];
+};
+static_assert(sizeof(SegTile) == 32, "segment table entry");
+
 // A walk over the CTA's KV tiles in schedule order: segment sg (KV block
 // s = sg / nseg of the CTA's list, segment e = sg % nseg) and tile t inside it,
-// with the segment itself and its tile counts for the CTA's last row (nt) and
-// the last rows of tiles A and B (na, nb).  The launch arguments are only read
-// when the walk enters a segment, so a step costs a few integer operations.
+// with the segment's tile counts for the CTA's last row (nt) and the last rows
+// of tiles A and B (na, nb).  The segment table is only read when the walk
+// enters a segment, so a step costs a few integer operations.
 struct KvWalk {
   int sg, t;
   int nt, na, nb;
-  Seg seg;
 };
 
 // Tiling modes (compile-time: each kernel instantiation carries only its own
@@ -221,26 +231,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int last_u = max(last_a, last_b);  // the CTA's last row: its KV range covers both tiles
   auto seg_of = [&](int s_, int e_) -> const Seg& { return a.kvseg[a.kv_list[qi][s_]][e_]; };
 
-  int total = 0;
-  for (int s = 0; s < a.nkv; ++s)
-    for (int e = 0; e < a.nseg; ++e) total += tiles_for(a, seg_of(s, e), last_u);
-  // this CTA's share [lo, hi) of the sequence (the cluster splits it in equal parts)
-  const int lo = kCl > 1 ? crank * total / kCl : 0;
-  const int hi = kCl > 1 ? (crank + 1) * total / kCl : total;
-  int work = hi - lo;
-  // Tile x's share of the CTA's KV tiles.  u = index in the CTA's sequence,
-  // t = index inside the segment.  KV-split: A takes [0, half), B [half, total).
-  const int half = (total + 1) / 2;
   // Walk helpers (see KvWalk): enter the segment sg (skipping segments the
   // CTA sees nothing of), start at the CTA's u-th tile, step to the next tile.
   const int nsg = a.nkv * a.nseg;
+  const SegTile* seg_tab = reinterpret_cast<const SegTile*>(smem + SL::kSegTab);
   auto enter = [&](KvWalk& k) {
     for (; k.sg < nsg; ++k.sg) {
-      k.seg = a.kvseg[a.kv_list[qi][k.sg / a.nseg]][k.sg % a.nseg];
-      k.nt = tiles_for(a, k.seg, last_u);
-      if (k.nt > 0) {
-        k.na = tiles_for(a, k.seg, last_a);
-        k.nb = tiles_for(a, k.seg, last_b);
+      const SegTile& e = seg_tab[k.sg];
+      if (e.nt > 0) {
+        k.nt = e.nt;
+        k.na = e.na;
+        k.nb = e.nb;
         return;
       }
     }
@@ -286,10 +287,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     fence_mbar_init();
   }
   if (warp == kMmaWarp) tmem_alloc(sb + SL::kTmemSlot, 512);
+  if (warp == kMmaWarp + 1) {
+    // the segment table, one segment per lane, and the CTA's tile count
+    int nt = 0;
+    if (lane < nsg) {
+      SegTile e;
+      e.seg = seg_of(lane / a.nseg, lane % a.nseg);
+      nt = e.nt = tiles_for(a, e.seg, last_u);
+      e.na = tiles_for(a, e.seg, last_a);
+      e.nb = tiles_for(a, e.seg, last_b);
+      e.pad[0] = e.pad[1] = 0;
+      reinterpret_cast<SegTile*>(smem + SL::kSegTab)[lane] = e;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) nt += __shfl_xor_sync(0xffffffffu, nt, o);
+    if (lane == 0) *reinterpret_cast<int*>(smem + SL::kTotal) = nt;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + SL::kTmemSlot);
+  const int total = *reinterpret_cast<volatile int*>(smem + SL::kTotal);
+  // this CTA's share [lo, hi) of the sequence (the cluster splits it in equal parts)
+  const int lo = kCl > 1 ? crank * total / kCl : 0;
+  const int hi = kCl > 1 ? (crank + 1) * total / kCl : total;
+  int work = hi - lo;
+  // Tile x's share of the CTA's KV tiles.  u = index in the CTA's sequence,
+  // t = index inside the segment.  KV-split: A takes [0, half), B [half, total).
+  const int half = (total + 1) / 2;
   if (*abort_flag) work = 0;
 
   // ---- staging buffers and the final row write (see the epilogue)
@@ -395,7 +420,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int g2 = 0; g2 < work && ok; ++g2) {
         const bool use_b = split && (g2 & 1);
         const int t = use_b ? wb.t : wa.t;
-        const Seg ks = use_b ? wb.seg : wa.seg;
+        const Seg ks = seg_tab[use_b ? wb.sg : wa.sg].seg;
         const int sk = g % NSK, sv = g % NSV;
         if (!mbar_wait(bar(BKE(sk)), ((g / NSK) & 1) ^ 1, abort_flag)) { ok = false; break; }
         mbar_expect_tx(bar(BKF(sk)), SL::kTile);
@@ -560,7 +585,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (!split && w.t >= (x ? w.nb : w.na)) continue;
       if (w.sg != lim_sg) {
         lim_sg = w.sg;
-        lim = visible_count(a, w.seg, qpos);
+        lim = visible_count(a, seg_tab[w.sg].seg, qpos);
       }
       const int t = w.t;
       ok = mbar_wait(bar(BSF(x)), c & 1, abort_flag);
