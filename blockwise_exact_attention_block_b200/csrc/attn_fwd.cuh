@@ -356,39 +356,56 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                                     : static_cast<long long>(b) * a.acc_brows + qs.mem + my_row0;
     const int per = kBM / nw;
     const int wr0 = wi * per;
-    const bool bf16_out = a.mode == kModeFinal && a.out_bf16;
-    const int lpr = bf16_out ? D / 8 : D / 4;  // lanes per row: 16 B per lane
-    const int rpi = 32 / lpr;                  // rows per warp instruction
-    const int ci = lane % lpr;
-    for (int r0 = 0; r0 < per; r0 += rpi) {
-      const int r = wr0 + r0 + lane / lpr;
-      if (r >= my_rows || r0 + lane / lpr >= per) continue;
-      const long long grow = (row_base + r) * a.Hq + h;
-      const float* src = stage + r * kStride;
-      if (bf16_out) {
-        const float4 lo4 = *reinterpret_cast<const float4*>(src + 8 * ci);
-        const float4 hi4 = *reinterpret_cast<const float4*>(src + 8 * ci + 4);
-        uint4 o;
-        o.x = pack_bf16x2(lo4.x, lo4.y);
-        o.y = pack_bf16x2(lo4.z, lo4.w);
-        o.z = pack_bf16x2(hi4.x, hi4.y);
-        o.w = pack_bf16x2(hi4.z, hi4.w);
-        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + grow * D)[ci] = o;
-      } else {
-        float4 v = *reinterpret_cast<const float4*>(src + 4 * ci);
-        float4* dst = reinterpret_cast<float4*>((a.mode == kModeFinal ? static_cast<float*>(a.out) : a.acc_out) +
-                                                grow * D) + ci;
-        if (a.mode == kModeMerge) {
-          const float wr = stage_w[r];
-          if (wr == 0.f) continue;
-          const float4 old = *dst;
-          v.x = merge_out(old.x, v.x, wr);
-          v.y = merge_out(old.y, v.y, wr);
-          v.z = merge_out(old.z, v.z, wr);
-          v.w = merge_out(old.w, v.w, wr);
+    const long long first = (row_base + wr0) * a.Hq + h;  // output row index of row wr0
+    const long long rstride = static_cast<long long>(a.Hq) * D;  // elements between consecutive rows
+    if (a.mode == kModeFinal && a.out_bf16) {
+      constexpr int lpr = D / 8, rpi = 32 / lpr;  // 16 B (8 bf16) per lane
+      const int ci = lane % lpr, rl = lane / lpr;
+      __nv_bfloat16* dst0 = static_cast<__nv_bfloat16*>(a.out) + first * D + 8 * ci;
+#pragma unroll 4
+      for (int r0 = 0; r0 < per; r0 += rpi) {
+        const int r = r0 + rl;
+        if (r < per && wr0 + r < my_rows) {
+          const float* src = stage + (wr0 + r) * kStride + 8 * ci;
+          const float4 lo4 = *reinterpret_cast<const float4*>(src);
+          const float4 hi4 = *reinterpret_cast<const float4*>(src + 4);
+          uint4 o;
+          o.x = pack_bf16x2(lo4.x, lo4.y);
+          o.y = pack_bf16x2(lo4.z, lo4.w);
+          o.z = pack_bf16x2(hi4.x, hi4.y);
+          o.w = pack_bf16x2(hi4.z, hi4.w);
+          *reinterpret_cast<uint4*>(dst0 + r * rstride) = o;
         }
-        *dst = v;
       }
+      return;
+    }
+    constexpr int lpr = D / 4, rpi = 32 / lpr;  // 16 B (4 floats) per lane
+    const int ci = lane % lpr, rl = lane / lpr;
+    float* dst0 = (a.mode == kModeFinal ? static_cast<float*>(a.out) : a.acc_out) + first * D + 4 * ci;
+    if (a.mode != kModeMerge) {
+#pragma unroll 4
+      for (int r0 = 0; r0 < per; r0 += rpi) {
+        const int r = r0 + rl;
+        if (r < per && wr0 + r < my_rows)
+          *reinterpret_cast<float4*>(dst0 + r * rstride) =
+              *reinterpret_cast<const float4*>(stage + (wr0 + r) * kStride + 4 * ci);
+      }
+      return;
+    }
+    // epilogue-fused schedule: the staged block partial merged into the running rows
+    for (int r0 = 0; r0 < per; r0 += rpi) {
+      const int r = r0 + rl;
+      if (r >= per || wr0 + r >= my_rows) continue;
+      const float wr = stage_w[wr0 + r];
+      if (wr == 0.f) continue;
+      float4* dst = reinterpret_cast<float4*>(dst0 + r * rstride);
+      float4 v = *reinterpret_cast<const float4*>(stage + (wr0 + r) * kStride + 4 * ci);
+      const float4 old = *dst;
+      v.x = merge_out(old.x, v.x, wr);
+      v.y = merge_out(old.y, v.y, wr);
+      v.z = merge_out(old.z, v.z, wr);
+      v.w = merge_out(old.w, v.w, wr);
+      *dst = v;
     }
   };
 
@@ -707,27 +724,65 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
 
     // ------------------------------------------------------------ epilogue
-    // Each tile's rows are normalised (and, in KV-split mode, stitched with
-    // the other half by the merge rule) into a staging buffer in shared
-    // memory, then every warp writes its 32 rows to HBM as whole, coalesced
-    // rows (commit_rows).  The K/V rings hold the staging buffers: they are
-    // idle once the last P V product of both tiles has landed (barrier below).
+    // Each tile's rows are normalised into a staging buffer in shared memory,
+    // then every warp writes whole rows to HBM with coalesced stores.  The K/V
+    // rings hold the staging buffers: they are idle once the last P V products
+    // of both tiles have landed (barrier below).
     if (ok && c > 0) {
       ok = mbar_wait(bar(BOD(x)), (c - 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
     }
-    float* stage = stage_of(x);
-    float* stage_w = stage + kBM * kStride;  // per-row merge weight (epilogue-fused mode)
-    float* stage_l = stage_w + kBM;          // per-row lse of the staged partial
+    const bool has = ok && l_sum > 0.f;
+    const float inv = has ? 1.f / l_sum : 0.f;
+    const float row_lse = has ? (m_use + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
     named_barrier_sync(1, 256);  // both tiles' MMAs are complete: the rings are free
     fence_proxy_async_smem();
-    if (split && x == 1) {
-      // B's normalised partial and its lse, for A to merge
-      const bool has = ok && l_sum > 0.f;
-      const float inv = has ? 1.f / l_sum : 0.f;
-      stage_l[row] = has ? (m_use + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
+    if (split) {
+      // KV-split: both tiles hold a partial of the same 128 rows.  The two
+      // warps of a row exchange (lse, 1/l) through shared memory, then each
+      // stitches half of the columns with the merge rule, reading both
+      // partials straight from tensor memory (same lanes).
+      float* xch = stage_of(1);  // [tile][lse, 1/l][row]
+      xch[x * 2 * kBM + row] = row_lse;
+      xch[x * 2 * kBM + kBM + row] = inv;
+      named_barrier_sync(1, 256);
+      tc_fence_after();
+      const float lse_a = xch[row], inv_a = xch[kBM + row];
+      const float lse_b = xch[2 * kBM + row], inv_b = xch[3 * kBM + row];
+      const bool has_a = lse_a != -INFINITY, has_b = lse_b != -INFINITY;
+      // tensor-memory loads are warp-collective: guarded by warp-uniform tile counts
+      const bool ld_a = ok && half > 0, ld_b = ok && total - half > 0;
+      const MergeWeights mw = merge_weights(lse_a, lse_b);
+      float* stage = stage_of(0);
+      if (x == 0) stage[kBM * kStride + kBM + row] = mw.lse;
+      const uint32_t tOa = tmem + lane_base + 256, tOb = tmem + lane_base + 384;
+#pragma unroll
+      for (int q = 0; q < D / 64; ++q) {
+        const int col = x * (D / 2) + 32 * q;  // this warpgroup's half of the columns
+        uint32_t oa[32], ob[32];
+        if (ld_a) tmem_ld32_wait(tOa + col, oa);
+        if (ld_b) tmem_ld32_wait(tOb + col, ob);
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          float v[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float va = ld_a && has_a ? __uint_as_float(oa[i + k]) * inv_a : 0.f;
+            const float vb = ld_b && has_b ? __uint_as_float(ob[i + k]) * inv_b : 0.f;
+            v[k] = merge_out(va, vb, mw.w);
+          }
+          *reinterpret_cast<float4*>(stage + row * kStride + col + i) = make_float4(v[0], v[1], v[2], v[3]);
+        }
+      }
+      if (x == 0 && (ok || work == 0)) commit_lse(0);
+      named_barrier_sync(1, 256);  // every row is staged (and its merge weight recorded)
+      if (ok || work == 0) store_rows(0, warp, 8);
+    } else if (ok || work == 0) {
+      // row pairs: each tile stages and writes its own rows
+      float* stage = stage_of(x);
+      stage[kBM * kStride + kBM + row] = row_lse;
       uint32_t ov[D];
-      if (ok && c > 0) {
+      if (c > 0) {  // c is uniform across the warp
         tc_fence_after();
         if constexpr (D == 128) tmem_ld128_wait(tO, ov);
         else tmem_ld64_wait(tO, ov);
@@ -737,54 +792,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         *reinterpret_cast<float4*>(stage + row * kStride + i) =
             make_float4(has ? __uint_as_float(ov[i]) * inv : 0.f, has ? __uint_as_float(ov[i + 1]) * inv : 0.f,
                         has ? __uint_as_float(ov[i + 2]) * inv : 0.f, has ? __uint_as_float(ov[i + 3]) * inv : 0.f);
-    }
-    if (split) named_barrier_sync(1, 256);
-    // rows are staged by every tile in row-pair mode, by A alone in KV-split mode
-    const bool writer = (ok || work == 0) && !(split && x == 1);
-    if (writer) {
-      const bool has = l_sum > 0.f;
-      const float inv = has ? 1.f / l_sum : 0.f;
-      float row_lse = has ? (m_use + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
-      const float* bstage = stage_of(1);  // B's region (KV-split)
-      MergeWeights mwb;  // KV-split: weight of B's partial in this row
-      mwb.w = 0.f;
-      if (split) {
-        mwb = merge_weights(row_lse, bstage[kBM * kStride + kBM + row]);
-        row_lse = mwb.lse;
-      }
-      stage_l[row] = row_lse;
-      uint32_t ov[D];
-      if (c > 0) {  // c is uniform across the warp
-        tc_fence_after();
-        if constexpr (D == 128) tmem_ld128_wait(tO, ov);
-        else tmem_ld64_wait(tO, ov);
-      }
-#pragma unroll
-      for (int i = 0; i < D; i += 4) {
-        float4 v = make_float4(has ? __uint_as_float(ov[i]) * inv : 0.f, has ? __uint_as_float(ov[i + 1]) * inv : 0.f,
-                               has ? __uint_as_float(ov[i + 2]) * inv : 0.f,
-                               has ? __uint_as_float(ov[i + 3]) * inv : 0.f);
-        if (split && mwb.w != 0.f) {
-          const float4 xb = *reinterpret_cast<const float4*>(bstage + row * kStride + i);
-          v.x = merge_out(v.x, xb.x, mwb.w);
-          v.y = merge_out(v.y, xb.y, mwb.w);
-          v.z = merge_out(v.z, xb.z, mwb.w);
-          v.w = merge_out(v.w, xb.w, mwb.w);
-        }
-        *reinterpret_cast<float4*>(stage + row * kStride + i) = v;
-      }
       if constexpr (kCl == 1) {
         commit_lse(x);
-        if (!split) {  // each warp stores the 32 rows it staged
-          __syncwarp();
-          store_rows(x, warp & 3, 4);
-        }
+        __syncwarp();  // each warp stores the 32 rows it staged
+        store_rows(x, warp & 3, 4);
       }
-    }
-    if (split) {
-      // KV-split: only A staged rows; all 8 warps store them (16 rows each)
-      named_barrier_sync(1, 256);
-      if (ok || work == 0) store_rows(0, warp, 8);
     }
   }
 
