@@ -40,7 +40,8 @@ SCHEDS = {"auto": RA_SCHED_AUTO, "unfused": RA_SCHED_UNFUSED, "fused": RA_SCHED_
 
 EXPORTED = ["ra_block_attn", "ra_merge_partial", "ra_merge_partials", "ra_ring_attention",
             "ra_ring_attention_workspace", "ra_zigzag_permute", "ra_get_device_status",
-            "ra_status_string", "ra_version", "ra_ring_attention_noalloc", "ra_noalloc_scratch_bytes"]
+            "ra_status_string", "ra_version", "ra_ring_attention_noalloc", "ra_noalloc_scratch_bytes",
+            "ra_decode_attention", "ra_decode_workspace", "ra_decode_splits"]
 
 
 class ra_options(ctypes.Structure):
@@ -76,6 +77,12 @@ _lib.ra_status_string.argtypes = [_i]
 _lib.ra_status_string.restype = ctypes.c_char_p
 _lib.ra_version.argtypes = []
 _lib.ra_version.restype = ctypes.c_char_p
+_lib.ra_decode_attention.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _sz, _vp]
+_lib.ra_decode_attention.restype = _i
+_lib.ra_decode_workspace.argtypes = [_i, _i, _i, _i, _i, _i, _i]
+_lib.ra_decode_workspace.restype = _sz
+_lib.ra_decode_splits.argtypes = [_i, _i, _i, _i, _i, _i, _i]
+_lib.ra_decode_splits.restype = _i
 
 
 class RAError(RuntimeError):
@@ -255,3 +262,43 @@ def ra_zigzag_permute(src, n_blocks: int, inverse: bool = False, dst=None, strea
 def ra_get_device_status(stream=None) -> int:
     """Reads and clears the device status word (synchronises the stream)."""
     return _lib.ra_get_device_status(_stream(stream))
+
+
+def ra_decode_workspace(B, Tq, Skv, Hq, Hkv, D, n_splits=0) -> int:
+    n = _lib.ra_decode_workspace(B, Tq, Skv, Hq, Hkv, D, n_splits)
+    if n == ctypes.c_size_t(-1).value:
+        raise RAError(RA_ERR_INVALID_ARG, "ra_decode_workspace")
+    return n
+
+
+def ra_decode_splits(B, Tq, Skv, Hq, Hkv, D, n_splits=0) -> int:
+    n = _lib.ra_decode_splits(B, Tq, Skv, Hq, Hkv, D, n_splits)
+    if n < 0:
+        raise RAError(RA_ERR_INVALID_ARG, "ra_decode_splits")
+    return n
+
+
+def ra_decode_attention(q, k, v, causal: bool = True, n_splits: int = 0, out=None, lse=None, out_dtype=None,
+                        workspace=None, stream=None):
+    """Decode attention of q [B, Tq, Hq, D] (the last Tq tokens) over the
+    cache k, v [B, Skv, Hkv, D], bf16, in n_splits chunks (0 = chosen to fill
+    the GPU).  Returns (out [B, Tq, Hq, D], lse [B, Tq, Hq] fp32)."""
+    B, Tq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    for t in (q, k, v):
+        if not t.is_contiguous():
+            raise RAError(RA_ERR_INVALID_ARG, "ra_decode_attention (tensors must be contiguous)")
+    odt = out_dtype or (out.dtype if out is not None else torch.float32)
+    if out is None:
+        out = torch.empty((B, Tq, Hq, D), dtype=odt, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Tq, Hq), dtype=torch.float32, device=q.device)
+    need = ra_decode_workspace(B, Tq, Skv, Hq, Hkv, D, n_splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _check(_lib.ra_decode_attention(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q.dtype), B, Tq, Skv, Hq, Hkv, D,
+                                    1 if causal else 0, n_splits, _ptr(out), _dtype_code(out.dtype), _ptr(lse),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream(stream)), "ra_decode_attention")
+    return out, lse
+

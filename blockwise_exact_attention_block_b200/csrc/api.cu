@@ -17,6 +17,7 @@
 #include <mutex>
 
 #include "attn_fwd.cuh"
+#include "decode.cuh"
 #include "merge.cuh"
 #include "permute.cuh"
 
@@ -42,17 +43,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor viewed as [NB][L][H][D] (innermost last), box = 128 rows x 64
-// columns of one head, 128-byte swizzle.  Rows beyond L read as zero.  The
+// bf16 tensor viewed as [NB][L][H][D] (innermost last), box = box_rows rows x
+// 64 columns of one head, 128-byte swizzle.  Rows beyond L read as zero.  The
 // 4th coordinate is the batch index.
-bool make_map(CUtensorMap* m, const void* ptr, int D, int H, int L, int NB) {
+bool make_map(CUtensorMap* m, const void* ptr, int D, int H, int L, int NB, int box_rows = kBM) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(NB)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
                                  static_cast<cuuint64_t>(L) * H * D * 2};
-  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kBM), 1};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t es[4] = {1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -308,6 +309,108 @@ bool valid_opts(const ra_options* o) {
   return o->sched >= RA_SCHED_AUTO && o->sched <= RA_SCHED_PERSISTENT;
 }
 
+// Chunking of a decode call: chunk = keys per CTA (a multiple of the tile),
+// n = chunks that cover the cache.  n_req = 0 picks the n that minimises
+// waves x (tiles per chunk + 2), the time of a grid of n * B * Hkv CTAs when
+// `per_sm` CTAs fit on each SM (from the kernel's shared memory) and each costs
+// about two tiles beyond its own, over chunks of at least four tiles.
+struct DecodePlan {
+  int n, chunk;
+  size_t part_out, part_lse, total;
+};
+
+int decode_smem_bytes(int D, int rows) {
+  const int mt = (rows + 15) / 16 <= 1 ? 1 : ((rows + 15) / 16 <= 2 ? 2 : 4);
+  if (D == 128) return mt == 1 ? DecSmem<128, 1>::kBytes : mt == 2 ? DecSmem<128, 2>::kBytes : DecSmem<128, 4>::kBytes;
+  return mt == 1 ? DecSmem<64, 1>::kBytes : mt == 2 ? DecSmem<64, 2>::kBytes : DecSmem<64, 4>::kBytes;
+}
+
+DecodePlan decode_plan(int B, int Tq, int Skv, int Hq, int Hkv, int D, int n_req) {
+  DecodePlan p;
+  memset(&p, 0, sizeof(p));
+  const long long tiles = (Skv + kDecKeys - 1) / kDecKeys;
+  long long n = n_req;
+  if (n <= 0) {
+    const long long ctas = static_cast<long long>(B) * Hkv;
+    const int smem = decode_smem_bytes(D, (Hq / Hkv) * Tq);
+    int per_sm = 233472 / (smem + 1024);  // 228 KB of shared memory per SM, 1 KB reserved per CTA
+    per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
+    const long long slots = static_cast<long long>(sm_count()) * per_sm;
+    const long long max_n = (tiles + 3) / 4 < 1 ? 1 : (tiles + 3) / 4;
+    long long best = -1;
+    for (long long c = 1; c <= max_n && c <= 65535; ++c) {
+      const long long per = (tiles + c - 1) / c;                 // tiles per chunk
+      if (c > 1 && (tiles + per - 1) / per != c) continue;       // the same chunking as a smaller count
+      const long long waves = (c * ctas + slots - 1) / slots;
+      const long long cost = waves * (per + 2);
+      if (best < 0 || cost < best) {
+        best = cost;
+        n = c;
+      }
+    }
+  }
+  long long chunk = (Skv + n - 1) / n;
+  chunk = (chunk + kDecKeys - 1) / kDecKeys * kDecKeys;
+  p.n = static_cast<int>((Skv + chunk - 1) / chunk);
+  if (p.n > 65535) {  // the chunk index is gridDim.y
+    chunk = ((Skv + 65534) / 65535 + kDecKeys - 1) / kDecKeys * kDecKeys;
+    p.n = static_cast<int>((Skv + chunk - 1) / chunk);
+  }
+  p.chunk = static_cast<int>(chunk);
+  const size_t rows = static_cast<size_t>(B) * Tq * Hq;
+  p.part_out = 0;
+  p.part_lse = align256(static_cast<size_t>(p.n) * rows * D * 4);
+  p.total = align256(p.part_lse + static_cast<size_t>(p.n) * rows * 4);
+  return p;
+}
+
+ra_status check_decode(int B, int Tq, int Skv, int Hq, int Hkv, int D, int n_splits) {
+  if (B < 1 || Tq < 1 || Skv < 1 || Hq < 1 || Hkv < 1 || n_splits < 0) return RA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0 || Tq > Skv) return RA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
+  if ((Hq / Hkv) * Tq > kDecMaxRows) return RA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv > 65535) return RA_ERR_UNSUPPORTED;
+  return RA_OK;
+}
+
+template <int D, int MT>
+ra_status launch_decode_partial(const DecodeArgs& a, const DecodePlan& p, const CUtensorMap& mk,
+                                const CUtensorMap& mv, cudaStream_t st) {
+  using SL = DecSmem<D, MT>;
+  static int attr_set[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(decode_partial_kernel<D, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SL::kBytes) != cudaSuccess)
+      return RA_ERR_CUDA;
+    attr_set[dev] = 1;
+  }
+  decode_partial_kernel<D, MT><<<dim3(a.Hkv, p.n, a.B), kDecThreads, SL::kBytes, st>>>(mk, mv, a);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int D>
+ra_status launch_decode_d(const DecodeArgs& a, const DecodePlan& p, const CUtensorMap& mk, const CUtensorMap& mv,
+                          void* out, ra_dtype out_dtype, float* lse, cudaStream_t st) {
+  // 16-row tiles of query rows per KV head: 1, 2 or 4
+  const int mt = (a.rows + 15) / 16;
+  ra_status s = mt <= 1   ? launch_decode_partial<D, 1>(a, p, mk, mv, st)
+                : mt <= 2 ? launch_decode_partial<D, 2>(a, p, mk, mv, st)
+                          : launch_decode_partial<D, 4>(a, p, mk, mv, st);
+  if (s != RA_OK) return s;
+  const long long rows = static_cast<long long>(a.B) * a.Tq * a.Hq;
+  const long long blocks = rows;  // one CTA per row
+  if (blocks > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
+  if (out_dtype == RA_BF16)
+    decode_combine_kernel<D, __nv_bfloat16><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        a.part_out, a.part_lse, p.n, rows, static_cast<__nv_bfloat16*>(out), lse);
+  else
+    decode_combine_kernel<D, float><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        a.part_out, a.part_lse, p.n, rows, static_cast<float*>(out), lse);
+  return cuda_status(cudaGetLastError());
+}
+
 }  // namespace
 
 extern "C" {
@@ -561,6 +664,51 @@ ra_status ra_ring_attention(const void* q, const void* k, const void* v, ra_dtyp
     s = cuda_status(cudaGetLastError());
   }
   return s;
+}
+
+size_t ra_decode_workspace(int B, int Tq, int Skv, int Hq, int Hkv, int D, int n_splits) {
+  if (check_decode(B, Tq, Skv, Hq, Hkv, D, n_splits) != RA_OK) return static_cast<size_t>(-1);
+  return decode_plan(B, Tq, Skv, Hq, Hkv, D, n_splits).total;
+}
+
+int ra_decode_splits(int B, int Tq, int Skv, int Hq, int Hkv, int D, int n_splits) {
+  if (check_decode(B, Tq, Skv, Hq, Hkv, D, n_splits) != RA_OK) return -1;
+  return decode_plan(B, Tq, Skv, Hq, Hkv, D, n_splits).n;
+}
+
+ra_status ra_decode_attention(const void* q, const void* k, const void* v, ra_dtype in_dtype, int B, int Tq, int Skv,
+                              int Hq, int Hkv, int D, int causal, int n_splits, void* out, ra_dtype out_dtype,
+                              float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  ra_status s = check_decode(B, Tq, Skv, Hq, Hkv, D, n_splits);
+  if (s != RA_OK) return s;
+  if (in_dtype != RA_BF16) return in_dtype == RA_F32 ? RA_ERR_UNSUPPORTED : RA_ERR_INVALID_ARG;
+  if (out_dtype != RA_F32 && out_dtype != RA_BF16) return RA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out || !lse) return RA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (reinterpret_cast<uintptr_t>(lse) & 3))
+    return RA_ERR_INVALID_ARG;
+  const DecodePlan p = decode_plan(B, Tq, Skv, Hq, Hkv, D, n_splits);
+  if (!workspace || workspace_bytes < p.total) return RA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return RA_ERR_INVALID_ARG;
+  CUtensorMap mk, mv;
+  if (!make_map(&mk, k, D, Hkv, Skv, B, kDecKeys) || !make_map(&mv, v, D, Hkv, Skv, B, kDecKeys)) return RA_ERR_CUDA;
+  DecodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = B;
+  a.Tq = Tq;
+  a.Skv = Skv;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.groups = Hq / Hkv;
+  a.causal = causal != 0;
+  a.rows = a.groups * Tq;
+  a.chunk = p.chunk;
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(D)));
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.part_out = reinterpret_cast<float*>(static_cast<char*>(workspace) + p.part_out);
+  a.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + p.part_lse);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return D == 128 ? launch_decode_d<128>(a, p, mk, mv, out, out_dtype, lse, st)
+                  : launch_decode_d<64>(a, p, mk, mv, out, out_dtype, lse, st);
 }
 
 }  // extern "C"

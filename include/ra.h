@@ -231,6 +231,39 @@ ra_status ra_ring_attention_noalloc(const void* q, const void* k, const void* v,
 /* Size in bytes of the fixed scratch array behind ra_ring_attention_noalloc. */
 size_t ra_noalloc_scratch_bytes(void);
 
+/*
+ * ra_decode_attention - decode-phase attention over a KV cache, by chunks.
+ * [TR] "Reading between the lines": the decode phase as KV-cache chunking;
+ * every chunk's partial (out, lse) is stitched with the update rule of
+ * ra_merge_partial ("What carries the argument"), in chunk order.
+ *  q          device, bf16, [B, Tq, Hq, D]: the last Tq tokens of each
+ *             sequence; query token i has position Skv - Tq + i.
+ *  k, v       device, bf16, [B, Skv, Hkv, D]: the cache of tokens 0..Skv-1.
+ *  in_dtype   must be RA_BF16 (else RA_ERR_UNSUPPORTED).
+ *  Hq, Hkv    Hq % Hkv == 0; query head h reads KV head h / (Hq / Hkv);
+ *             (Hq / Hkv) * Tq <= 64 (else RA_ERR_UNSUPPORTED).  D in {64, 128}.
+ *             1 <= Tq <= Skv.
+ *  causal     nonzero: query token i sees keys j <= Skv - Tq + i.
+ *  n_splits   chunks of the cache (0 = enough to fill the GPU); the chunk
+ *             length is rounded up to 64 keys, so the count actually used is
+ *             ra_decode_splits() of the same arguments.
+ *  out        device, out_dtype (RA_F32 or RA_BF16, nearest even), [B, Tq, Hq, D].
+ *  lse        device fp32 [B, Tq, Hq], natural log.
+ *  workspace  device scratch of ra_decode_workspace() bytes, 256-byte aligned
+ *             (the per-chunk partials).
+ */
+ra_status ra_decode_attention(const void* q, const void* k, const void* v, ra_dtype in_dtype,
+                              int B, int Tq, int Skv, int Hq, int Hkv, int D, int causal,
+                              int n_splits, void* out, ra_dtype out_dtype, float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes of ra_decode_attention for these arguments ((size_t)-1 when
+ * they are invalid). */
+size_t ra_decode_workspace(int B, int Tq, int Skv, int Hq, int Hkv, int D, int n_splits);
+
+/* Chunks ra_decode_attention uses for these arguments (-1 when invalid). */
+int ra_decode_splits(int B, int Tq, int Skv, int Hq, int Hkv, int D, int n_splits);
+
 /* Reads and clears the device status word (synchronises `stream`).  Returns
  * RA_OK, RA_ERR_TIMEOUT or RA_ERR_DEVICE_BOUNDS, or RA_ERR_CUDA when the read
  * itself fails. */

@@ -13,6 +13,8 @@ Recipe (one CPU ``torch.Generator`` per call, seeded):
   Tensors above ``CHUNK_ROWS`` tokens are drawn in consecutive token chunks of
   ``CHUNK_ROWS`` from the same generator, so that a 1M-token draw never holds
   more than one fp32 chunk at a time.
+* decode workloads draw ``q`` ``[B, Tq, Hq, D]``, then the cache ``k``, ``v``
+  ``[B, Skv, Hkv, D]``, ``randn`` rounded to bf16, in that order.
 * merge workloads draw, for partial i = 0..k-1 in turn, ``out_i`` ~ N(0, 1) of
   ``[T, H, D]`` fp32 and then ``lse_i`` ~ U(-5, 15) of ``[T, H]`` fp32
   (``rand * 20 - 5``).
@@ -68,6 +70,41 @@ WORKLOADS = {
     "long1m": AttnWorkload("long1m", 1, 1048576, 8, 2, 128, 8, True, "zigzag", "bf16", "bf16"),
 }
 
+
+@dataclass(frozen=True)
+class DecodeWorkload:
+    """Decode phase: the last Tq tokens against a cache of Skv tokens."""
+
+    name: str
+    B: int
+    Tq: int
+    Skv: int
+    Hq: int
+    Hkv: int
+    D: int
+    causal: bool
+    out_dtype: str  # "f32" or "bf16"
+
+    @property
+    def gqa_groups(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def bytes(self) -> int:
+        """Bytes one call must move: the K and V cache and Q read (bf16), out
+        written and lse (fp32) written."""
+        ob = 4 if self.out_dtype == "f32" else 2
+        rows = self.B * self.Tq * self.Hq
+        return 2 * 2 * self.B * self.Skv * self.Hkv * self.D + rows * self.D * (2 + ob) + rows * 4
+
+
+# Decode against the long-context cache (one token, the 1M-token GQA shape)
+# and a batch of sequences shaped like the 24k profile with four tokens each.
+DECODE_WORKLOADS = {
+    "decode1m": DecodeWorkload("decode1m", 1, 1, 1048576, 8, 2, 128, True, "f32"),
+    "decode24k": DecodeWorkload("decode24k", 8, 4, 24000, 32, 8, 128, True, "f32"),
+}
+
 MERGE_HEADS = 32
 MERGE_DIM = 128
 MERGE_TOKENS = [4096 * 2 ** i for i in range(9)]  # 4,096 ... 1,048,576
@@ -93,6 +130,16 @@ def attention_inputs(B: int, S: int, Hq: int, Hkv: int, D: int, dtype: str = "bf
     q = _draw(gen, (B, S, Hq, D), tdt)
     k = _draw(gen, (B, S, Hkv, D), tdt)
     v = _draw(gen, (B, S, Hkv, D), tdt)
+    return q, k, v
+
+
+def decode_inputs(B: int, Tq: int, Skv: int, Hq: int, Hkv: int, D: int, seed: int = 0):
+    """q [B, Tq, Hq, D], then the cache k, v [B, Skv, Hkv, D], bf16, drawn in
+    that order from one generator."""
+    gen = torch.Generator("cpu").manual_seed(seed)
+    q = _draw(gen, (B, Tq, Hq, D), torch.bfloat16)
+    k = _draw(gen, (B, Skv, Hkv, D), torch.bfloat16)
+    v = _draw(gen, (B, Skv, Hkv, D), torch.bfloat16)
     return q, k, v
 
 

@@ -131,3 +131,48 @@ def test_workspace_query(ra):
     assert n_unf16 >= n_unf + 4096 * 8 * 128 * 4
     with pytest.raises(ra.RAError):
         ra.ra_ring_attention_workspace(1, 4095, 8, 128, 4, 1, "zigzag")
+
+
+def decode(ra, **kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, in_dtype=ra.RA_BF16, B=1, Tq=1, Skv=4096, Hq=8, Hkv=2, D=128, causal=1,
+                n_splits=0, out=FAKE, out_dtype=ra.RA_F32, lse=FAKE, ws=FAKE, ws_bytes=1 << 40, stream=None)
+    args.update(kw)
+    return ra._lib.ra_decode_attention(args["q"], args["k"], args["v"], args["in_dtype"], args["B"], args["Tq"],
+                                       args["Skv"], args["Hq"], args["Hkv"], args["D"], args["causal"],
+                                       args["n_splits"], args["out"], args["out_dtype"], args["lse"], args["ws"],
+                                       args["ws_bytes"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Hq=6, Hkv=4), 1),                 # Hq not a multiple of Hkv
+    (dict(Tq=5000), 1),                     # more query tokens than cached ones
+    (dict(Skv=0), 1),
+    (dict(n_splits=-1), 1),
+    (dict(D=96), 2),
+    (dict(Hq=32, Hkv=2, Tq=5), 2),          # 16 heads x 5 tokens > 64 rows per KV head
+    (dict(in_dtype=0), 2),                  # fp32 cache
+    (dict(out_dtype=7), 1),
+    (dict(q=None), 1),
+    (dict(lse=FAKE + 2), 1),                # misaligned lse
+    (dict(ws_bytes=16), 3),                 # workspace too small
+    (dict(ws=FAKE + 64), 1),                # workspace not 256-byte aligned
+])
+def test_decode_rejects_invalid_arguments(ra, kw, status):
+    assert decode(ra, **kw) == status
+
+
+def test_decode_plan(ra):
+    # chunks cover the cache in multiples of 64 keys; workspace holds one
+    # fp32 partial (out and lse) per chunk and row
+    for (B, Tq, Skv, Hq, Hkv, D, n) in [(1, 1, 1048576, 8, 2, 128, 0), (8, 4, 24000, 32, 8, 128, 0),
+                                         (2, 3, 1000, 8, 2, 128, 5), (1, 1, 64, 2, 1, 64, 0), (1, 2, 100, 4, 4, 64, 50)]:
+        splits = ra.ra_decode_splits(B, Tq, Skv, Hq, Hkv, D, n)
+        chunk = -(-Skv // (n if n else splits))
+        chunk = -(-chunk // 64) * 64
+        assert splits == -(-Skv // chunk)
+        assert 1 <= splits <= max(n, 1) if n else splits >= 1
+        rows = B * Tq * Hq
+        assert ra.ra_decode_workspace(B, Tq, Skv, Hq, Hkv, D, n) >= splits * rows * (D + 1) * 4
+    assert ra._lib.ra_decode_splits(1, 1, 10, 8, 3, 128, 0) == -1
+    with pytest.raises(ra.RAError):
+        ra.ra_decode_workspace(1, 1, 10, 8, 3, 128, 0)

@@ -14,7 +14,7 @@ import torch
 
 from oracle import attention as F
 from oracle import blockwise as K
-from seeded_inputs import WORKLOADS, attention_inputs, merge_inputs, workload_inputs
+from seeded_inputs import DECODE_WORKLOADS, WORKLOADS, attention_inputs, decode_inputs, merge_inputs, workload_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -297,4 +297,62 @@ def test_long1m_workload_sampled_rows(cuda_lib):
     torch.cuda.synchronize()
     rows = sample_rows(w, per_head=24)
     check_sampled(w, q, k, v, o, l, rows, "long1m")
+    assert ra.ra_get_device_status() == 0
+
+
+# ------------------------------------------------------------------ decode
+
+DECODE_CASES = [
+    # B, Tq, Skv, Hq, Hkv, D, causal, n_splits
+    (2, 1, 1000, 8, 2, 128, True, 0),       # ragged cache (not a multiple of 64), GQA 4
+    (1, 3, 777, 4, 4, 64, True, 5),         # MHA, D=64, three causal tokens, explicit chunks
+    (1, 16, 2048, 16, 4, 128, True, 3),     # 4 heads x 16 tokens = 64 rows per KV head (the limit)
+    (3, 2, 130, 6, 2, 128, False, 1),       # non-causal, one chunk, ragged last tile
+    (1, 1, 64, 2, 1, 128, True, 0),         # exactly one tile
+    (1, 4, 4, 4, 2, 128, True, 0),          # Tq == Skv: the first token sees key 0 only
+    (2, 2, 5000, 8, 8, 64, True, 40),       # many chunks
+]
+
+
+@pytest.mark.parametrize("case", DECODE_CASES,
+                         ids=lambda c: f"B{c[0]}Tq{c[1]}S{c[2]}H{c[3]}/{c[4]}D{c[5]}{'C' if c[6] else ''}n{c[7]}")
+def test_decode_matches_oracle(cuda_lib, case):
+    ra = cuda_lib
+    B, Tq, Skv, Hq, Hkv, D, causal, n = case
+    q, k, v = decode_inputs(B, Tq, Skv, Hq, Hkv, D, seed=11)
+    ro, rl = F.decode_attention(q, k, v, causal, Hq // Hkv)
+    for out_dtype in (torch.float32, torch.bfloat16):
+        o, l = ra.ra_decode_attention(q.cuda(), k.cuda(), v.cuda(), causal, n, out_dtype=out_dtype)
+        assert_close_bf16(to_np(o), ro, f"decode out {out_dtype}")
+        assert_close_bf16(to_np(l), rl, f"decode lse {out_dtype}")
+    assert ra.ra_get_device_status() == 0
+
+
+def test_decode_chunk_count_invariance(cuda_lib):
+    # the chunks are stitched by the merge rule: any chunk count gives the
+    # same attention (to rounding), and matches the oracle's own chunked form
+    ra = cuda_lib
+    B, Tq, Skv, Hq, Hkv, D = 1, 2, 3000, 8, 2, 128
+    q, k, v = decode_inputs(B, Tq, Skv, Hq, Hkv, D, seed=12)
+    ro, rl = K.decode_blockwise(q, k, v, True, Hq // Hkv, 7)
+    base = None
+    for n in (1, 2, 7, 23, 0):
+        o, l = ra.ra_decode_attention(q.cuda(), k.cuda(), v.cuda(), True, n)
+        assert_close_bf16(to_np(o), ro, f"decode out n={n}")
+        assert_close_bf16(to_np(l), rl, f"decode lse n={n}")
+        if base is None:
+            base = (o.clone(), l.clone())
+        assert float((o - base[0]).abs().max()) <= 2e-3
+        assert float((l - base[1]).abs().max()) <= 2e-3
+
+
+@pytest.mark.parametrize("name", sorted(DECODE_WORKLOADS))
+def test_decode_workloads_full_oracle(cuda_lib, name):
+    ra = cuda_lib
+    w = DECODE_WORKLOADS[name]
+    q, k, v = decode_inputs(w.B, w.Tq, w.Skv, w.Hq, w.Hkv, w.D)
+    o, l = ra.ra_decode_attention(q.cuda(), k.cuda(), v.cuda(), w.causal, 0)
+    ro, rl = F.decode_attention(q, k, v, w.causal, w.gqa_groups)
+    assert_close_bf16(to_np(o), ro, f"{name} out")
+    assert_close_bf16(to_np(l), rl, f"{name} lse")
     assert ra.ra_get_device_status() == 0
