@@ -57,6 +57,9 @@ def parse():
                    help="time the merge kernels over the whole token / partial sweep instead")
     p.add_argument("--merge-T", type=int, nargs="*", default=None, help="token counts of the merge sweep")
     p.add_argument("--merge-k", type=int, nargs="*", default=None, help="partial counts of the merge sweep")
+    p.add_argument("--decode", action="store_true",
+                   help="time decode-phase attention over a KV cache (both decode workloads) instead")
+    p.add_argument("--no-decode", action="store_true")
     a = p.parse_args()
     if a.steps is None:
         a.steps = DEFAULT_STEPS[a.workload]
@@ -170,6 +173,16 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def local_gpu_id(dev):
+    """nvidia-smi id of this process's GPU (its UUID; the index as fallback)."""
+    import torch
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = getattr(props, "uuid", None)
+    if gpu_id is None:
+        return dev.index
+    return f"GPU-{gpu_id}" if not str(gpu_id).startswith("GPU-") else gpu_id
+
+
 def kernel_sha():
     import hashlib
     h = hashlib.sha256()
@@ -254,6 +267,73 @@ def bench_merge(ra, dev, T, k, reps, flush, kway=False):
     return nbytes / (ms * 1e-3) / 1e9, ms
 
 
+# ------------------------------------------------------------ decode phase
+
+def bench_decode(ra, dev, w, reps, flush):
+    """GB/s of one ra_decode_attention call on workload w: the bytes it must
+    move (K and V cache and Q read, out and lse written) over the call's time,
+    both kernels (chunk partials and their merge) included.  The cache is
+    drawn on the device (its values do not change the time; the parity tests
+    use the seeded host inputs)."""
+    import torch
+    g = torch.Generator(device=dev).manual_seed(2)
+    q = torch.randn((w.B, w.Tq, w.Hq, w.D), device=dev, generator=g).to(torch.bfloat16)
+    k = torch.randn((w.B, w.Skv, w.Hkv, w.D), device=dev, generator=g).to(torch.bfloat16)
+    v = torch.randn((w.B, w.Skv, w.Hkv, w.D), device=dev, generator=g).to(torch.bfloat16)
+    out = torch.empty((w.B, w.Tq, w.Hq, w.D), dtype=torch.float32 if w.out_dtype == "f32" else torch.bfloat16,
+                      device=dev)
+    lse = torch.empty((w.B, w.Tq, w.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(ra.ra_decode_workspace(w.B, w.Tq, w.Skv, w.Hq, w.Hkv, w.D, 0), 1), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+    times = []
+    for rep in range(reps + 3):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        ra.ra_decode_attention(q, k, v, w.causal, 0, out=out, lse=lse, workspace=ws)
+        e1.record(stream)
+        e1.synchronize()
+        if rep >= 3:
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    splits = ra.ra_decode_splits(w.B, w.Tq, w.Skv, w.Hq, w.Hkv, w.D, 0)
+    del q, k, v, out, lse, ws
+    torch.cuda.empty_cache()
+    return w.bytes / (ms * 1e-3) / 1e9, ms, splits
+
+
+def run_decode(args):
+    import torch
+    import blockwise_exact_attention_block_b200 as ra
+    from seeded_inputs import DECODE_WORKLOADS
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    pk, pk_kind = peaks()
+    lines = []
+    clocks = Clocks(local_gpu_id(dev))
+    time.sleep(0.3)
+    for name, w in DECODE_WORKLOADS.items():
+        gbs, ms, splits = bench_decode(ra, dev, w, min(max(args.steps, 10), 50), flush)
+        lines.append((name, w, gbs, ms, splits))
+    clk = clocks.stop()
+    status = ra.ra_get_device_status()
+    for name, w, gbs, ms, splits in lines:
+        line = {"metric": "decode GB/s (% of HBM peak)", "value": gbs, "unit": "GB/s", "n_gpus": 1, "steps": None,
+                "warmup": 3, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic (device randn, bf16-rounded)",
+                "config": {"workload": name, "B": w.B, "Tq": w.Tq, "Skv": w.Skv, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                           "causal": w.causal, "chunks": splits, "bytes_per_call": w.bytes,
+                           "l2": f"flushed ({L2_FLUSH_BYTES >> 20} MiB write between calls)"},
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                             "frac": gbs / pk["hbm_gbs"], "traffic": None, "kernel": "decode_partial_kernel",
+                             "peak_source": f"{pk_kind} copy bandwidth"},
+                "clocks": clk, "gpu_launches": 2, "device_status": ra.ra_status_string(status)}
+        print(json.dumps(line))
+    return 0 if status == 0 else 1
+
+
 # ---------------------------------------------------------------- our arm
 
 def launches_per_step(w, sched):
@@ -315,10 +395,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    props = torch.cuda.get_device_properties(dev)
-    gpu_id = getattr(props, "uuid", None)
-    gpu_id = f"GPU-{gpu_id}" if gpu_id is not None and not str(gpu_id).startswith("GPU-") else gpu_id
-    clocks = Clocks(gpu_id if gpu_id is not None else local)
+    clocks = Clocks(local_gpu_id(dev))
     time.sleep(0.3)
     for i in range(K):
         flush.zero_()
@@ -390,6 +467,15 @@ def run_ours(args):
                  "GB/s": gbs, "ms": mms, "peak_GB/s": pk["hbm_gbs"], "frac": gbs / pk["hbm_gbs"],
                  "bytes_per_row": 12 * 128 + 12}
 
+    decode = None
+    if not args.no_decode and world == 1:
+        from seeded_inputs import DECODE_WORKLOADS
+        dw = DECODE_WORKLOADS["decode1m"]
+        gbs, dms, splits = bench_decode(ra, dev, dw, 10, flush)
+        decode = {"kernel": "decode_partial_kernel + decode_combine_kernel", "workload": "decode1m", "B": dw.B,
+                  "Tq": dw.Tq, "Skv": dw.Skv, "Hq": dw.Hq, "Hkv": dw.Hkv, "D": dw.D, "chunks": splits,
+                  "GB/s": gbs, "ms": dms, "peak_GB/s": pk["hbm_gbs"], "frac": gbs / pk["hbm_gbs"]}
+
     value = replica_throughput(w.flops, world, K, total_ms)
     line = {"metric": "causal-adj attention TFLOP/s (% of dense bf16 peak)", "value": value, "unit": "TFLOP/s",
             "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
@@ -399,7 +485,7 @@ def run_ours(args):
                                                f"L2 {l2_bytes >> 20} MiB)"),
             "pct_of_peak": 100.0 * value / peak, "attn_kernel_ms": attn_mean, "roofline": roof,
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "gpu_launches": K * launches_per_step(w, args.sched),
-            "merge": merge,
+            "merge": merge, "decode": decode,
             "device_status": ra.ra_status_string(status)}
     if rank == 0:
         print(json.dumps(line))
@@ -446,6 +532,8 @@ def main():
         return run_reference(args)
     if args.merge_sweep:
         return run_merge_sweep(args)
+    if args.decode:
+        return run_decode(args)
     return run_ours(args)
 
 
