@@ -30,10 +30,12 @@ Modules:
 * ``attention``  - plain full softmax attention (the definition), fp64.
 * ``blockwise``  - partitions, ring / TokenRing schedules, per-block partials
   and the pages' merge rule, fp64.  Shares no code with ``attention``.
+* ``backward``   - gradients (dq, dk, dv): the definition over whole rows and
+  the same gradient as sums over block pairs rebuilt from the full-row lse.
 
 Every function here is pinned by ``tests/test_oracle.py`` against brute force,
 closed forms, a library routine or an invariant the pages fix.  The timing
 columns of the pages (7.6 ms / 3.5 ms on four A10s) are "parity unpinned": they
 need hardware and a model shape the pages do not give.
 """
-from . import attention, blockwise  # noqa: F401
+from . import attention, backward, blockwise  # noqa: F401

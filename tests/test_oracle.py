@@ -405,3 +405,122 @@ def test_kv_splits_cover_the_cache():
         sp = K.kv_splits(Skv, n)
         assert sp[0][0] == 0 and sp[-1][1] == Skv
         assert all(a1 == b0 for (_, a1), (b0, _) in zip(sp, sp[1:]))
+
+
+# ---------------------------------------------------------------- backward
+
+from oracle import backward as G  # noqa: E402
+
+
+def autograd_backward(q, k, v, dout, causal, groups):
+    """torch's scaled-dot-product attention in fp64, differentiated by autograd."""
+    qt, kt, vt = (torch.as_tensor(np.asarray(x, dtype=np.float64)).permute(0, 2, 1, 3).clone().requires_grad_(True)
+                  for x in (q, k, v))
+    kr = kt.repeat_interleave(groups, dim=1)
+    vr = vt.repeat_interleave(groups, dim=1)
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kr, vr, is_causal=causal)
+    o.backward(torch.as_tensor(np.asarray(dout, dtype=np.float64)).permute(0, 2, 1, 3))
+    return tuple(t.grad.permute(0, 2, 1, 3).numpy() for t in (qt, kt, vt))
+
+
+def rand64(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("groups", [1, 2])
+def test_backward_matches_autograd(causal, groups):
+    B, S, Hq, D = 2, 40, 4, 16
+    q, do = rand64((B, S, Hq, D), 1), rand64((B, S, Hq, D), 2)
+    k, v = rand64((B, S, Hq // groups, D), 3), rand64((B, S, Hq // groups, D), 4)
+    got = G.attention_backward(q, k, v, do, causal, groups)
+    ref = autograd_backward(q, k, v, do, causal, groups)
+    for a, r, nm in zip(got, ref, "qkv"):
+        assert np.max(np.abs(a - r)) <= 1e-10 * max(1.0, np.max(np.abs(r))), nm
+
+
+def test_backward_finite_differences():
+    # central differences of L = sum(dO * O) on a tiny problem
+    B, S, Hq, Hkv, D = 1, 5, 2, 1, 3
+    q, k, v = rand64((B, S, Hq, D), 5), rand64((B, S, Hkv, D), 6), rand64((B, S, Hkv, D), 7)
+    do = rand64((B, S, Hq, D), 8)
+    dq, dk, dv = G.attention_backward(q, k, v, do, True, 2)
+
+    def loss(qq, kk, vv):
+        o, _ = F.full_attention(qq, kk, vv, True, 2)
+        return float(np.sum(do * o))
+
+    eps = 1e-6
+    for x, g in ((q, dq), (k, dk), (v, dv)):
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = [xp if x is y else y for y in (q, k, v)]
+            args_m = [xm if x is y else y for y in (q, k, v)]
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(fd - g[idx]) <= 1e-6, (idx, fd, g[idx])
+
+
+def test_backward_closed_forms():
+    B, S, Hq, Hkv, D = 1, 24, 4, 2, 8
+    q, k, v = rand64((B, S, Hq, D), 9), rand64((B, S, Hkv, D), 10), rand64((B, S, Hkv, D), 11)
+    # no upstream gradient, no gradient
+    for gr in G.attention_backward(q, k, v, np.zeros((B, S, Hq, D)), True, 2):
+        assert np.all(gr == 0.0)
+    do = rand64((B, S, Hq, D), 12)
+    dq, dk, dv = G.attention_backward(q, k, v, do, True, 2)
+    # softmax rows sum to one: the keys' dV adds up to the queries' dO of the group
+    assert np.allclose(dv.sum(axis=1), do.reshape(B, S, Hkv, 2, D).sum(axis=(1, 3)), atol=1e-12)
+    # every dS row sums to zero: the keys' dK adds up to zero
+    assert np.allclose(dk.sum(axis=1), 0.0, atol=1e-12)
+
+
+@pytest.mark.parametrize("partition,n", [("contiguous", 1), ("contiguous", 4), ("zigzag", 2), ("zigzag", 4)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_blockwise_backward_equals_full(partition, n, causal):
+    B, S, Hq, Hkv, D = 2, 64, 4, 2, 8
+    q, k, v = attention_inputs(B, S, Hq, Hkv, D, "f32", seed=13)
+    do = torch.as_tensor(rand64((B, S, Hq, D), 14))
+    o, lse = F.full_attention(q, k, v, causal, 2)
+    ref = G.attention_backward(q, k, v, do, causal, 2)
+    got = G.blockwise_backward(q, k, v, do, o, lse, n, causal, partition, 2)
+    for a, r in zip(got, ref):
+        assert np.max(np.abs(a - r)) <= TOL * max(1.0, np.max(np.abs(r)))
+
+
+def _backward_mutant(kind):
+    """A copy of the definition with one plausible mistake planted."""
+    def f(q, k, v, dout, causal, groups):
+        q, k, v, do = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dout))
+        B, S, Hq, D = q.shape
+        s = 1.0 / math.sqrt(D)
+        dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+        mask = np.tril(np.ones((S, S), dtype=bool)) if causal else np.ones((S, S), dtype=bool)
+        for b in range(B):
+            for h in range(Hq):
+                g = h // groups
+                lg = np.where(mask, (q[b, :, h] @ k[b, :, g].T) * s, -np.inf)
+                e = np.exp(lg - lg.max(axis=1, keepdims=True))
+                p = e / e.sum(axis=1, keepdims=True)
+                o = p @ v[b, :, g]
+                dv[b, :, g] += p.T @ do[b, :, h]
+                dp = do[b, :, h] @ v[b, :, g].T
+                delta = 0.0 if kind == "no_delta" else (do[b, :, h] * o).sum(axis=1, keepdims=True)
+                ds = p * (dp - delta)
+                dq[b, :, h] = (1.0 if kind == "no_scale" else s) * (ds @ k[b, :, g])
+                dk[b, :, g] += s * ((ds if kind == "ds_not_transposed" else ds.T) @ q[b, :, h])
+        return dq, dk, dv
+    return f
+
+
+@pytest.mark.parametrize("kind", ["no_delta", "no_scale", "ds_not_transposed"])
+def test_backward_pins_catch_planted_mistakes(kind):
+    B, S, Hq, D = 1, 16, 2, 16
+    q, do = rand64((B, S, Hq, D), 15), rand64((B, S, Hq, D), 16)
+    k, v = rand64((B, S, Hq, D), 17), rand64((B, S, Hq, D), 18)
+    ref = autograd_backward(q, k, v, do, True, 1)
+    got = _backward_mutant(kind)(q, k, v, do, True, 1)
+    assert any(np.max(np.abs(a - r)) > 1e-6 for a, r in zip(got, ref))
+    good = _backward_mutant("none")(q, k, v, do, True, 1)
+    assert all(np.max(np.abs(a - r)) <= 1e-10 for a, r in zip(good, ref))
