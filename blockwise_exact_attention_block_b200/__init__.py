@@ -41,7 +41,8 @@ SCHEDS = {"auto": RA_SCHED_AUTO, "unfused": RA_SCHED_UNFUSED, "fused": RA_SCHED_
 EXPORTED = ["ra_block_attn", "ra_merge_partial", "ra_merge_partials", "ra_ring_attention",
             "ra_ring_attention_workspace", "ra_zigzag_permute", "ra_get_device_status",
             "ra_status_string", "ra_version", "ra_ring_attention_noalloc", "ra_noalloc_scratch_bytes",
-            "ra_decode_attention", "ra_decode_workspace", "ra_decode_splits"]
+            "ra_decode_attention", "ra_decode_workspace", "ra_decode_splits", "ra_ring_attention_backward",
+            "ra_ring_attention_backward_workspace"]
 
 
 class ra_options(ctypes.Structure):
@@ -83,6 +84,11 @@ _lib.ra_decode_workspace.argtypes = [_i, _i, _i, _i, _i, _i, _i]
 _lib.ra_decode_workspace.restype = _sz
 _lib.ra_decode_splits.argtypes = [_i, _i, _i, _i, _i, _i, _i]
 _lib.ra_decode_splits.restype = _i
+_lib.ra_ring_attention_backward.argtypes = [_vp, _vp, _vp, _i, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
+                                            _vp, _vp, _vp, _vp, _sz, ctypes.POINTER(ra_options), _vp]
+_lib.ra_ring_attention_backward.restype = _i
+_lib.ra_ring_attention_backward_workspace.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
+_lib.ra_ring_attention_backward_workspace.restype = _sz
 
 
 class RAError(RuntimeError):
@@ -243,6 +249,48 @@ def ra_ring_attention_noalloc(q, k, v, n_blocks: int, causal: bool, partition: s
                                           _dtype_code(out.dtype), _ptr(lse), ctypes.byref(o), _stream(stream)),
            "ra_ring_attention_noalloc")
     return out, lse
+
+
+def ra_ring_attention_backward_workspace(B, S, Hq, D, n_blocks, gqa_groups, partition="contiguous",
+                                         in_dtype=torch.bfloat16) -> int:
+    n = _lib.ra_ring_attention_backward_workspace(B, S, Hq, D, n_blocks, gqa_groups, PARTITIONS[partition],
+                                                  _dtype_code(in_dtype))
+    if n == ctypes.c_size_t(-1).value:
+        raise RAError(RA_ERR_INVALID_ARG, "ra_ring_attention_backward_workspace")
+    return n
+
+
+def ra_ring_attention_backward(q, k, v, out, lse, dout, n_blocks: int, causal: bool, partition: str = "contiguous",
+                               gqa_groups: int | None = None, dq=None, dk=None, dv=None, workspace=None,
+                               order: str = "ring", stream=None, attn_events=None):
+    """Gradients of ra_ring_attention.  q, k, v, dout share one dtype (bf16 or
+    fp32); out, lse are the forward's results.  Returns fp32 (dq, dk, dv).
+
+    attn_events: optional pair of torch.cuda.Event recorded around the two
+    tensor-core launches (dK/dV, then dQ) inside the call."""
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if gqa_groups is None:
+        gqa_groups = Hq // Hkv
+    if dout.dtype != q.dtype:
+        raise ValueError("dout must have the dtype of q, k and v")
+    if dq is None:
+        dq = torch.empty((B, S, Hq, D), dtype=torch.float32, device=q.device)
+    if dk is None:
+        dk = torch.empty((B, S, Hkv, D), dtype=torch.float32, device=q.device)
+    if dv is None:
+        dv = torch.empty((B, S, Hkv, D), dtype=torch.float32, device=q.device)
+    need = ra_ring_attention_backward_workspace(B, S, Hq, D, n_blocks, gqa_groups, partition, q.dtype)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    o = _opts(order, "auto", attn_events)
+    _check(_lib.ra_ring_attention_backward(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q.dtype), _ptr(out),
+                                           _dtype_code(out.dtype), _ptr(lse), _ptr(dout), B, S, Hq, D, n_blocks,
+                                           int(bool(causal)), PARTITIONS[partition], gqa_groups, _ptr(dq), _ptr(dk),
+                                           _ptr(dv), _ptr(workspace), ws_bytes, ctypes.byref(o), _stream(stream)),
+           "ra_ring_attention_backward")
+    return dq, dk, dv
 
 
 def ra_noalloc_scratch_bytes() -> int:

@@ -17,6 +17,7 @@
 #include <mutex>
 
 #include "attn_fwd.cuh"
+#include "attn_bwd.cuh"
 #include "decode.cuh"
 #include "merge.cuh"
 #include "permute.cuh"
@@ -411,6 +412,83 @@ ra_status launch_decode_d(const DecodeArgs& a, const DecodePlan& p, const CUtens
   return cuda_status(cudaGetLastError());
 }
 
+// ------------------------------------------------------------ backward
+// Workspace of ra_ring_attention_backward: Delta and lse * log2(e) as
+// [B][Hq][S] fp32, then the bf16 rounding of q, k, v and dout when in_dtype
+// is fp32.
+struct BwdPlan {
+  bool cast_inputs;
+  size_t delta, lse2, q, k, v, dout, total;
+};
+
+BwdPlan bwd_plan(const Geom& g, ra_dtype in_dtype) {
+  BwdPlan p;
+  memset(&p, 0, sizeof(p));
+  const size_t rows = static_cast<size_t>(g.B) * g.S;
+  size_t off = 0;
+  p.delta = off;
+  off = align256(off + rows * g.Hq * 4);
+  p.lse2 = off;
+  off = align256(off + rows * g.Hq * 4);
+  p.cast_inputs = in_dtype == RA_F32;
+  if (p.cast_inputs) {
+    p.q = off;
+    off = align256(off + rows * g.Hq * g.D * 2);
+    p.k = off;
+    off = align256(off + rows * g.Hkv * g.D * 2);
+    p.v = off;
+    off = align256(off + rows * g.Hkv * g.D * 2);
+    p.dout = off;
+    off = align256(off + rows * g.Hq * g.D * 2);
+  }
+  p.total = off;
+  return p;
+}
+
+// Segments of the backward launch in weight order: latest positions first
+// (queries that see the most keys) or earliest first (keys seen by the most
+// queries); every order is correct, this one shortens the tail of the grid.
+void bwd_segment_order(BwdArgs& a, bool latest_first) {
+  const int m = a.nblk * a.nseg;
+  for (int i = 0; i < m; ++i) a.seg_order[i] = static_cast<signed char>(i);
+  if (!a.causal) return;
+  for (int i = 1; i < m; ++i)
+    for (int j = i; j > 0; --j) {
+      const Seg& x = a.seg[a.seg_order[j] / a.nseg][a.seg_order[j] % a.nseg];
+      const Seg& y = a.seg[a.seg_order[j - 1] / a.nseg][a.seg_order[j - 1] % a.nseg];
+      if (latest_first ? x.pos > y.pos : x.pos < y.pos) {
+        const signed char t = a.seg_order[j];
+        a.seg_order[j] = a.seg_order[j - 1];
+        a.seg_order[j - 1] = t;
+      }
+    }
+}
+
+template <int D>
+ra_status launch_bwd_d(const BwdArgs& adq, const BwdArgs& adkv, const CUtensorMap& mq, const CUtensorMap& mk,
+                       const CUtensorMap& mv, const CUtensorMap& mdo, cudaStream_t st) {
+  using SL = BwdSmem<D>;
+  static int attr_set[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, SL::kBytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, SL::kBytes) !=
+            cudaSuccess)
+      return RA_ERR_CUDA;
+    attr_set[dev] = 1;
+  }
+  const long long tiles = static_cast<long long>(adq.B) * adq.nblk * adq.nseg * adq.seg_tiles;
+  const long long gkv = tiles * adkv.Hkv, gq = tiles * adq.Hq;
+  if (gq > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
+  bwd_dkv_kernel<D><<<static_cast<unsigned>(gkv), kBwdThreads, SL::kBytes, st>>>(mq, mk, mv, mdo, adkv);
+  ra_status s = cuda_status(cudaGetLastError());
+  if (s != RA_OK) return s;
+  bwd_dq_kernel<D><<<static_cast<unsigned>(gq), kBwdThreads, SL::kBytes, st>>>(mq, mk, mv, mdo, adq);
+  return cuda_status(cudaGetLastError());
+}
+
 }  // namespace
 
 extern "C" {
@@ -709,6 +787,122 @@ ra_status ra_decode_attention(const void* q, const void* k, const void* v, ra_dt
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return D == 128 ? launch_decode_d<128>(a, p, mk, mv, out, out_dtype, lse, st)
                   : launch_decode_d<64>(a, p, mk, mv, out, out_dtype, lse, st);
+}
+
+size_t ra_ring_attention_backward_workspace(int B, int S, int Hq, int D, int n_blocks, int gqa_groups,
+                                            ra_partition partition, ra_dtype in_dtype) {
+  if (gqa_groups < 1 || Hq % gqa_groups != 0) return static_cast<size_t>(-1);
+  Geom g;
+  if (check_geom(B, S, n_blocks, Hq, Hq / gqa_groups, D, partition, &g) != RA_OK) return static_cast<size_t>(-1);
+  if (in_dtype != RA_F32 && in_dtype != RA_BF16) return static_cast<size_t>(-1);
+  return bwd_plan(g, in_dtype).total;
+}
+
+ra_status ra_ring_attention_backward(const void* q, const void* k, const void* v, ra_dtype in_dtype,
+                                     const void* out, ra_dtype out_dtype, const float* lse, const void* dout,
+                                     int B, int S, int Hq, int D, int n_blocks, int causal, ra_partition partition,
+                                     int gqa_groups, float* dq, float* dk, float* dv, void* workspace,
+                                     size_t workspace_bytes, const ra_options* opts, void* stream) {
+  if (gqa_groups < 1 || Hq < 1 || Hq % gqa_groups != 0) return RA_ERR_INVALID_ARG;
+  Geom g;
+  ra_status s = check_geom(B, S, n_blocks, Hq, Hq / gqa_groups, D, partition, &g);
+  if (s != RA_OK) return s;
+  g.causal = causal != 0;
+  if (in_dtype != RA_F32 && in_dtype != RA_BF16) return RA_ERR_INVALID_ARG;
+  if (out_dtype != RA_F32 && out_dtype != RA_BF16) return RA_ERR_INVALID_ARG;
+  if (!valid_opts(opts)) return RA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv) return RA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return RA_ERR_INVALID_ARG;
+  const BwdPlan p = bwd_plan(g, in_dtype);
+  if (!workspace || workspace_bytes < p.total) return RA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return RA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  const long long rows = static_cast<long long>(B) * S;
+
+  // fp32 inputs are rounded to bf16 (nearest even) once, as in the forward
+  const void* qb = q;
+  const void* kb = k;
+  const void* vb = v;
+  const void* dob = dout;
+  if (p.cast_inputs) {
+    PermGeom ident;
+    memset(&ident, 0, sizeof(ident));
+    ident.S = S;
+    ident.L = g.L;
+    ident.n = g.n;
+    struct { const void* src; size_t off; int H; } mv[4] = {
+        {q, p.q, g.Hq}, {k, p.k, g.Hkv}, {v, p.v, g.Hkv}, {dout, p.dout, g.Hq}};
+    for (auto& m : mv) {
+      const long long row_elems = static_cast<long long>(m.H) * D;
+      permute_cast_kernel<float, __nv_bfloat16><<<grid_for(rows * row_elems / 8, 256), 256, 0, st>>>(
+          static_cast<const float*>(m.src), reinterpret_cast<__nv_bfloat16*>(ws + m.off), B, ident, row_elems, 0);
+      s = cuda_status(cudaGetLastError());
+      if (s != RA_OK) return s;
+    }
+    qb = ws + p.q;
+    kb = ws + p.k;
+    vb = ws + p.v;
+    dob = ws + p.dout;
+  }
+
+  // Delta = rowsum(dO * O) and lse * log2(e), per (batch, head) over positions
+  float* delta = reinterpret_cast<float*>(ws + p.delta);
+  float* lse2 = reinterpret_cast<float*>(ws + p.lse2);
+  const long long prep_threads = rows * Hq * (D / 4);
+  if (out_dtype == RA_F32)
+    bwd_prep_kernel<float><<<grid_for(prep_threads, 256), 256, 0, st>>>(
+        static_cast<const float*>(out), static_cast<const __nv_bfloat16*>(dob), lse, B, S, Hq, D, delta, lse2);
+  else
+    bwd_prep_kernel<__nv_bfloat16><<<grid_for(prep_threads, 256), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dob), lse, B, S, Hq, D, delta,
+        lse2);
+  s = cuda_status(cudaGetLastError());
+  if (s != RA_OK) return s;
+
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, qb, D, g.Hq, S, B) || !make_map(&mk, kb, D, g.Hkv, S, B) ||
+      !make_map(&mv, vb, D, g.Hkv, S, B) || !make_map(&mdo, dob, D, g.Hq, S, B))
+    return RA_ERR_CUDA;
+
+  BwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = B;
+  a.S = S;
+  a.Hq = Hq;
+  a.Hkv = g.Hkv;
+  a.groups = g.groups;
+  a.causal = g.causal;
+  a.nblk = g.n;
+  a.nseg = g.zigzag ? 2 : 1;
+  a.seg_tiles = (seg_len_of(g) + kBM - 1) / kBM;
+  a.scale = static_cast<float>(1.0 / sqrt(static_cast<double>(D)));
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(D)));
+  a.lse2 = lse2;
+  a.delta = delta;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  for (int r = 0; r < g.n; ++r) block_segments(g, r, false, a.seg[r]);
+  // dQ: query block r meets the KV blocks in the schedule's order (as in the
+  // forward); dK/dV: KV block j meets the query blocks that meet it there
+  const ra_order order = opts ? opts->order : RA_ORDER_RING;
+  BwdArgs adq = a, adkv = a;
+  for (int r = 0; r < g.n; ++r)
+    for (int t = 0; t < g.n; ++t) {
+      const int fwd = order == RA_ORDER_RING ? r - t : r + t;
+      const int bwd = order == RA_ORDER_RING ? r + t : r - t;
+      adq.order[r][t] = static_cast<signed char>(((fwd % g.n) + g.n) % g.n);
+      adkv.order[r][t] = static_cast<signed char>(((bwd % g.n) + g.n) % g.n);
+    }
+  bwd_segment_order(adq, true);
+  bwd_segment_order(adkv, false);
+  if (opts && opts->attn_event_begin) cudaEventRecord(static_cast<cudaEvent_t>(opts->attn_event_begin), st);
+  s = D == 128 ? launch_bwd_d<128>(adq, adkv, mq, mk, mv, mdo, st) : launch_bwd_d<64>(adq, adkv, mq, mk, mv, mdo, st);
+  if (s == RA_OK && opts && opts->attn_event_end) cudaEventRecord(static_cast<cudaEvent_t>(opts->attn_event_end), st);
+  return s;
 }
 
 }  // extern "C"

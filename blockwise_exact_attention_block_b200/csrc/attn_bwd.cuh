@@ -1,0 +1,659 @@
+// attn_bwd.cuh - gradients of exact blockwise attention on the 5th-generation
+// tensor cores (sm_100a).
+//
+// Anthology of the SOTA, SOTA-181: ring attention trains models, so the
+// blockwise computation has a backward pass; TokenRing review (pith.science,
+// arXiv 2412.20501), "What carries the argument": the forward returns, per
+// query row, the log-sum-exp of the whole row.  With that lse every
+// (query block, KV block) pair's share of the gradient is independent of the
+// other pairs, and the shares add up (s = 1 / sqrt(D)):
+//     P  = exp(s Q K^T - lse)            (rebuilt, never stored)
+//     dV += P^T dO                       dP = dO V^T
+//     dS = P (dP - Delta)                Delta = rowsum(dO * O)
+//     dQ += s dS K                       dK += s dS^T Q
+// Two kernels, each owning the output rows it writes (no atomics):
+//   bwd_dq_kernel:  one 128-row query tile of one head per CTA walks the KV
+//                   tiles its rows see, KV blocks in the schedule's order
+//                   (the query block stays, as in the ring);
+//   bwd_dkv_kernel: one 128-key tile of one KV head per CTA walks the query
+//                   tiles that see it, for every query head of its group
+//                   (the KV block stays, as in TokenRing).
+// bwd_prep_kernel first writes Delta and lse * log2(e) per (batch, head),
+// contiguous over positions.
+//
+// Warp roles (320 threads):
+//   warps 0-7  elementwise: thread (warp % 4) * 32 + lane owns TMEM lane /
+//              tile row (warp % 4) * 32 + lane; warps 0-3 take columns
+//              [0, 64) of the 128 x 128 score tile, warps 4-7 columns [64, 128)
+//   warp 8     TMA producer
+//   warp 9     TMEM allocator and MMA issuer (one thread)
+// Both kernels use only the forward kernel's operand forms: SS products of
+// K-major SW128 tiles, and TS products with a bf16 A operand in tensor memory
+// and an MN-major B tile.
+#pragma once
+
+#include "attn_fwd.cuh"
+#include "permute.cuh"
+
+namespace ra {
+
+constexpr int kBwdThreads = 320;
+constexpr int kBwdElem = 256;  // elementwise threads (warps 0-7)
+constexpr int kBwdProducer = 8;
+constexpr int kBwdMma = 9;
+
+struct BwdArgs {
+  int B, S, Hq, Hkv, groups, causal;
+  int nblk;            // ring blocks
+  int nseg;            // segments per block: 1 (contiguous) or 2 (zigzag)
+  int seg_tiles;       // 128-row tiles per segment
+  float scale;         // 1 / sqrt(D)
+  float scale_log2;    // log2(e) / sqrt(D)
+  const float* lse2;   // [B][Hq][S]: lse * log2(e)
+  const float* delta;  // [B][Hq][S]
+  float* dq;           // [B, S, Hq, D]
+  float* dk;           // [B, S, Hkv, D]
+  float* dv;           // [B, S, Hkv, D]
+  Seg seg[kMaxBlocks][2];                     // segments of block r (queries and keys alike)
+  signed char order[kMaxBlocks][kMaxBlocks];  // order[r][s]: s-th block that block r meets
+  signed char seg_order[2 * kMaxBlocks];      // (r * nseg + e) of the CTA segments, heaviest first
+};
+
+template <int D>
+struct BwdSmem {
+  static constexpr int kBox = kBM * 128;  // 128 rows x 64 bf16: one TMA box, 16 KB
+  static constexpr int kTile = kBox * (D / 64);
+  static constexpr int kNS = D == 128 ? 2 : 4;        // stages of the streamed pair
+  static constexpr int kX = 0;                        // stationary pair: (Q, dO) or (K, V)
+  static constexpr int kY = 2 * kTile;                // ring of streamed pairs
+  static constexpr int kStat = kY + kNS * 2 * kTile;  // dK/dV kernel: [2 sets][lse2 | delta][128]
+  static constexpr int kBar = kStat + 2 * 2 * kBM * 4;
+  // barriers: X, Yfull[NS], Yempty[NS], Sfull, Pfull, Odone, End
+  static constexpr int kNBar = 1 + 2 * kNS + 4;
+  static constexpr int kTmemSlot = kBar + kNBar * 8;
+  static constexpr int kAbort = kTmemSlot + 4;
+  static constexpr int kBytes = kAbort + 4 + 1024;  // + slack to align the base to 1024
+  static_assert(kBytes <= 232448, "shared memory budget");
+  // epilogue staging of two 128-row fp32 tiles of up to D columns (+4 pad)
+  static_assert(2 * kBM * (D + 4) * 4 <= kStat, "output staging fits in the tile buffers");
+};
+
+// TMEM columns: both kernels keep the two score-shaped products at [0, 128)
+// and [128, 256) and their fp32 accumulators from 256.
+constexpr int kTmS = 0, kTmP = 128, kTmAcc = 256;
+constexpr int kTmDS = 384;  // dQ kernel: bf16 dS (64 columns), clear of S, dP and dQ
+// dK/dV kernel: bf16 P^T written at [32, 96) over S^T, bf16 dS^T at [160, 224)
+// over dP^T.  Column half h of a row writes only columns that half h has
+// already read (see bwd_dkv_kernel), so the two halves never race.
+constexpr int kTmPT = 32, kTmDST = 160;
+
+// Delta = rowsum(dO * O) and lse * log2(e), written as [B][Hq][S].  D / 4
+// threads per row, 4 elements each.
+template <typename TO>
+__global__ void __launch_bounds__(256)
+    bwd_prep_kernel(const TO* __restrict__ out, const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
+                    int B, int S, int Hq, int D, float* __restrict__ delta, float* __restrict__ lse2) {
+  const int tpr = D / 4;  // 16 or 32: a power of two dividing 32
+  const long long rows = static_cast<long long>(B) * S * Hq;
+  const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long nthreads = static_cast<long long>(gridDim.x) * blockDim.x;
+  const int sub = threadIdx.x % tpr;
+  // every lane of a warp runs the same number of iterations (the row range is
+  // padded to whole warps), so the shuffles below see all 32 lanes
+  const long long rows_pad = (rows * tpr + 31) / 32 * 32 / tpr;
+  for (long long r = tid / tpr; r < rows_pad; r += nthreads / tpr) {
+    float acc = 0.f;
+    if (r < rows) {
+      const long long e = r * D + 4 * sub;
+      float o[4];
+      if constexpr (sizeof(TO) == 4) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(out + e));
+        o[0] = v.x, o[1] = v.y, o[2] = v.z, o[3] = v.w;
+      } else {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(out + e));
+        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&v);
+        o[0] = __low2float(hv[0]), o[1] = __high2float(hv[0]), o[2] = __low2float(hv[1]), o[3] = __high2float(hv[1]);
+      }
+      const uint2 w = __ldg(reinterpret_cast<const uint2*>(dout + e));
+      const __nv_bfloat162* gv = reinterpret_cast<const __nv_bfloat162*>(&w);
+      acc = o[0] * __low2float(gv[0]) + o[1] * __high2float(gv[0]) + o[2] * __low2float(gv[1]) +
+            o[3] * __high2float(gv[1]);
+    }
+    for (int m = tpr / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if (sub == 0 && r < rows) {
+      const int h = static_cast<int>(r % Hq);
+      const long long bs = r / Hq;
+      const int s = static_cast<int>(bs % S), b = static_cast<int>(bs / S);
+      const long long t = (static_cast<long long>(b) * Hq + h) * S + s;
+      delta[t] = acc;
+      lse2[t] = lse[r] * 1.4426950408889634f;
+    }
+  }
+}
+
+// Keys of segment kv visible to a query at original position qpos (a prefix
+// of the segment); qpos < 0 marks a padding row.
+__device__ __forceinline__ int bwd_visible(const BwdArgs& a, const Seg& kv, int qpos) {
+  if (qpos < 0) return 0;
+  if (!a.causal) return kv.len;
+  return min(max(qpos - kv.pos + 1, 0), kv.len);
+}
+
+// Two 32-column TMEM loads of this thread's lane, then one wait (warp-collective).
+__device__ __forceinline__ void tmem_ld32x2_wait(uint32_t ta, uint32_t tb, uint32_t (&va)[32], uint32_t (&vb)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,"
+      "%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(va[0]), "=r"(va[1]), "=r"(va[2]), "=r"(va[3]), "=r"(va[4]), "=r"(va[5]), "=r"(va[6]), "=r"(va[7]),
+        "=r"(va[8]), "=r"(va[9]), "=r"(va[10]), "=r"(va[11]), "=r"(va[12]), "=r"(va[13]), "=r"(va[14]),
+        "=r"(va[15]), "=r"(va[16]), "=r"(va[17]), "=r"(va[18]), "=r"(va[19]), "=r"(va[20]), "=r"(va[21]),
+        "=r"(va[22]), "=r"(va[23]), "=r"(va[24]), "=r"(va[25]), "=r"(va[26]), "=r"(va[27]), "=r"(va[28]),
+        "=r"(va[29]), "=r"(va[30]), "=r"(va[31]), "=r"(vb[0]), "=r"(vb[1]), "=r"(vb[2]), "=r"(vb[3]), "=r"(vb[4]),
+        "=r"(vb[5]), "=r"(vb[6]), "=r"(vb[7]), "=r"(vb[8]), "=r"(vb[9]), "=r"(vb[10]), "=r"(vb[11]), "=r"(vb[12]),
+        "=r"(vb[13]), "=r"(vb[14]), "=r"(vb[15]), "=r"(vb[16]), "=r"(vb[17]), "=r"(vb[18]), "=r"(vb[19]),
+        "=r"(vb[20]), "=r"(vb[21]), "=r"(vb[22]), "=r"(vb[23]), "=r"(vb[24]), "=r"(vb[25]), "=r"(vb[26]),
+        "=r"(vb[27]), "=r"(vb[28]), "=r"(vb[29]), "=r"(vb[30]), "=r"(vb[31])
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
+
+// AND of `pred` over the `count` threads that reach named barrier `id`.
+__device__ __forceinline__ bool bar_and(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
+// One warp's 32 rows of an fp32 128 x NC tile in TMEM (columns taddr ..
+// taddr + NC) to global memory: through a padded staging buffer, then whole
+// rows, 16 bytes per lane.  Row r of the tile goes to
+// dst + (first_row + r * row_stride) * ld; rows r >= nrows are not written.
+template <int NC>
+__device__ __forceinline__ void bwd_store_rows(float* stage, uint32_t taddr, int quad, int lane, float* dst,
+                                               long long first_row, long long row_stride, int ld, int nrows) {
+  constexpr int kStride = NC + 4;
+  const int row = quad * 32 + lane;
+#pragma unroll
+  for (int q = 0; q < NC / 32; ++q) {
+    uint32_t v[32];
+    tmem_ld32_wait(taddr + 32 * q, v);
+#pragma unroll
+    for (int i = 0; i < 32; i += 4)
+      *reinterpret_cast<float4*>(stage + row * kStride + 32 * q + i) =
+          make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
+                      __uint_as_float(v[i + 3]));
+  }
+  __syncwarp();
+  constexpr int lpr = NC / 4, rpi = 32 / lpr;  // lanes per row, rows per pass
+  const int ci = lane % lpr, rl = lane / lpr;
+#pragma unroll 4
+  for (int r0 = 0; r0 < 32; r0 += rpi) {
+    const int r = quad * 32 + r0 + rl;
+    if (r < nrows)
+      *reinterpret_cast<float4*>(dst + (first_row + r * row_stride) * ld + 4 * ci) =
+          *reinterpret_cast<const float4*>(stage + r * kStride + 4 * ci);
+  }
+  __syncwarp();
+}
+
+// Barrier indices shared by both kernels.
+struct BwdBars {
+  static constexpr int kX = 0;
+  int ns;
+  __device__ int yfull(int s) const { return 1 + s; }
+  __device__ int yempty(int s) const { return 1 + ns + s; }
+  __device__ int sfull() const { return 1 + 2 * ns; }
+  __device__ int pfull() const { return 2 + 2 * ns; }
+  __device__ int odone() const { return 3 + 2 * ns; }
+  __device__ int end() const { return 4 + 2 * ns; }
+};
+
+// ------------------------------------------------------------------- dQ
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                  const __grid_constant__ BwdArgs a) {
+  using SL = BwdSmem<D>;
+  constexpr int NS = SL::kNS;
+  extern __shared__ uint8_t bsm_raw[];
+  uint8_t* smem = bsm_raw + ((1024u - (smem_u32(bsm_raw) & 1023u)) & 1023u);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // tile: heads fastest, then batch, then query segments heaviest first,
+  // then tiles of the segment, latest first
+  int idx = blockIdx.x;
+  const int h = idx % a.Hq;
+  idx /= a.Hq;
+  const int b = idx % a.B;
+  idx /= a.B;
+  const int so = a.seg_order[idx / a.seg_tiles];
+  const int qt = a.seg_tiles - 1 - idx % a.seg_tiles;
+  const int qi = so / a.nseg;
+  const Seg qs = a.seg[qi][so % a.nseg];
+  const int hk = h / a.groups;
+  const int row0 = qt * kBM;
+  const int rows = min(max(qs.len - row0, 0), kBM);
+  const int last = rows > 0 ? qs.pos + row0 + rows - 1 : -1;
+  // the walk: KV blocks in order, their segments, the tiles the last row sees
+  auto nt_of = [&](int s_, int e_) { return (bwd_visible(a, a.seg[a.order[qi][s_]][e_], last) + kBN - 1) / kBN; };
+  int total = 0;
+  for (int s_ = 0; s_ < a.nblk; ++s_)
+    for (int e_ = 0; e_ < a.nseg; ++e_) total += nt_of(s_, e_);
+
+  const BwdBars ib{NS};
+  auto bar = [&](int i) -> uint32_t { return sb + SL::kBar + 8u * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SL::kAbort);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < SL::kNBar; ++i) mbar_init(bar(i), 1);
+    mbar_init(bar(ib.pfull()), kBwdElem / 32);  // one arrival per elementwise warp
+    *abort_flag = grid_timed_out() ? 1 : 0;
+    fence_mbar_init();
+  }
+  if (warp == kBwdMma) tmem_alloc(sb + SL::kTmemSlot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + SL::kTmemSlot);
+  const int work = *abort_flag || rows == 0 ? 0 : total;
+
+  if (warp == kBwdProducer) {
+    if (lane == 0 && work > 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmdO);
+      mbar_expect_tx(bar(ib.kX), 2 * SL::kTile);
+      for (int bx = 0; bx < D / 64; ++bx) {
+        tma_load_4d(sb + SL::kX + bx * SL::kBox, &tmQ, bx * 64, h, qs.mem + row0, b, bar(ib.kX));
+        tma_load_4d(sb + SL::kX + SL::kTile + bx * SL::kBox, &tmdO, bx * 64, h, qs.mem + row0, b, bar(ib.kX));
+      }
+      int j = 0, issued[NS];
+      for (int s = 0; s < NS; ++s) issued[s] = -1;
+      bool ok = true;
+      for (int s_ = 0; s_ < a.nblk && ok; ++s_)
+        for (int e_ = 0; e_ < a.nseg && ok; ++e_) {
+          const Seg ks = a.seg[a.order[qi][s_]][e_];
+          const int nt = nt_of(s_, e_);
+          for (int t = 0; t < nt; ++t, ++j) {
+            const int st = j % NS;
+            if (!mbar_wait(bar(ib.yempty(st)), ((j / NS) & 1) ^ 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            const uint32_t y = sb + SL::kY + st * 2 * SL::kTile;
+            mbar_expect_tx(bar(ib.yfull(st)), 2 * SL::kTile);
+            for (int bx = 0; bx < D / 64; ++bx) {
+              tma_load_4d(y + bx * SL::kBox, &tmK, bx * 64, hk, ks.mem + t * kBN, b, bar(ib.yfull(st)));
+              tma_load_4d(y + SL::kTile + bx * SL::kBox, &tmV, bx * 64, hk, ks.mem + t * kBN, b, bar(ib.yfull(st)));
+            }
+            issued[st] = j;
+          }
+        }
+      // every copy issued lands before the CTA can release its shared memory
+      mbar_drain(bar(ib.kX), 0);
+      for (int s = 0; s < NS; ++s)
+        if (issued[s] >= 0) mbar_drain(bar(ib.yfull(s)), (issued[s] / NS) & 1);
+    }
+  } else if (warp == kBwdMma) {
+    if (lane == 0 && work > 0) {
+      constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t kIdescQ = idesc_bf16_f32(kBM, D, true);
+      // S = Q K^T into [0, 128), dP = dO V^T into [128, 256): K-major A and B
+      auto issue_sdp = [&](int st) {
+        const uint32_t y = sb + SL::kY + st * 2 * SL::kTile;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
+          mma_ss(tmem + kTmS, smem_desc_sw128(sb + SL::kX + off, 16, 1024), smem_desc_sw128(y + off, 16, 1024),
+                 kIdescS, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
+          mma_ss(tmem + kTmP, smem_desc_sw128(sb + SL::kX + SL::kTile + off, 16, 1024),
+                 smem_desc_sw128(y + SL::kTile + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(ib.sfull()));
+      };
+      // dQ += dS K: A = bf16 dS in TMEM, B = the K tile read MN-major
+      auto issue_dq = [&](int st, bool acc) {
+        const uint32_t y = sb + SL::kY + st * 2 * SL::kTile;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_ts(tmem + kTmAcc, tmem + kTmDS + kk * 8, smem_desc_sw128(y + kk * 2048, SL::kBox, 1024), kIdescQ,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(bar(ib.kX), 0, abort_flag) && mbar_wait(bar(ib.yfull(0)), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_sdp(0);
+      }
+      for (int j = 0; ok && j < work; ++j) {
+        const int st = j % NS;
+        if (!mbar_wait_spin(bar(ib.pfull()), j & 1, abort_flag)) break;
+        tc_fence_after();
+        issue_dq(st, j > 0);
+        tc_commit(bar(ib.yempty(st)));
+        if (j + 1 < work) {
+          const int st1 = (j + 1) % NS;
+          if (!mbar_wait(bar(ib.yfull(st1)), ((j + 1) / NS) & 1, abort_flag)) break;
+          tc_fence_after();
+          issue_sdp(st1);
+        }
+      }
+      tc_commit(bar(ib.odone()));
+      tc_commit(bar(ib.end()));
+      mbar_drain(bar(ib.end()), 0);
+    }
+  } else {
+    // ---------------------------------------------------------- elementwise
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;
+    const bool valid = row < rows;
+    const int qpos = valid ? qs.pos + row0 + row : -1;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const long long stat = (static_cast<long long>(b) * a.Hq + h) * a.S + max(qpos, 0);
+    const float lse2 = valid ? a.lse2[stat] : INFINITY;  // padding rows: every P is 0
+    const float dlt = valid ? a.delta[stat] : 0.f;
+    const float ss = a.scale_log2, sc = a.scale;
+    bool ok = work > 0;
+    int j = 0;
+    for (int s_ = 0; s_ < a.nblk && ok; ++s_)
+      for (int e_ = 0; e_ < a.nseg && ok; ++e_) {
+        const Seg ks = a.seg[a.order[qi][s_]][e_];
+        const int nt = nt_of(s_, e_);
+        const int lim = bwd_visible(a, ks, qpos);
+        for (int t = 0; t < nt; ++t, ++j) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(ib.sfull()), j & 1, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+          const int cnt = lim - t * kBN;  // visible keys of this tile for this row
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const int c0 = half * 64 + cc * 32;
+            uint32_t sv[32], pv[32], pk[16];
+            tmem_ld32x2_wait(tmem + lane_base + kTmS + c0, tmem + lane_base + kTmP + c0, sv, pv);
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              float ds[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const float p = c0 + i + e < cnt ? fast_exp2(__uint_as_float(sv[i + e]) * ss - lse2) : 0.f;
+                ds[e] = p * (__uint_as_float(pv[i + e]) - dlt) * sc;
+              }
+              pk[i / 2] = pack_bf16x2(ds[0], ds[1]);
+            }
+            tmem_st16(tmem + lane_base + kTmDS + c0 / 2, pk);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(ib.pfull()));
+        }
+      }
+    // ---- epilogue: this CTA's dQ rows; column half h of every row by warps 4h..4h+3
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(ib.odone()), 0, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      constexpr int NC = D / 2;
+      // every product is complete (odone): the tile buffers are free
+      float* stage = reinterpret_cast<float*>(smem) + half * kBM * (NC + 4);
+      bwd_store_rows<NC>(stage, tmem + lane_base + kTmAcc + half * NC, quad, lane, a.dq + half * NC,
+                         (static_cast<long long>(b) * a.S + qs.pos + row0) * a.Hq + h, a.Hq, D, rows);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kBwdMma) tmem_dealloc(tmem, 512);
+}
+
+// ----------------------------------------------------------------- dK, dV
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                   const __grid_constant__ BwdArgs a) {
+  using SL = BwdSmem<D>;
+  constexpr int NS = SL::kNS;
+  extern __shared__ uint8_t bsm_raw[];
+  uint8_t* smem = bsm_raw + ((1024u - (smem_u32(bsm_raw) & 1023u)) & 1023u);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // tile: KV heads fastest, then batch, then key segments heaviest first,
+  // then tiles of the segment, earliest first
+  int idx = blockIdx.x;
+  const int g = idx % a.Hkv;
+  idx /= a.Hkv;
+  const int b = idx % a.B;
+  idx /= a.B;
+  const int so = a.seg_order[idx / a.seg_tiles];
+  const int kt = idx % a.seg_tiles;
+  const int kj = so / a.nseg;
+  const Seg ks = a.seg[kj][so % a.nseg];
+  const int key0 = kt * kBN;
+  const int krows = min(max(ks.len - key0, 0), kBN);
+  const int first_k = ks.pos + key0;  // earliest key of the tile
+  // query tile t of segment e_ of the s_-th query block this KV block meets:
+  // its first position and rows; false when none of its rows sees this tile
+  auto q_tile = [&](int s_, int e_, int t, int& q0, int& qrows) -> bool {
+    const Seg qsg = a.seg[a.order[kj][s_]][e_];
+    q0 = qsg.pos + t * kBM;
+    qrows = min(qsg.len - t * kBM, kBM);
+    if (qrows <= 0) return false;
+    return !a.causal || q0 + qrows - 1 >= first_k;
+  };
+  auto q_mem = [&](int s_, int e_, int t) { return a.seg[a.order[kj][s_]][e_].mem + t * kBM; };
+  int total = 0;
+  for (int s_ = 0; s_ < a.nblk; ++s_)
+    for (int e_ = 0; e_ < a.nseg; ++e_)
+      for (int t = 0; t < a.seg_tiles; ++t) {
+        int q0, qr;
+        total += q_tile(s_, e_, t, q0, qr) ? 1 : 0;
+      }
+  total *= a.groups;
+
+  const BwdBars ib{NS};
+  auto bar = [&](int i) -> uint32_t { return sb + SL::kBar + 8u * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SL::kAbort);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < SL::kNBar; ++i) mbar_init(bar(i), 1);
+    mbar_init(bar(ib.pfull()), kBwdElem / 32);
+    *abort_flag = grid_timed_out() ? 1 : 0;
+    fence_mbar_init();
+  }
+  if (warp == kBwdMma) tmem_alloc(sb + SL::kTmemSlot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + SL::kTmemSlot);
+  const int work = *abort_flag || krows == 0 ? 0 : total;
+
+  if (warp == kBwdProducer) {
+    if (lane == 0 && work > 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmdO);
+      mbar_expect_tx(bar(ib.kX), 2 * SL::kTile);
+      for (int bx = 0; bx < D / 64; ++bx) {
+        tma_load_4d(sb + SL::kX + bx * SL::kBox, &tmK, bx * 64, g, ks.mem + key0, b, bar(ib.kX));
+        tma_load_4d(sb + SL::kX + SL::kTile + bx * SL::kBox, &tmV, bx * 64, g, ks.mem + key0, b, bar(ib.kX));
+      }
+      int j = 0, issued[NS];
+      for (int s = 0; s < NS; ++s) issued[s] = -1;
+      bool ok = true;
+      for (int hh = 0; hh < a.groups && ok; ++hh)
+        for (int s_ = 0; s_ < a.nblk && ok; ++s_)
+          for (int e_ = 0; e_ < a.nseg && ok; ++e_)
+            for (int t = 0; t < a.seg_tiles; ++t) {
+              int q0, qr;
+              if (!q_tile(s_, e_, t, q0, qr)) continue;
+              const int st = j % NS;
+              if (!mbar_wait(bar(ib.yempty(st)), ((j / NS) & 1) ^ 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              const uint32_t y = sb + SL::kY + st * 2 * SL::kTile;
+              const int hq = g * a.groups + hh, qm = q_mem(s_, e_, t);
+              mbar_expect_tx(bar(ib.yfull(st)), 2 * SL::kTile);
+              for (int bx = 0; bx < D / 64; ++bx) {
+                tma_load_4d(y + bx * SL::kBox, &tmQ, bx * 64, hq, qm, b, bar(ib.yfull(st)));
+                tma_load_4d(y + SL::kTile + bx * SL::kBox, &tmdO, bx * 64, hq, qm, b, bar(ib.yfull(st)));
+              }
+              issued[st] = j;
+              ++j;
+            }
+      mbar_drain(bar(ib.kX), 0);
+      for (int s = 0; s < NS; ++s)
+        if (issued[s] >= 0) mbar_drain(bar(ib.yfull(s)), (issued[s] / NS) & 1);
+    }
+  } else if (warp == kBwdMma) {
+    if (lane == 0 && work > 0) {
+      constexpr uint32_t kIdescS = idesc_bf16_f32(kBN, kBM, false);
+      constexpr uint32_t kIdescO = idesc_bf16_f32(kBN, D, true);
+      // S^T = K Q^T into [0, 128), dP^T = V dO^T into [128, 256)
+      auto issue_sdp = [&](int st) {
+        const uint32_t y = sb + SL::kY + st * 2 * SL::kTile;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
+          mma_ss(tmem + kTmS, smem_desc_sw128(sb + SL::kX + off, 16, 1024), smem_desc_sw128(y + off, 16, 1024),
+                 kIdescS, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
+          mma_ss(tmem + kTmP, smem_desc_sw128(sb + SL::kX + SL::kTile + off, 16, 1024),
+                 smem_desc_sw128(y + SL::kTile + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(ib.sfull()));
+      };
+      // dV += P^T dO and dK += dS^T Q: A = bf16 P^T / dS^T in TMEM, B read MN-major
+      auto issue_dkv = [&](int st, bool acc) {
+        const uint32_t y = sb + SL::kY + st * 2 * SL::kTile;
+#pragma unroll
+        for (int kk = 0; kk < kBM / 16; ++kk)
+          mma_ts(tmem + kTmAcc, tmem + kTmPT + kk * 8, smem_desc_sw128(y + SL::kTile + kk * 2048, SL::kBox, 1024),
+                 kIdescO, (acc || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < kBM / 16; ++kk)
+          mma_ts(tmem + kTmAcc + 128, tmem + kTmDST + kk * 8, smem_desc_sw128(y + kk * 2048, SL::kBox, 1024),
+                 kIdescO, (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(bar(ib.kX), 0, abort_flag) && mbar_wait(bar(ib.yfull(0)), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_sdp(0);
+      }
+      for (int j = 0; ok && j < work; ++j) {
+        const int st = j % NS;
+        if (!mbar_wait_spin(bar(ib.pfull()), j & 1, abort_flag)) break;
+        tc_fence_after();
+        issue_dkv(st, j > 0);
+        tc_commit(bar(ib.yempty(st)));
+        if (j + 1 < work) {
+          const int st1 = (j + 1) % NS;
+          if (!mbar_wait(bar(ib.yfull(st1)), ((j + 1) / NS) & 1, abort_flag)) break;
+          tc_fence_after();
+          issue_sdp(st1);
+        }
+      }
+      tc_commit(bar(ib.odone()));
+      tc_commit(bar(ib.end()));
+      mbar_drain(bar(ib.end()), 0);
+    }
+  } else {
+    // ---------------------------------------------------------- elementwise
+    // Thread (quad, lane) owns key row quad * 32 + lane; half h owns query
+    // columns [64h, 64h + 64).  Half 0 converts its 32-column chunks in the
+    // order 1, 0 and half 1 in the order 2, 3: the bf16 results of a chunk
+    // land only on columns of its own half that it has already read.
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;
+    const int kpos = row < krows ? first_k + row : INT_MAX;  // padding keys: every P is 0
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    float* stat = reinterpret_cast<float*>(smem + SL::kStat);  // [2 sets][lse2 | delta][128]
+    const float ss = a.scale_log2, sc = a.scale;
+    bool ok = work > 0;
+    int j = 0;
+    for (int hh = 0; hh < a.groups && ok; ++hh)
+      for (int s_ = 0; s_ < a.nblk && ok; ++s_)
+        for (int e_ = 0; e_ < a.nseg && ok; ++e_)
+          for (int t = 0; t < a.seg_tiles; ++t) {
+            int q0, qrows;
+            if (!q_tile(s_, e_, t, q0, qrows)) continue;
+            // lse2 (threads 0-127) and delta (threads 128-255) of the tile's
+            // queries, into the set that tile j - 1 does not read
+            float* set = stat + (j & 1) * 2 * kBM;
+            {
+              const int c = threadIdx.x & (kBM - 1);
+              const long long base = (static_cast<long long>(b) * a.Hq + g * a.groups + hh) * a.S + q0;
+              set[threadIdx.x] = threadIdx.x < kBM ? (c < qrows ? a.lse2[base + c] : INFINITY)
+                                                   : (c < qrows ? a.delta[base + c] : 0.f);
+            }
+            const bool w = mbar_wait(bar(ib.sfull()), j & 1, abort_flag);
+            ok = bar_and(1, kBwdElem, w);  // one decision for all 8 warps; also publishes `set`
+            if (!ok) break;
+            tc_fence_after();
+            // query columns below c_lo precede this key (masked when causal)
+            const int c_lo = a.causal ? min(max(kpos - q0, 0), kBM) : (kpos == INT_MAX ? kBM : 0);
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+              const int c0 = half == 0 ? 32 - 32 * cc : 64 + 32 * cc;
+              uint32_t sv[32], pv[32], pp[16], pd[16];
+              tmem_ld32x2_wait(tmem + lane_base + kTmS + c0, tmem + lane_base + kTmP + c0, sv, pv);
+#pragma unroll
+              for (int i = 0; i < 32; i += 4) {
+                const float4 l4 = *reinterpret_cast<const float4*>(set + c0 + i);
+                const float4 d4 = *reinterpret_cast<const float4*>(set + kBM + c0 + i);
+                const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dl[4] = {d4.x, d4.y, d4.z, d4.w};
+                float p[4], ds[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  p[e] = c0 + i + e >= c_lo ? fast_exp2(__uint_as_float(sv[i + e]) * ss - lv[e]) : 0.f;
+                  ds[e] = p[e] * (__uint_as_float(pv[i + e]) - dl[e]) * sc;
+                }
+                pp[i / 2] = pack_bf16x2(p[0], p[1]);
+                pp[i / 2 + 1] = pack_bf16x2(p[2], p[3]);
+                pd[i / 2] = pack_bf16x2(ds[0], ds[1]);
+                pd[i / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+              }
+              tmem_st16(tmem + lane_base + kTmPT + c0 / 2, pp);
+              tmem_st16(tmem + lane_base + kTmDST + c0 / 2, pd);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(ib.pfull()));
+            ++j;
+          }
+    // ---- epilogue: dV rows by warps 0-3, dK rows by warps 4-7
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(ib.odone()), 0, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      float* stage = reinterpret_cast<float*>(smem) + half * kBM * (D + 4);
+      bwd_store_rows<D>(stage, tmem + lane_base + kTmAcc + half * 128, quad, lane, half ? a.dk : a.dv,
+                        (static_cast<long long>(b) * a.S + ks.pos + key0) * a.Hkv + g, a.Hkv, D, krows);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kBwdMma) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace ra

@@ -264,6 +264,49 @@ size_t ra_decode_workspace(int B, int Tq, int Skv, int Hq, int Hkv, int D, int n
 /* Chunks ra_decode_attention uses for these arguments (-1 when invalid). */
 int ra_decode_splits(int B, int Tq, int Skv, int Hq, int Hkv, int D, int n_splits);
 
+/*
+ * ra_ring_attention_backward - gradients of ra_ring_attention.
+ * [RA] SOTA-181: ring attention trains models (the backward pass of exact
+ * attention); [TR] "What carries the argument": the forward's lse is the
+ * log-sum-exp of the whole row, so every (query block, KV block) pair's
+ * share of the gradient is rebuilt from it alone, P = exp(s Q K^T - lse), and
+ * the shares add up:
+ *     dV = sum P^T dO,  dS = P (dO V^T - Delta),  Delta = rowsum(dO * out),
+ *     dQ = s sum dS K,  dK = s sum dS^T Q,        s = 1 / sqrt(D).
+ *  q, k, v       device, in_dtype (RA_BF16, or RA_F32 rounded to bf16 first,
+ *                as in the forward), original token order, [B, S, Hq, D] /
+ *                [B, S, Hkv, D] / [B, S, Hkv, D].
+ *  out           device, out_dtype (RA_F32 or RA_BF16), [B, S, Hq, D]: the
+ *                forward's output for the same arguments.
+ *  lse           device fp32 [B, S, Hq]: the forward's lse (natural log).
+ *  dout          device, in_dtype, [B, S, Hq, D]: gradient of the loss with
+ *                respect to out.
+ *  B .. gqa_groups  as in ra_ring_attention (same limits).
+ *  dq            device fp32 [B, S, Hq, D], written.
+ *  dk, dv        device fp32 [B, S, Hkv, D], written; a KV head's gradient
+ *                sums over the query heads of its group.
+ *  workspace     device scratch of ra_ring_attention_backward_workspace()
+ *                bytes, 256-byte aligned (never NULL: it holds Delta).
+ *  opts          NULL for defaults; `order` sets the order in which the
+ *                block pairs are summed (results agree up to rounding);
+ *                attn_event_begin / attn_event_end bracket the two
+ *                tensor-core kernels (dK/dV, then dQ).  sched and tiling are
+ *                ignored.
+ * Every pointer must be 16-byte aligned (else RA_ERR_INVALID_ARG).  Each
+ * output row is written by exactly one CTA (no atomics): the result does not
+ * depend on scheduling.
+ */
+ra_status ra_ring_attention_backward(const void* q, const void* k, const void* v, ra_dtype in_dtype,
+                                     const void* out, ra_dtype out_dtype, const float* lse, const void* dout,
+                                     int B, int S, int Hq, int D, int n_blocks, int causal, ra_partition partition,
+                                     int gqa_groups, float* dq, float* dk, float* dv, void* workspace,
+                                     size_t workspace_bytes, const ra_options* opts, void* stream);
+
+/* Workspace bytes of ra_ring_attention_backward ((size_t)-1 when the
+ * arguments are invalid). */
+size_t ra_ring_attention_backward_workspace(int B, int S, int Hq, int D, int n_blocks, int gqa_groups,
+                                            ra_partition partition, ra_dtype in_dtype);
+
 /* Reads and clears the device status word (synchronises `stream`).  Returns
  * RA_OK, RA_ERR_TIMEOUT or RA_ERR_DEVICE_BOUNDS, or RA_ERR_CUDA when the read
  * itself fails. */

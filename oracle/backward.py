@@ -27,6 +27,10 @@ heads that read it.
   KV block) pairs of a partition, each pair's probabilities rebuilt from the
   full-row lse: P_ij = exp(s Q_i K_j^T - lse_i).  It shares no code with
   ``attention_backward``.
+* ``backward_query_rows`` / ``backward_key_rows`` - the definition evaluated
+  one row at a time, for sampled rows of workloads too large for the whole
+  matrices: dq of a query row needs only that row's keys; dk, dv of a key need
+  every query row that sees it, each with its own full row.
 """
 from __future__ import annotations
 
@@ -111,3 +115,46 @@ def blockwise_backward(q, k, v, dout, out, lse, n_blocks: int, causal: bool, par
                     dq[b, qi, h] += s * (ds @ kb)
                     dk[b, kj, g] += s * (ds.T @ qb)
     return dq, dk, dv
+
+
+def _row(q_row, keys, vals, do_row, s):
+    """One query row against its visible keys: (p, dp, delta)."""
+    logits = (keys @ q_row) * s
+    e = np.exp(logits - logits.max())
+    p = e / e.sum()
+    o = p @ vals
+    return p, vals @ do_row, float(do_row @ o)
+
+
+def backward_query_rows(q, k, v, dout, rows, causal: bool, gqa_groups: int = 1) -> np.ndarray:
+    """dq at the (b, i, h) triples of ``rows``, one fp64 [D] vector each."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
+    S, D = q.shape[1], q.shape[3]
+    s = 1.0 / math.sqrt(D)
+    out = np.zeros((len(rows), D))
+    for n, (b, i, h) in enumerate(rows):
+        g = h // gqa_groups
+        end = i + 1 if causal else S
+        keys, vals = k[b, :end, g], v[b, :end, g]
+        p, dp, delta = _row(q[b, i, h], keys, vals, do[b, i, h], s)
+        out[n] = s * ((p * (dp - delta)) @ keys)
+    return out
+
+
+def backward_key_rows(q, k, v, dout, keys, causal: bool, gqa_groups: int = 1):
+    """(dk, dv) at the (b, j, g) triples of ``keys``: sums over every query
+    head of group g and every query row that sees key j (i >= j when causal),
+    each row's probabilities normalised over its own visible keys."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
+    S, D = q.shape[1], q.shape[3]
+    s = 1.0 / math.sqrt(D)
+    dk = np.zeros((len(keys), D))
+    dv = np.zeros((len(keys), D))
+    for n, (b, j, g) in enumerate(keys):
+        for h in range(g * gqa_groups, (g + 1) * gqa_groups):
+            for i in range(j if causal else 0, S):
+                end = i + 1 if causal else S
+                p, dp, delta = _row(q[b, i, h], k[b, :end, g], v[b, :end, g], do[b, i, h], s)
+                dv[n] += p[j] * do[b, i, h]
+                dk[n] += s * p[j] * (dp[j] - delta) * q[b, i, h]
+    return dk, dv

@@ -13,6 +13,9 @@ Recipe (one CPU ``torch.Generator`` per call, seeded):
   Tensors above ``CHUNK_ROWS`` tokens are drawn in consecutive token chunks of
   ``CHUNK_ROWS`` from the same generator, so that a 1M-token draw never holds
   more than one fp32 chunk at a time.
+* backward inputs draw Q, K, V as the attention workloads do, then the
+  upstream gradient dO ``[B, S, Hq, D]`` ``randn`` from the same generator,
+  rounded like Q.
 * decode workloads draw ``q`` ``[B, Tq, Hq, D]``, then the cache ``k``, ``v``
   ``[B, Skv, Hkv, D]``, ``randn`` rounded to bf16, in that order.
 * merge workloads draw, for partial i = 0..k-1 in turn, ``out_i`` ~ N(0, 1) of
@@ -131,6 +134,17 @@ def attention_inputs(B: int, S: int, Hq: int, Hkv: int, D: int, dtype: str = "bf
     k = _draw(gen, (B, S, Hkv, D), tdt)
     v = _draw(gen, (B, S, Hkv, D), tdt)
     return q, k, v
+
+
+def backward_inputs(B: int, S: int, Hq: int, Hkv: int, D: int, dtype: str = "bf16", seed: int = 0):
+    """Q, K, V (as ``attention_inputs``) and then dO, from one generator."""
+    tdt = {"bf16": torch.bfloat16, "f32": torch.float32}[dtype]
+    gen = torch.Generator("cpu").manual_seed(seed)
+    q = _draw(gen, (B, S, Hq, D), tdt)
+    k = _draw(gen, (B, S, Hkv, D), tdt)
+    v = _draw(gen, (B, S, Hkv, D), tdt)
+    do = _draw(gen, (B, S, Hq, D), tdt)
+    return q, k, v, do
 
 
 def decode_inputs(B: int, Tq: int, Skv: int, Hq: int, Hkv: int, D: int, seed: int = 0):

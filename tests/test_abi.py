@@ -176,3 +176,36 @@ def test_decode_plan(ra):
     assert ra._lib.ra_decode_splits(1, 1, 10, 8, 3, 128, 0) == -1
     with pytest.raises(ra.RAError):
         ra.ra_decode_workspace(1, 1, 10, 8, 3, 128, 0)
+
+
+def backward(ra, **kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, in_dtype=ra.RA_BF16, out=FAKE, out_dtype=ra.RA_F32, lse=FAKE, dout=FAKE,
+                B=1, S=4096, Hq=8, D=128, n=4, causal=1, part=ra.RA_PART_ZIGZAG, groups=2, dq=FAKE, dk=FAKE,
+                dv=FAKE, ws=FAKE, ws_bytes=1 << 40, opts=None, stream=None)
+    args.update(kw)
+    a = args
+    return ra._lib.ra_ring_attention_backward(a["q"], a["k"], a["v"], a["in_dtype"], a["out"], a["out_dtype"],
+                                              a["lse"], a["dout"], a["B"], a["S"], a["Hq"], a["D"], a["n"],
+                                              a["causal"], a["part"], a["groups"], a["dq"], a["dk"], a["dv"],
+                                              a["ws"], a["ws_bytes"], a["opts"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(S=4100), 1), (dict(groups=3), 1), (dict(D=96), 2), (dict(n=17), 2), (dict(n=0), 1),
+    (dict(dout=None), 1), (dict(dq=None), 1), (dict(dk=FAKE + 4), 1), (dict(lse=FAKE + 8), 1),
+    (dict(in_dtype=7), 1), (dict(out_dtype=5), 1), (dict(part=2), 1), (dict(ws=None), 3), (dict(ws_bytes=64), 3),
+    (dict(ws=FAKE + 16), 1),
+])
+def test_backward_rejects_invalid_arguments(ra, kw, status):
+    assert backward(ra, **kw) == status
+
+
+def test_backward_workspace_query(ra):
+    # Delta and lse * log2(e): two fp32 values per (row, query head)
+    n = ra.ra_ring_attention_backward_workspace(1, 24000, 32, 128, 4, 4, "zigzag")
+    assert n >= 2 * 24000 * 32 * 4
+    # fp32 inputs add bf16 copies of q, k, v and dout
+    n32 = ra.ra_ring_attention_backward_workspace(1, 24000, 32, 128, 4, 4, "zigzag", in_dtype=torch.float32)
+    assert n32 >= n + 24000 * (32 + 8 + 8 + 32) * 128 * 2
+    with pytest.raises(ra.RAError):
+        ra.ra_ring_attention_backward_workspace(1, 4095, 8, 128, 4, 1, "zigzag")

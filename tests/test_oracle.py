@@ -524,3 +524,20 @@ def test_backward_pins_catch_planted_mistakes(kind):
     assert any(np.max(np.abs(a - r)) > 1e-6 for a, r in zip(got, ref))
     good = _backward_mutant("none")(q, k, v, do, True, 1)
     assert all(np.max(np.abs(a - r)) <= 1e-10 for a, r in zip(good, ref))
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_backward_rows_match_autograd(causal):
+    B, S, Hq, Hkv, D = 2, 30, 4, 2, 8
+    q, do = rand64((B, S, Hq, D), 19), rand64((B, S, Hq, D), 20)
+    k, v = rand64((B, S, Hkv, D), 21), rand64((B, S, Hkv, D), 22)
+    dq, dk, dv = autograd_backward(q, k, v, do, causal, 2)
+    rows = [(0, 0, 0), (1, 7, 3), (0, 29, 1), (1, 15, 2)]
+    got = G.backward_query_rows(q, k, v, do, rows, causal, 2)
+    for n, (b, i, h) in enumerate(rows):
+        assert np.max(np.abs(got[n] - dq[b, i, h])) <= 1e-10
+    keys = [(0, 0, 0), (1, 29, 1), (0, 13, 1), (1, 28, 0)]
+    gk, gv = G.backward_key_rows(q, k, v, do, keys, causal, 2)
+    for n, (b, j, g) in enumerate(keys):
+        assert np.max(np.abs(gk[n] - dk[b, j, g])) <= 1e-10
+        assert np.max(np.abs(gv[n] - dv[b, j, g])) <= 1e-10
