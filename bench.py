@@ -60,6 +60,9 @@ def parse():
     p.add_argument("--decode", action="store_true",
                    help="time decode-phase attention over a KV cache (both decode workloads) instead")
     p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--backward", action="store_true",
+                   help="time the backward pass (ra_ring_attention_backward) on --workload instead")
+    p.add_argument("--no-backward", action="store_true")
     a = p.parse_args()
     if a.steps is None:
         a.steps = DEFAULT_STEPS[a.workload]
@@ -336,6 +339,76 @@ def run_decode(args):
 
 # ---------------------------------------------------------------- our arm
 
+# ------------------------------------------------------------ backward pass
+
+def bench_backward(ra, dev, w, reps, flush, order="ring"):
+    """One ra_ring_attention_backward call on workload w (inputs and the
+    forward's out and lse resident in HBM, L2 flushed before each call).
+    The algorithmic work is five products of the forward's size (S = Q K^T,
+    dP = dO V^T, dV = P^T dO, dQ = dS K, dK = dS^T Q): 2.5x the forward's
+    causal-adjusted FLOPs.  Returns (call TFLOP/s, kernels TFLOP/s, call ms,
+    kernels ms): the kernels are the dK/dV and dQ launches alone (events the
+    library records around them), the call adds the Delta / lse pass."""
+    import torch
+    from seeded_inputs import backward_inputs
+    q, k, v, do = (x.to(dev) for x in backward_inputs(w.B, w.S, w.Hq, w.Hkv, w.D, w.in_dtype, seed=10))
+    odt = torch.bfloat16 if w.out_dtype == "bf16" else torch.float32
+    o, l = ra.ra_ring_attention(q, k, v, w.n_blocks, w.causal, w.partition, w.gqa_groups, out_dtype=odt)
+    ws = torch.empty(ra.ra_ring_attention_backward_workspace(w.B, w.S, w.Hq, w.D, w.n_blocks, w.gqa_groups,
+                                                             w.partition, q.dtype), dtype=torch.uint8, device=dev)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=dev)
+    dv = torch.empty(k.shape, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    call, kern = [], []
+    for rep in range(reps + 3):
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        ra.ra_ring_attention_backward(q, k, v, o, l, do, w.n_blocks, w.causal, w.partition, w.gqa_groups, dq=dq,
+                                      dk=dk, dv=dv, workspace=ws, order=order, attn_events=(ev[2], ev[3]))
+        ev[1].record(stream)
+        ev[1].synchronize()
+        if rep >= 3:
+            call.append(ev[0].elapsed_time(ev[1]))
+            kern.append(ev[2].elapsed_time(ev[3]))
+    ms, kms = statistics.median(call), statistics.median(kern)
+    del q, k, v, do, o, l, ws, dq, dk, dv
+    torch.cuda.empty_cache()
+    fl = 2.5 * w.flops
+    return fl / (ms * 1e-3) / 1e12, fl / (kms * 1e-3) / 1e12, ms, kms
+
+
+def run_backward(args):
+    import torch
+    import blockwise_exact_attention_block_b200 as ra
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    w = WORKLOADS[args.workload]
+    pk, pk_kind = peaks()
+    clocks = Clocks(local_gpu_id(dev))
+    time.sleep(0.3)
+    reps = min(max(args.steps, 5), 200)
+    tf, ktf, ms, kms = bench_backward(ra, dev, w, reps, flush, args.order)
+    clk = clocks.stop()
+    status = ra.ra_get_device_status()
+    sustained = kms > 100.0
+    peak = pk["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    line = {"metric": "backward causal-adj TFLOP/s (2.5x forward FLOPs)", "value": tf, "unit": "TFLOP/s",
+            "n_gpus": 1, "steps": reps, "warmup": 3, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded randn, bf16-rounded)",
+            "config": dict(workload_config(w, args, f"flushed ({L2_FLUSH_BYTES >> 20} MiB write between calls)"),
+                           flops_per_step=2.5 * w.flops),
+            "roofline": {"bound": "tensor", "achieved": ktf, "peak": peak, "unit": "TFLOP/s", "frac": ktf / peak,
+                         "traffic": None, "kernel": "bwd_dkv_kernel + bwd_dq_kernel",
+                         "peak_source": f"{pk_kind} {'sustained' if sustained else 'burst'} bf16 dense"},
+            "kernels_ms": kms, "clocks": clk, "gpu_launches": reps * (3 if w.in_dtype == "bf16" else 7),
+            "device_status": ra.ra_status_string(status)}
+    print(json.dumps(line))
+    return 0 if status == 0 else 1
+
+
 def launches_per_step(w, sched):
     """Kernels of ours launched by one ra_ring_attention call."""
     cast = 3 if w.in_dtype == "f32" else 0
@@ -476,6 +549,14 @@ def run_ours(args):
                   "Tq": dw.Tq, "Skv": dw.Skv, "Hq": dw.Hq, "Hkv": dw.Hkv, "D": dw.D, "chunks": splits,
                   "GB/s": gbs, "ms": dms, "peak_GB/s": pk["hbm_gbs"], "frac": gbs / pk["hbm_gbs"]}
 
+    backward = None
+    if not args.no_backward and world == 1:
+        tf, ktf, bms, bkms = bench_backward(ra, dev, w, 20 if w.S <= 32768 else 2, flush, args.order)
+        bpeak = pk["bf16_tflops_sustained" if bkms > 100.0 else "bf16_tflops"]
+        backward = {"kernel": "bwd_dkv_kernel + bwd_dq_kernel (+ bwd_prep_kernel in the call)",
+                    "workload": w.name, "flops_per_step": 2.5 * w.flops, "TFLOP/s": tf, "kernels_TFLOP/s": ktf,
+                    "ms": bms, "kernels_ms": bkms, "peak_TFLOP/s": bpeak, "frac": ktf / bpeak}
+
     value = replica_throughput(w.flops, world, K, total_ms)
     line = {"metric": "causal-adj attention TFLOP/s (% of dense bf16 peak)", "value": value, "unit": "TFLOP/s",
             "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
@@ -485,7 +566,7 @@ def run_ours(args):
                                                f"L2 {l2_bytes >> 20} MiB)"),
             "pct_of_peak": 100.0 * value / peak, "attn_kernel_ms": attn_mean, "roofline": roof,
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "gpu_launches": K * launches_per_step(w, args.sched),
-            "merge": merge, "decode": decode,
+            "merge": merge, "decode": decode, "backward": backward,
             "device_status": ra.ra_status_string(status)}
     if rank == 0:
         print(json.dumps(line))
@@ -534,6 +615,8 @@ def main():
         return run_merge_sweep(args)
     if args.decode:
         return run_decode(args)
+    if args.backward:
+        return run_backward(args)
     return run_ours(args)
 
 

@@ -66,10 +66,11 @@ struct BwdSmem {
   static constexpr int kNS = D == 128 ? 2 : 4;        // stages of the streamed pair
   static constexpr int kX = 0;                        // stationary pair: (Q, dO) or (K, V)
   static constexpr int kY = 2 * kTile;                // ring of streamed pairs
-  static constexpr int kStat = kY + kNS * 2 * kTile;  // dK/dV kernel: [2 sets][lse2 | delta][128]
+  // dK/dV kernel: per-query statistics, [2 sets][2 halves][-lse2 x 64 | -delta x 64]
+  static constexpr int kStat = kY + kNS * 2 * kTile;
   static constexpr int kBar = kStat + 2 * 2 * kBM * 4;
-  // barriers: X, Yfull[NS], Yempty[NS], Sfull, Pfull, Odone, End
-  static constexpr int kNBar = 1 + 2 * kNS + 4;
+  // barriers: X, Yfull[NS], Yempty[NS], Sfull[2], Pfull[2], Odone, End
+  static constexpr int kNBar = 1 + 2 * kNS + 6;
   static constexpr int kTmemSlot = kBar + kNBar * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4 + 1024;  // + slack to align the base to 1024
@@ -78,14 +79,15 @@ struct BwdSmem {
   static_assert(2 * kBM * (D + 4) * 4 <= kStat, "output staging fits in the tile buffers");
 };
 
-// TMEM columns: both kernels keep the two score-shaped products at [0, 128)
-// and [128, 256) and their fp32 accumulators from 256.
-constexpr int kTmS = 0, kTmP = 128, kTmAcc = 256;
-constexpr int kTmDS = 384;  // dQ kernel: bf16 dS (64 columns), clear of S, dP and dQ
-// dK/dV kernel: bf16 P^T written at [32, 96) over S^T, bf16 dS^T at [160, 224)
-// over dP^T.  Column half h of a row writes only columns that half h has
-// already read (see bwd_dkv_kernel), so the two halves never race.
-constexpr int kTmPT = 32, kTmDST = 160;
+// Tensor memory (512 columns).  Each 128-wide score tile is handled as two
+// 64-column halves h = 0, 1 with their own MMAs and barriers, so the
+// elementwise pass over one half overlaps the tensor-core work of the other:
+//   half h: scores S_h at [128h, 128h + 64), dP_h at [128h + 64, 128h + 128)
+//   fp32 accumulators from 256 (dQ; or dV, then dK)
+// The bf16 results of half h (dS, or P^T and dS^T) are written over the
+// first 32 columns of its own S_h / dP_h: chunk c (32 columns) lands on
+// columns of chunk 0 that the same thread has already read.
+constexpr int kTmAcc = 256;
 
 // Delta = rowsum(dO * O) and lse * log2(e), written as [B][Hq][S].  D / 4
 // threads per row, 4 elements each.
@@ -175,12 +177,13 @@ __device__ __forceinline__ bool bar_and(int id, int count, bool pred) {
 }
 
 // One warp's 32 rows of an fp32 128 x NC tile in TMEM (columns taddr ..
-// taddr + NC) to global memory: through a padded staging buffer, then whole
-// rows, 16 bytes per lane.  Row r of the tile goes to
+// taddr + NC), times `mul`, to global memory: through a padded staging
+// buffer, then whole rows, 16 bytes per lane.  Row r of the tile goes to
 // dst + (first_row + r * row_stride) * ld; rows r >= nrows are not written.
 template <int NC>
 __device__ __forceinline__ void bwd_store_rows(float* stage, uint32_t taddr, int quad, int lane, float* dst,
-                                               long long first_row, long long row_stride, int ld, int nrows) {
+                                               long long first_row, long long row_stride, int ld, int nrows,
+                                               float mul) {
   constexpr int kStride = NC + 4;
   const int row = quad * 32 + lane;
 #pragma unroll
@@ -190,8 +193,8 @@ __device__ __forceinline__ void bwd_store_rows(float* stage, uint32_t taddr, int
 #pragma unroll
     for (int i = 0; i < 32; i += 4)
       *reinterpret_cast<float4*>(stage + row * kStride + 32 * q + i) =
-          make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
-                      __uint_as_float(v[i + 3]));
+          make_float4(__uint_as_float(v[i]) * mul, __uint_as_float(v[i + 1]) * mul, __uint_as_float(v[i + 2]) * mul,
+                      __uint_as_float(v[i + 3]) * mul);
   }
   __syncwarp();
   constexpr int lpr = NC / 4, rpi = 32 / lpr;  // lanes per row, rows per pass
@@ -206,19 +209,69 @@ __device__ __forceinline__ void bwd_store_rows(float* stage, uint32_t taddr, int
   __syncwarp();
 }
 
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// One 32-column chunk of a row: from fp32 scores s and dP (raw TMEM bits) to
+// bf16 pairs of P = 2^(s * ss - lse2) and dS = P (dP - Delta), two columns per
+// packed fp32x2 operation.  nl / nd: -lse2 and -Delta per column (COLS) or
+// the row's own (nl[0], nd[0]).  MASK: columns c < lo or c >= hi get P = 0.
+template <bool COLS, bool MASK, bool WANT_P>
+__device__ __forceinline__ void bwd_convert(const uint32_t (&sv)[32], const uint32_t (&pv)[32], float ss,
+                                            const float* nl, const float* nd, int lo, int hi, uint32_t (&pp)[16],
+                                            uint32_t (&pd)[16]) {
+  const uint64_t ss2 = f2_pack(ss, ss);
+  const uint64_t nl_row = f2_pack(nl[0], nl[0]), nd_row = f2_pack(nd[0], nd[0]);
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) {
+    float4 l4, d4;
+    if constexpr (COLS) {
+      l4 = *reinterpret_cast<const float4*>(nl + i);
+      d4 = *reinterpret_cast<const float4*>(nd + i);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; e += 2) {
+      const uint64_t nlv = COLS ? f2_pack(e ? l4.z : l4.x, e ? l4.w : l4.y) : nl_row;
+      const uint64_t ndv = COLS ? f2_pack(e ? d4.z : d4.x, e ? d4.w : d4.y) : nd_row;
+      float x0, x1;
+      f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[i + e]), __uint_as_float(sv[i + e + 1])), ss2, nlv), x0, x1);
+      float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+      if constexpr (MASK) {
+        const int c = i + e;
+        p0 = c >= lo && c < hi ? p0 : 0.f;
+        p1 = c + 1 >= lo && c + 1 < hi ? p1 : 0.f;
+      }
+      const uint64_t t = f2_add(f2_pack(__uint_as_float(pv[i + e]), __uint_as_float(pv[i + e + 1])), ndv);
+      float d0, d1;
+      f2_unpack(f2_mul(f2_pack(p0, p1), t), d0, d1);
+      if constexpr (WANT_P) pp[(i + e) / 2] = pack_bf16x2(p0, p1);
+      pd[(i + e) / 2] = pack_bf16x2(d0, d1);
+    }
+  }
+}
+
 // Barrier indices shared by both kernels.
 struct BwdBars {
   static constexpr int kX = 0;
   int ns;
   __device__ int yfull(int s) const { return 1 + s; }
   __device__ int yempty(int s) const { return 1 + ns + s; }
-  __device__ int sfull() const { return 1 + 2 * ns; }
-  __device__ int pfull() const { return 2 + 2 * ns; }
-  __device__ int odone() const { return 3 + 2 * ns; }
-  __device__ int end() const { return 4 + 2 * ns; }
+  __device__ int sfull(int h) const { return 1 + 2 * ns + h; }
+  __device__ int pfull(int h) const { return 3 + 2 * ns + h; }
+  __device__ int odone() const { return 5 + 2 * ns; }
+  __device__ int end() const { return 6 + 2 * ns; }
 };
 
 // ------------------------------------------------------------------- dQ
+// MMA issue order over the CTA's KV tiles j (half h = keys 64h .. 64h + 63):
+//   S_0(0) dP_0(0), S_1(0) dP_1(0), then for every j:
+//   [P_0 ready] dQ += dS_0 K_0, S_0(j+1) dP_0(j+1),
+//   [P_1 ready] dQ += dS_1 K_1, release tile j, S_1(j+1) dP_1(j+1)
+// so the tensor core computes one half while the elementwise warps of the
+// other half run (warps 0-3 own half 0, warps 4-7 half 1).
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -257,7 +310,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SL::kAbort);
   if (threadIdx.x == 0) {
     for (int i = 0; i < SL::kNBar; ++i) mbar_init(bar(i), 1);
-    mbar_init(bar(ib.pfull()), kBwdElem / 32);  // one arrival per elementwise warp
+    mbar_init(bar(ib.pfull(0)), kBwdElem / 64);  // one arrival per warp of the half
+    mbar_init(bar(ib.pfull(1)), kBwdElem / 64);
     *abort_flag = grid_timed_out() ? 1 : 0;
     fence_mbar_init();
   }
@@ -308,49 +362,56 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp == kBwdMma) {
     if (lane == 0 && work > 0) {
-      constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, 64, false);
       constexpr uint32_t kIdescQ = idesc_bf16_f32(kBM, D, true);
-      // S = Q K^T into [0, 128), dP = dO V^T into [128, 256): K-major A and B
-      auto issue_sdp = [&](int st) {
-        const uint32_t y = sb + SL::kY + st * 2 * SL::kTile;
+      // S_h = Q K_h^T and dP_h = dO V_h^T (K_h, V_h: rows 64h.. of the tile), K-major operands
+      auto issue_sdp = [&](int st, int hf) {
+        const uint32_t y = sb + SL::kY + st * 2 * SL::kTile + hf * 64 * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
-          mma_ss(tmem + kTmS, smem_desc_sw128(sb + SL::kX + off, 16, 1024), smem_desc_sw128(y + off, 16, 1024),
+          mma_ss(tmem + 128 * hf, smem_desc_sw128(sb + SL::kX + off, 16, 1024), smem_desc_sw128(y + off, 16, 1024),
                  kIdescS, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
-          mma_ss(tmem + kTmP, smem_desc_sw128(sb + SL::kX + SL::kTile + off, 16, 1024),
+          mma_ss(tmem + 128 * hf + 64, smem_desc_sw128(sb + SL::kX + SL::kTile + off, 16, 1024),
                  smem_desc_sw128(y + SL::kTile + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(ib.sfull()));
+        tc_commit(bar(ib.sfull(hf)));
       };
-      // dQ += dS K: A = bf16 dS in TMEM, B = the K tile read MN-major
-      auto issue_dq = [&](int st, bool acc) {
+      // dQ += dS_h K_h: A = bf16 dS_h in TMEM, B = rows 64h.. of the K tile read MN-major
+      auto issue_dq = [&](int st, int hf, bool acc) {
         const uint32_t y = sb + SL::kY + st * 2 * SL::kTile;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(tmem + kTmAcc, tmem + kTmDS + kk * 8, smem_desc_sw128(y + kk * 2048, SL::kBox, 1024), kIdescQ,
-                 (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + kTmAcc, tmem + 128 * hf + kk * 8, smem_desc_sw128(y + (hf * 4 + kk) * 2048, SL::kBox, 1024),
+                 kIdescQ, (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(bar(ib.kX), 0, abort_flag) && mbar_wait(bar(ib.yfull(0)), 0, abort_flag);
       if (ok) {
         tc_fence_after();
-        issue_sdp(0);
+        issue_sdp(0, 0);
+        issue_sdp(0, 1);
       }
       for (int j = 0; ok && j < work; ++j) {
-        const int st = j % NS;
-        if (!mbar_wait_spin(bar(ib.pfull()), j & 1, abort_flag)) break;
-        tc_fence_after();
-        issue_dq(st, j > 0);
-        tc_commit(bar(ib.yempty(st)));
-        if (j + 1 < work) {
-          const int st1 = (j + 1) % NS;
-          if (!mbar_wait(bar(ib.yfull(st1)), ((j + 1) / NS) & 1, abort_flag)) break;
+        const int st = j % NS, st1 = (j + 1) % NS;
+        const bool more = j + 1 < work;
+        for (int hf = 0; hf < 2 && ok; ++hf) {
+          ok = mbar_wait(bar(ib.pfull(hf)), j & 1, abort_flag);
+          if (!ok) break;
           tc_fence_after();
-          issue_sdp(st1);
+          issue_dq(st, hf, j > 0 || hf > 0);
+          if (hf == 1) tc_commit(bar(ib.yempty(st)));
+          if (more) {
+            if (hf == 0) {
+              ok = mbar_wait(bar(ib.yfull(st1)), ((j + 1) / NS) & 1, abort_flag);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            issue_sdp(st1, hf);
+          }
         }
       }
       tc_commit(bar(ib.odone()));
@@ -364,10 +425,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool valid = row < rows;
     const int qpos = valid ? qs.pos + row0 + row : -1;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_base + 128 * half, tP = tS + 64;
     const long long stat = (static_cast<long long>(b) * a.Hq + h) * a.S + max(qpos, 0);
-    const float lse2 = valid ? a.lse2[stat] : INFINITY;  // padding rows: every P is 0
-    const float dlt = valid ? a.delta[stat] : 0.f;
-    const float ss = a.scale_log2, sc = a.scale;
+    // padding rows: -lse2 = -inf, so every P is 0
+    const float nl = valid ? -a.lse2[stat] : -INFINITY;
+    const float nd = valid ? -a.delta[stat] : 0.f;
+    const float ss = a.scale_log2;
     bool ok = work > 0;
     int j = 0;
     for (int s_ = 0; s_ < a.nblk && ok; ++s_)
@@ -376,31 +439,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int nt = nt_of(s_, e_);
         const int lim = bwd_visible(a, ks, qpos);
         for (int t = 0; t < nt; ++t, ++j) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(ib.sfull()), j & 1, abort_flag));
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(ib.sfull(half)), j & 1, abort_flag));
           if (!ok) break;
           tc_fence_after();
-          const int cnt = lim - t * kBN;  // visible keys of this tile for this row
+          // keys of this half visible to the row: [0, cnt)
+          const int cnt = lim - t * kBN - 64 * half;
+          const bool full = __all_sync(0xffffffffu, !valid || cnt >= 64);
 #pragma unroll
           for (int cc = 0; cc < 2; ++cc) {
-            const int c0 = half * 64 + cc * 32;
             uint32_t sv[32], pv[32], pk[16];
-            tmem_ld32x2_wait(tmem + lane_base + kTmS + c0, tmem + lane_base + kTmP + c0, sv, pv);
-#pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              float ds[2];
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const float p = c0 + i + e < cnt ? fast_exp2(__uint_as_float(sv[i + e]) * ss - lse2) : 0.f;
-                ds[e] = p * (__uint_as_float(pv[i + e]) - dlt) * sc;
-              }
-              pk[i / 2] = pack_bf16x2(ds[0], ds[1]);
-            }
-            tmem_st16(tmem + lane_base + kTmDS + c0 / 2, pk);
+            tmem_ld32x2_wait(tS + 32 * cc, tP + 32 * cc, sv, pv);
+            if (full)
+              bwd_convert<false, false, false>(sv, pv, ss, &nl, &nd, 0, 0, pk, pk);
+            else
+              bwd_convert<false, true, false>(sv, pv, ss, &nl, &nd, 0, cnt - 32 * cc, pk, pk);
+            tmem_st16(tS + 16 * cc, pk);  // over columns this thread has read
           }
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(ib.pfull()));
+          if (lane == 0) mbar_arrive(bar(ib.pfull(half)));
         }
       }
     // ---- epilogue: this CTA's dQ rows; column half h of every row by warps 4h..4h+3
@@ -411,7 +469,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // every product is complete (odone): the tile buffers are free
       float* stage = reinterpret_cast<float*>(smem) + half * kBM * (NC + 4);
       bwd_store_rows<NC>(stage, tmem + lane_base + kTmAcc + half * NC, quad, lane, a.dq + half * NC,
-                         (static_cast<long long>(b) * a.S + qs.pos + row0) * a.Hq + h, a.Hq, D, rows);
+                         (static_cast<long long>(b) * a.S + qs.pos + row0) * a.Hq + h, a.Hq, D, rows, a.scale);
     }
   }
   tc_fence_before();
@@ -421,6 +479,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // ----------------------------------------------------------------- dK, dV
+// Same pipeline over the CTA's query tiles j (half h = queries 64h .. 64h + 63):
+//   S^T_h = K Q_h^T, dP^T_h = V dO_h^T; then dV += P^T_h dO_h, dK += dS^T_h Q_h.
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -471,7 +531,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SL::kAbort);
   if (threadIdx.x == 0) {
     for (int i = 0; i < SL::kNBar; ++i) mbar_init(bar(i), 1);
-    mbar_init(bar(ib.pfull()), kBwdElem / 32);
+    mbar_init(bar(ib.pfull(0)), kBwdElem / 64);
+    mbar_init(bar(ib.pfull(1)), kBwdElem / 64);
     *abort_flag = grid_timed_out() ? 1 : 0;
     fence_mbar_init();
   }
@@ -523,53 +584,61 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp == kBwdMma) {
     if (lane == 0 && work > 0) {
-      constexpr uint32_t kIdescS = idesc_bf16_f32(kBN, kBM, false);
+      constexpr uint32_t kIdescS = idesc_bf16_f32(kBN, 64, false);
       constexpr uint32_t kIdescO = idesc_bf16_f32(kBN, D, true);
-      // S^T = K Q^T into [0, 128), dP^T = V dO^T into [128, 256)
-      auto issue_sdp = [&](int st) {
-        const uint32_t y = sb + SL::kY + st * 2 * SL::kTile;
+      // S^T_h = K Q_h^T and dP^T_h = V dO_h^T (Q_h, dO_h: rows 64h.. of the tile)
+      auto issue_sdp = [&](int st, int hf) {
+        const uint32_t y = sb + SL::kY + st * 2 * SL::kTile + hf * 64 * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
-          mma_ss(tmem + kTmS, smem_desc_sw128(sb + SL::kX + off, 16, 1024), smem_desc_sw128(y + off, 16, 1024),
+          mma_ss(tmem + 128 * hf, smem_desc_sw128(sb + SL::kX + off, 16, 1024), smem_desc_sw128(y + off, 16, 1024),
                  kIdescS, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
-          mma_ss(tmem + kTmP, smem_desc_sw128(sb + SL::kX + SL::kTile + off, 16, 1024),
+          mma_ss(tmem + 128 * hf + 64, smem_desc_sw128(sb + SL::kX + SL::kTile + off, 16, 1024),
                  smem_desc_sw128(y + SL::kTile + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(ib.sfull()));
+        tc_commit(bar(ib.sfull(hf)));
       };
-      // dV += P^T dO and dK += dS^T Q: A = bf16 P^T / dS^T in TMEM, B read MN-major
-      auto issue_dkv = [&](int st, bool acc) {
+      // dV += P^T_h dO_h and dK += dS^T_h Q_h: A = bf16 in TMEM, B read MN-major
+      auto issue_dkv = [&](int st, int hf, bool acc) {
         const uint32_t y = sb + SL::kY + st * 2 * SL::kTile;
 #pragma unroll
-        for (int kk = 0; kk < kBM / 16; ++kk)
-          mma_ts(tmem + kTmAcc, tmem + kTmPT + kk * 8, smem_desc_sw128(y + SL::kTile + kk * 2048, SL::kBox, 1024),
-                 kIdescO, (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + kTmAcc, tmem + 128 * hf + kk * 8,
+                 smem_desc_sw128(y + SL::kTile + (hf * 4 + kk) * 2048, SL::kBox, 1024), kIdescO,
+                 (acc || kk > 0) ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < kBM / 16; ++kk)
-          mma_ts(tmem + kTmAcc + 128, tmem + kTmDST + kk * 8, smem_desc_sw128(y + kk * 2048, SL::kBox, 1024),
-                 kIdescO, (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + kTmAcc + 128, tmem + 128 * hf + 64 + kk * 8,
+                 smem_desc_sw128(y + (hf * 4 + kk) * 2048, SL::kBox, 1024), kIdescO, (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(bar(ib.kX), 0, abort_flag) && mbar_wait(bar(ib.yfull(0)), 0, abort_flag);
       if (ok) {
         tc_fence_after();
-        issue_sdp(0);
+        issue_sdp(0, 0);
+        issue_sdp(0, 1);
       }
       for (int j = 0; ok && j < work; ++j) {
-        const int st = j % NS;
-        if (!mbar_wait_spin(bar(ib.pfull()), j & 1, abort_flag)) break;
-        tc_fence_after();
-        issue_dkv(st, j > 0);
-        tc_commit(bar(ib.yempty(st)));
-        if (j + 1 < work) {
-          const int st1 = (j + 1) % NS;
-          if (!mbar_wait(bar(ib.yfull(st1)), ((j + 1) / NS) & 1, abort_flag)) break;
+        const int st = j % NS, st1 = (j + 1) % NS;
+        const bool more = j + 1 < work;
+        for (int hf = 0; hf < 2 && ok; ++hf) {
+          ok = mbar_wait(bar(ib.pfull(hf)), j & 1, abort_flag);
+          if (!ok) break;
           tc_fence_after();
-          issue_sdp(st1);
+          issue_dkv(st, hf, j > 0 || hf > 0);
+          if (hf == 1) tc_commit(bar(ib.yempty(st)));
+          if (more) {
+            if (hf == 0) {
+              ok = mbar_wait(bar(ib.yfull(st1)), ((j + 1) / NS) & 1, abort_flag);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            issue_sdp(st1, hf);
+          }
         }
       }
       tc_commit(bar(ib.odone()));
@@ -578,16 +647,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- elementwise
-    // Thread (quad, lane) owns key row quad * 32 + lane; half h owns query
-    // columns [64h, 64h + 64).  Half 0 converts its 32-column chunks in the
-    // order 1, 0 and half 1 in the order 2, 3: the bf16 results of a chunk
-    // land only on columns of its own half that it has already read.
+    // Thread (quad, lane) owns key row quad * 32 + lane; warps 4h..4h+3 own
+    // query half h of every tile.
     const int quad = warp & 3, half = warp >> 2;
     const int row = quad * 32 + lane;
-    const int kpos = row < krows ? first_k + row : INT_MAX;  // padding keys: every P is 0
+    const int kpos = row < krows ? first_k + row : -1;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    float* stat = reinterpret_cast<float*>(smem + SL::kStat);  // [2 sets][lse2 | delta][128]
-    const float ss = a.scale_log2, sc = a.scale;
+    const uint32_t tS = tmem + lane_base + 128 * half, tP = tS + 64;
+    float* stat = reinterpret_cast<float*>(smem + SL::kStat);
+    const float ss = a.scale_log2;
     bool ok = work > 0;
     int j = 0;
     for (int hh = 0; hh < a.groups && ok; ++hh)
@@ -596,49 +664,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           for (int t = 0; t < a.seg_tiles; ++t) {
             int q0, qrows;
             if (!q_tile(s_, e_, t, q0, qrows)) continue;
-            // lse2 (threads 0-127) and delta (threads 128-255) of the tile's
-            // queries, into the set that tile j - 1 does not read
-            float* set = stat + (j & 1) * 2 * kBM;
+            // -lse2 (rows 0-63 of the half's warps) and -delta (rows 64-127) of
+            // the half's 64 queries, into the set that tile j - 1 does not read
+            float* set = stat + ((j & 1) * 2 + half) * kBM;
             {
-              const int c = threadIdx.x & (kBM - 1);
-              const long long base = (static_cast<long long>(b) * a.Hq + g * a.groups + hh) * a.S + q0;
-              set[threadIdx.x] = threadIdx.x < kBM ? (c < qrows ? a.lse2[base + c] : INFINITY)
-                                                   : (c < qrows ? a.delta[base + c] : 0.f);
+              const int c = 64 * half + (row & 63);
+              const long long at = (static_cast<long long>(b) * a.Hq + g * a.groups + hh) * a.S + q0 + c;
+              set[row] = row < 64 ? (c < qrows ? -a.lse2[at] : -INFINITY) : (c < qrows ? -a.delta[at] : 0.f);
             }
-            const bool w = mbar_wait(bar(ib.sfull()), j & 1, abort_flag);
-            ok = bar_and(1, kBwdElem, w);  // one decision for all 8 warps; also publishes `set`
+            const bool w = mbar_wait(bar(ib.sfull(half)), j & 1, abort_flag);
+            ok = bar_and(1 + half, kBM, w);  // one decision for the half's 4 warps; publishes `set`
             if (!ok) break;
             tc_fence_after();
-            // query columns below c_lo precede this key (masked when causal)
-            const int c_lo = a.causal ? min(max(kpos - q0, 0), kBM) : (kpos == INT_MAX ? kBM : 0);
+            // when causal, this key sees the half's query columns [lo, 64)
+            const int lo = a.causal && kpos >= 0 ? kpos - q0 - 64 * half : -64;
+            const bool full = __all_sync(0xffffffffu, lo <= 0);
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
-              const int c0 = half == 0 ? 32 - 32 * cc : 64 + 32 * cc;
               uint32_t sv[32], pv[32], pp[16], pd[16];
-              tmem_ld32x2_wait(tmem + lane_base + kTmS + c0, tmem + lane_base + kTmP + c0, sv, pv);
-#pragma unroll
-              for (int i = 0; i < 32; i += 4) {
-                const float4 l4 = *reinterpret_cast<const float4*>(set + c0 + i);
-                const float4 d4 = *reinterpret_cast<const float4*>(set + kBM + c0 + i);
-                const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dl[4] = {d4.x, d4.y, d4.z, d4.w};
-                float p[4], ds[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  p[e] = c0 + i + e >= c_lo ? fast_exp2(__uint_as_float(sv[i + e]) * ss - lv[e]) : 0.f;
-                  ds[e] = p[e] * (__uint_as_float(pv[i + e]) - dl[e]) * sc;
-                }
-                pp[i / 2] = pack_bf16x2(p[0], p[1]);
-                pp[i / 2 + 1] = pack_bf16x2(p[2], p[3]);
-                pd[i / 2] = pack_bf16x2(ds[0], ds[1]);
-                pd[i / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
-              }
-              tmem_st16(tmem + lane_base + kTmPT + c0 / 2, pp);
-              tmem_st16(tmem + lane_base + kTmDST + c0 / 2, pd);
+              tmem_ld32x2_wait(tS + 32 * cc, tP + 32 * cc, sv, pv);
+              if (full)
+                bwd_convert<true, false, true>(sv, pv, ss, set + 32 * cc, set + 64 + 32 * cc, 0, 0, pp, pd);
+              else
+                bwd_convert<true, true, true>(sv, pv, ss, set + 32 * cc, set + 64 + 32 * cc, lo - 32 * cc, 64, pp,
+                                              pd);
+              tmem_st16(tS + 16 * cc, pp);  // P^T over columns this thread has read
+              tmem_st16(tP + 16 * cc, pd);  // dS^T likewise
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(ib.pfull()));
+            if (lane == 0) mbar_arrive(bar(ib.pfull(half)));
             ++j;
           }
     // ---- epilogue: dV rows by warps 0-3, dK rows by warps 4-7
@@ -647,7 +703,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       float* stage = reinterpret_cast<float*>(smem) + half * kBM * (D + 4);
       bwd_store_rows<D>(stage, tmem + lane_base + kTmAcc + half * 128, quad, lane, half ? a.dk : a.dv,
-                        (static_cast<long long>(b) * a.S + ks.pos + key0) * a.Hkv + g, a.Hkv, D, krows);
+                        (static_cast<long long>(b) * a.S + ks.pos + key0) * a.Hkv + g, a.Hkv, D, krows,
+                        half ? a.scale : 1.f);
     }
   }
   tc_fence_before();
