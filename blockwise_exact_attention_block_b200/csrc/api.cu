@@ -467,14 +467,14 @@ void bwd_segment_order(BwdArgs& a, bool latest_first) {
 template <int D>
 ra_status launch_bwd_d(const BwdArgs& adq, const BwdArgs& adkv, const CUtensorMap& mq, const CUtensorMap& mk,
                        const CUtensorMap& mv, const CUtensorMap& mdo, cudaStream_t st) {
-  using SL = BwdSmem<D>;
+  constexpr int kQBytes = BwdQSmem<D>::kBytes, kKVBytes = BwdKVSmem<D>::kBytes;
   static int attr_set[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, SL::kBytes) !=
+    if (cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kQBytes) !=
             cudaSuccess ||
-        cudaFuncSetAttribute(bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, SL::kBytes) !=
+        cudaFuncSetAttribute(bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kKVBytes) !=
             cudaSuccess)
       return RA_ERR_CUDA;
     attr_set[dev] = 1;
@@ -482,10 +482,10 @@ ra_status launch_bwd_d(const BwdArgs& adq, const BwdArgs& adkv, const CUtensorMa
   const long long tiles = static_cast<long long>(adq.B) * adq.nblk * adq.nseg * adq.seg_tiles;
   const long long gkv = tiles * adkv.Hkv, gq = tiles * adq.Hq;
   if (gq > 0x7fffffffLL) return RA_ERR_UNSUPPORTED;
-  bwd_dkv_kernel<D><<<static_cast<unsigned>(gkv), kBwdThreads, SL::kBytes, st>>>(mq, mk, mv, mdo, adkv);
+  bwd_dkv_kernel<D><<<static_cast<unsigned>(gkv), kBwdThreads, kKVBytes, st>>>(mq, mk, mv, mdo, adkv);
   ra_status s = cuda_status(cudaGetLastError());
   if (s != RA_OK) return s;
-  bwd_dq_kernel<D><<<static_cast<unsigned>(gq), kBwdThreads, SL::kBytes, st>>>(mq, mk, mv, mdo, adq);
+  bwd_dq_kernel<D><<<static_cast<unsigned>(gq), kBwdThreads, kQBytes, st>>>(mq, mk, mv, mdo, adq);
   return cuda_status(cudaGetLastError());
 }
 

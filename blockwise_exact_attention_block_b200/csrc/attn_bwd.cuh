@@ -23,13 +23,20 @@
 //
 // Warp roles (320 threads):
 //   warps 0-7  elementwise: thread (warp % 4) * 32 + lane owns TMEM lane /
-//              tile row (warp % 4) * 32 + lane; warps 0-3 take columns
-//              [0, 64) of the 128 x 128 score tile, warps 4-7 columns [64, 128)
+//              tile row (warp % 4) * 32 + lane; warps 4w..4w+3 take columns
+//              64h + 32w .. 64h + 32w + 31 of column half h = 0, 1 of the
+//              128 x 128 score tile
 //   warp 8     TMA producer
 //   warp 9     TMEM allocator and MMA issuer (one thread)
-// Both kernels use only the forward kernel's operand forms: SS products of
-// K-major SW128 tiles, and TS products with a bf16 A operand in tensor memory
-// and an MN-major B tile.
+// Each tile's elementwise pass first loads its scores into registers and
+// signals "read"; the tensor core then starts the next tile's score-shaped
+// products (both of them in the dQ kernel, dP^T in the dK/dV kernel) while
+// the pass converts P and dS to bf16.  The pass converts column half 0 of the
+// tile (all 8 warps, 32 columns each), signals it, then half 1, so the
+// products that consume half 0 run while half 1 is converted.  All
+// products are 128 wide: SS products of K-major SW128 tiles, and TS products
+// with a bf16 A operand in tensor memory and an MN-major B tile, the operand
+// forms of the forward kernel.
 #pragma once
 
 #include "attn_fwd.cuh"
@@ -59,35 +66,60 @@ struct BwdArgs {
   signed char seg_order[2 * kMaxBlocks];      // (r * nseg + e) of the CTA segments, heaviest first
 };
 
+// Shared memory of the dQ kernel: Q and dO stay; K and V stream through
+// rings.  V(j) is free once dP(j) completes, K(j) only after dQ(j), so the K
+// ring is deeper.
 template <int D>
-struct BwdSmem {
+struct BwdQSmem {
   static constexpr int kBox = kBM * 128;  // 128 rows x 64 bf16: one TMA box, 16 KB
   static constexpr int kTile = kBox * (D / 64);
-  static constexpr int kNS = D == 128 ? 2 : 4;        // stages of the streamed pair
-  static constexpr int kX = 0;                        // stationary pair: (Q, dO) or (K, V)
-  static constexpr int kY = 2 * kTile;                // ring of streamed pairs
-  // dK/dV kernel: per-query statistics, [2 sets][2 halves][-lse2 x 64 | -delta x 64]
-  static constexpr int kStat = kY + kNS * 2 * kTile;
-  static constexpr int kBar = kStat + 2 * 2 * kBM * 4;
-  // barriers: X, Yfull[NS], Yempty[NS], Sfull[2], Pfull[2], Odone, End
-  static constexpr int kNBar = 1 + 2 * kNS + 6;
+  static constexpr int kNK = D == 128 ? 3 : 6;
+  static constexpr int kNV = D == 128 ? 2 : 4;
+  static constexpr int kX = 0;  // Q, then dO
+  static constexpr int kK = 2 * kTile;
+  static constexpr int kV = kK + kNK * kTile;
+  static constexpr int kBar = kV + kNV * kTile;
+  // barriers: X, Kfull[NK], Kempty[NK], Vfull[NV], Vempty[NV], Sfull, Read, Done[2], Odone, End
+  static constexpr int kNBar = 1 + 2 * kNK + 2 * kNV + 6;
   static constexpr int kTmemSlot = kBar + kNBar * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4 + 1024;  // + slack to align the base to 1024
   static_assert(kBytes <= 232448, "shared memory budget");
-  // epilogue staging of two 128-row fp32 tiles of up to D columns (+4 pad)
+  static_assert(2 * kBM * (D / 2 + 4) * 4 <= kBar, "output staging fits in the tile buffers");
+};
+
+// Shared memory of the dK/dV kernel: K and V stay; Q and dO stream (dO(j+1)
+// is needed first, as soon as tile j's scores are read, so its ring is the
+// deeper one), plus the -lse2 / -Delta of the current query tile.
+template <int D>
+struct BwdKVSmem {
+  static constexpr int kBox = kBM * 128;
+  static constexpr int kTile = kBox * (D / 64);
+  static constexpr int kNQ = D == 128 ? 2 : 4;
+  static constexpr int kNO = D == 128 ? 3 : 4;
+  static constexpr int kX = 0;  // K, then V
+  static constexpr int kQ = 2 * kTile;
+  static constexpr int kO = kQ + kNQ * kTile;
+  static constexpr int kStat = kO + kNO * kTile;  // -lse2 x 128 | -delta x 128
+  static constexpr int kBar = kStat + 2 * kBM * 4;
+  // barriers: X, Qfull[NQ], Qempty[NQ], Ofull[NO], Oempty[NO], Sfull, Read, Done[2], Odone, End
+  static constexpr int kNBar = 1 + 2 * kNQ + 2 * kNO + 6;
+  static constexpr int kTmemSlot = kBar + kNBar * 8;
+  static constexpr int kAbort = kTmemSlot + 4;
+  static constexpr int kBytes = kAbort + 4 + 1024;
+  static_assert(kBytes <= 232448, "shared memory budget");
   static_assert(2 * kBM * (D + 4) * 4 <= kStat, "output staging fits in the tile buffers");
 };
 
-// Tensor memory (512 columns).  Each 128-wide score tile is handled as two
-// 64-column halves h = 0, 1 with their own MMAs and barriers, so the
-// elementwise pass over one half overlaps the tensor-core work of the other:
-//   half h: scores S_h at [128h, 128h + 64), dP_h at [128h + 64, 128h + 128)
-//   fp32 accumulators from 256 (dQ; or dV, then dK)
-// The bf16 results of half h (dS, or P^T and dS^T) are written over the
-// first 32 columns of its own S_h / dP_h: chunk c (32 columns) lands on
-// columns of chunk 0 that the same thread has already read.
-constexpr int kTmAcc = 256;
+// Tensor memory (512 columns).
+//   dQ kernel:   S [0, 128), dP [128, 256), dQ [256, 256 + D),
+//                bf16 dS of tile j at [384 + 64 (j & 1), + 64) (two buffers,
+//                so tile j + 1's scores never wait for dQ(j) to read dS(j))
+//   dK/dV kernel: S^T [0, 128), dP^T [128, 256), dV [256, 256 + D),
+//                dK [384, 384 + D); the bf16 results of column half h go over
+//                S^T once every warp has read it: P^T at [64h, 64h + 32),
+//                dS^T at [64h + 32, 64h + 64)
+constexpr int kTmS = 0, kTmP = 128, kTmAcc = 256, kTmDS = 384;
 
 // Delta = rowsum(dO * O) and lse * log2(e), written as [B][Hq][S].  D / 4
 // threads per row, 4 elements each.
@@ -253,32 +285,32 @@ __device__ __forceinline__ void bwd_convert(const uint32_t (&sv)[32], const uint
   }
 }
 
-// Barrier indices shared by both kernels.
+// Barrier indices of the ring pair (r0 ring of n0 stages, r1 ring of n1).
 struct BwdBars {
   static constexpr int kX = 0;
-  int ns;
-  __device__ int yfull(int s) const { return 1 + s; }
-  __device__ int yempty(int s) const { return 1 + ns + s; }
-  __device__ int sfull(int h) const { return 1 + 2 * ns + h; }
-  __device__ int pfull(int h) const { return 3 + 2 * ns + h; }
-  __device__ int odone() const { return 5 + 2 * ns; }
-  __device__ int end() const { return 6 + 2 * ns; }
+  int n0, n1;
+  __device__ int full0(int s) const { return 1 + s; }
+  __device__ int empty0(int s) const { return 1 + n0 + s; }
+  __device__ int full1(int s) const { return 1 + 2 * n0 + s; }
+  __device__ int empty1(int s) const { return 1 + 2 * n0 + n1 + s; }
+  __device__ int sfull() const { return 1 + 2 * n0 + 2 * n1; }
+  __device__ int read() const { return 2 + 2 * n0 + 2 * n1; }
+  // column half h of the tile converted (P / dS in bf16 written)
+  __device__ int done(int h) const { return 3 + 2 * n0 + 2 * n1 + h; }
+  __device__ int odone() const { return 5 + 2 * n0 + 2 * n1; }
+  __device__ int end() const { return 6 + 2 * n0 + 2 * n1; }
 };
 
 // ------------------------------------------------------------------- dQ
-// MMA issue order over the CTA's KV tiles j (half h = keys 64h .. 64h + 63):
-//   S_0(0) dP_0(0), S_1(0) dP_1(0), then for every j:
-//   [P_0 ready] dQ += dS_0 K_0, S_0(j+1) dP_0(j+1),
-//   [P_1 ready] dQ += dS_1 K_1, release tile j, S_1(j+1) dP_1(j+1)
-// so the tensor core computes one half while the elementwise warps of the
-// other half run (warps 0-3 own half 0, warps 4-7 half 1).
+// MMA issue order over the CTA's KV tiles j:
+//   S(0) dP(0); then per j: [tile j read] S(j+1) dP(j+1), [dS(j) written] dQ += dS(j) K(j)
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                   const __grid_constant__ BwdArgs a) {
-  using SL = BwdSmem<D>;
-  constexpr int NS = SL::kNS;
+  using SL = BwdQSmem<D>;
+  constexpr int NK = SL::kNK, NV = SL::kNV;
   extern __shared__ uint8_t bsm_raw[];
   uint8_t* smem = bsm_raw + ((1024u - (smem_u32(bsm_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
@@ -305,13 +337,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   for (int s_ = 0; s_ < a.nblk; ++s_)
     for (int e_ = 0; e_ < a.nseg; ++e_) total += nt_of(s_, e_);
 
-  const BwdBars ib{NS};
+  const BwdBars ib{NK, NV};
   auto bar = [&](int i) -> uint32_t { return sb + SL::kBar + 8u * i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SL::kAbort);
   if (threadIdx.x == 0) {
     for (int i = 0; i < SL::kNBar; ++i) mbar_init(bar(i), 1);
-    mbar_init(bar(ib.pfull(0)), kBwdElem / 64);  // one arrival per warp of the half
-    mbar_init(bar(ib.pfull(1)), kBwdElem / 64);
+    mbar_init(bar(ib.read()), kBwdElem / 32);  // one arrival per elementwise warp
+    mbar_init(bar(ib.done(0)), kBwdElem / 32);  // one arrival per elementwise warp
+    mbar_init(bar(ib.done(1)), kBwdElem / 32);
     *abort_flag = grid_timed_out() ? 1 : 0;
     fence_mbar_init();
   }
@@ -333,85 +366,92 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tma_load_4d(sb + SL::kX + bx * SL::kBox, &tmQ, bx * 64, h, qs.mem + row0, b, bar(ib.kX));
         tma_load_4d(sb + SL::kX + SL::kTile + bx * SL::kBox, &tmdO, bx * 64, h, qs.mem + row0, b, bar(ib.kX));
       }
-      int j = 0, issued[NS];
-      for (int s = 0; s < NS; ++s) issued[s] = -1;
+      int j = 0, lastk[NK], lastv[NV];
+      for (int s = 0; s < NK; ++s) lastk[s] = -1;
+      for (int s = 0; s < NV; ++s) lastv[s] = -1;
       bool ok = true;
       for (int s_ = 0; s_ < a.nblk && ok; ++s_)
         for (int e_ = 0; e_ < a.nseg && ok; ++e_) {
           const Seg ks = a.seg[a.order[qi][s_]][e_];
           const int nt = nt_of(s_, e_);
           for (int t = 0; t < nt; ++t, ++j) {
-            const int st = j % NS;
-            if (!mbar_wait(bar(ib.yempty(st)), ((j / NS) & 1) ^ 1, abort_flag)) {
+            const int sk = j % NK, sv = j % NV, r = ks.mem + t * kBN;
+            if (!mbar_wait(bar(ib.empty0(sk)), ((j / NK) & 1) ^ 1, abort_flag)) {
               ok = false;
               break;
             }
-            const uint32_t y = sb + SL::kY + st * 2 * SL::kTile;
-            mbar_expect_tx(bar(ib.yfull(st)), 2 * SL::kTile);
-            for (int bx = 0; bx < D / 64; ++bx) {
-              tma_load_4d(y + bx * SL::kBox, &tmK, bx * 64, hk, ks.mem + t * kBN, b, bar(ib.yfull(st)));
-              tma_load_4d(y + SL::kTile + bx * SL::kBox, &tmV, bx * 64, hk, ks.mem + t * kBN, b, bar(ib.yfull(st)));
+            mbar_expect_tx(bar(ib.full0(sk)), SL::kTile);
+            for (int bx = 0; bx < D / 64; ++bx)
+              tma_load_4d(sb + SL::kK + sk * SL::kTile + bx * SL::kBox, &tmK, bx * 64, hk, r, b, bar(ib.full0(sk)));
+            lastk[sk] = j;
+            if (!mbar_wait(bar(ib.empty1(sv)), ((j / NV) & 1) ^ 1, abort_flag)) {
+              ok = false;
+              break;
             }
-            issued[st] = j;
+            mbar_expect_tx(bar(ib.full1(sv)), SL::kTile);
+            for (int bx = 0; bx < D / 64; ++bx)
+              tma_load_4d(sb + SL::kV + sv * SL::kTile + bx * SL::kBox, &tmV, bx * 64, hk, r, b, bar(ib.full1(sv)));
+            lastv[sv] = j;
           }
         }
       // every copy issued lands before the CTA can release its shared memory
       mbar_drain(bar(ib.kX), 0);
-      for (int s = 0; s < NS; ++s)
-        if (issued[s] >= 0) mbar_drain(bar(ib.yfull(s)), (issued[s] / NS) & 1);
+      for (int s = 0; s < NK; ++s)
+        if (lastk[s] >= 0) mbar_drain(bar(ib.full0(s)), (lastk[s] / NK) & 1);
+      for (int s = 0; s < NV; ++s)
+        if (lastv[s] >= 0) mbar_drain(bar(ib.full1(s)), (lastv[s] / NV) & 1);
     }
   } else if (warp == kBwdMma) {
     if (lane == 0 && work > 0) {
-      constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, 64, false);
+      constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t kIdescQ = idesc_bf16_f32(kBM, D, true);
-      // S_h = Q K_h^T and dP_h = dO V_h^T (K_h, V_h: rows 64h.. of the tile), K-major operands
-      auto issue_sdp = [&](int st, int hf) {
-        const uint32_t y = sb + SL::kY + st * 2 * SL::kTile + hf * 64 * 128;
+      // S = Q K(j)^T into [0, 128), dP = dO V(j)^T into [128, 256): K-major operands
+      auto issue_sdp = [&](int j) -> bool {
+        const int sk = j % NK, sv = j % NV;
+        if (!mbar_wait(bar(ib.full0(sk)), (j / NK) & 1, abort_flag) ||
+            !mbar_wait(bar(ib.full1(sv)), (j / NV) & 1, abort_flag))
+          return false;
+        tc_fence_after();
+        const uint32_t yk = sb + SL::kK + sk * SL::kTile, yv = sb + SL::kV + sv * SL::kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
-          mma_ss(tmem + 128 * hf, smem_desc_sw128(sb + SL::kX + off, 16, 1024), smem_desc_sw128(y + off, 16, 1024),
+          mma_ss(tmem + kTmS, smem_desc_sw128(sb + SL::kX + off, 16, 1024), smem_desc_sw128(yk + off, 16, 1024),
                  kIdescS, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
-          mma_ss(tmem + 128 * hf + 64, smem_desc_sw128(sb + SL::kX + SL::kTile + off, 16, 1024),
-                 smem_desc_sw128(y + SL::kTile + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + kTmP, smem_desc_sw128(sb + SL::kX + SL::kTile + off, 16, 1024),
+                 smem_desc_sw128(yv + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(ib.sfull(hf)));
+        tc_commit(bar(ib.empty1(sv)));  // V(j) is read only by dP(j)
+        tc_commit(bar(ib.sfull()));
+        return true;
       };
-      // dQ += dS_h K_h: A = bf16 dS_h in TMEM, B = rows 64h.. of the K tile read MN-major
-      auto issue_dq = [&](int st, int hf, bool acc) {
-        const uint32_t y = sb + SL::kY + st * 2 * SL::kTile;
+      // dQ += dS_h(j) K_h(j) over keys 64h .. 64h + 63: A = bf16 dS in TMEM,
+      // B = rows of K(j) read MN-major; after half 1, K(j) is free
+      auto issue_dq = [&](int j, int hf) {
+        const int sk = j % NK;
+        const uint32_t yk = sb + SL::kK + sk * SL::kTile;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + kTmAcc, tmem + 128 * hf + kk * 8, smem_desc_sw128(y + (hf * 4 + kk) * 2048, SL::kBox, 1024),
-                 kIdescQ, (acc || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + kTmAcc, tmem + kTmDS + 64 * (j & 1) + 32 * hf + kk * 8,
+                 smem_desc_sw128(yk + (4 * hf + kk) * 2048, SL::kBox, 1024), kIdescQ,
+                 (j > 0 || hf > 0 || kk > 0) ? 1u : 0u);
+        if (hf == 1) tc_commit(bar(ib.empty0(sk)));
       };
-      bool ok = mbar_wait(bar(ib.kX), 0, abort_flag) && mbar_wait(bar(ib.yfull(0)), 0, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        issue_sdp(0, 0);
-        issue_sdp(0, 1);
-      }
+      bool ok = mbar_wait(bar(ib.kX), 0, abort_flag) && issue_sdp(0);
       for (int j = 0; ok && j < work; ++j) {
-        const int st = j % NS, st1 = (j + 1) % NS;
-        const bool more = j + 1 < work;
+        if (j + 1 < work) {
+          ok = mbar_wait(bar(ib.read()), j & 1, abort_flag) && issue_sdp(j + 1);
+          if (!ok) break;
+        }
         for (int hf = 0; hf < 2 && ok; ++hf) {
-          ok = mbar_wait(bar(ib.pfull(hf)), j & 1, abort_flag);
+          ok = mbar_wait(bar(ib.done(hf)), j & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          issue_dq(st, hf, j > 0 || hf > 0);
-          if (hf == 1) tc_commit(bar(ib.yempty(st)));
-          if (more) {
-            if (hf == 0) {
-              ok = mbar_wait(bar(ib.yfull(st1)), ((j + 1) / NS) & 1, abort_flag);
-              if (!ok) break;
-              tc_fence_after();
-            }
-            issue_sdp(st1, hf);
-          }
+          issue_dq(j, hf);
         }
       }
       tc_commit(bar(ib.odone()));
@@ -420,12 +460,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- elementwise
-    const int quad = warp & 3, half = warp >> 2;
+    const int quad = warp & 3, half = warp >> 2;  // half: the 32-column slice of each column half
     const int row = quad * 32 + lane;
     const bool valid = row < rows;
     const int qpos = valid ? qs.pos + row0 + row : -1;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_base + 128 * half, tP = tS + 64;
+    const uint32_t tS = tmem + lane_base + kTmS + 32 * half, tP = tmem + lane_base + kTmP + 32 * half;
     const long long stat = (static_cast<long long>(b) * a.Hq + h) * a.S + max(qpos, 0);
     // padding rows: -lse2 = -inf, so every P is 0
     const float nl = valid ? -a.lse2[stat] : -INFINITY;
@@ -439,26 +479,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int nt = nt_of(s_, e_);
         const int lim = bwd_visible(a, ks, qpos);
         for (int t = 0; t < nt; ++t, ++j) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(ib.sfull(half)), j & 1, abort_flag));
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(ib.sfull()), j & 1, abort_flag));
           if (!ok) break;
           tc_fence_after();
-          // keys of this half visible to the row: [0, cnt)
-          const int cnt = lim - t * kBN - 64 * half;
-          const bool full = __all_sync(0xffffffffu, !valid || cnt >= 64);
-#pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            uint32_t sv[32], pv[32], pk[16];
-            tmem_ld32x2_wait(tS + 32 * cc, tP + 32 * cc, sv, pv);
-            if (full)
-              bwd_convert<false, false, false>(sv, pv, ss, &nl, &nd, 0, 0, pk, pk);
-            else
-              bwd_convert<false, true, false>(sv, pv, ss, &nl, &nd, 0, cnt - 32 * cc, pk, pk);
-            tmem_st16(tS + 16 * cc, pk);  // over columns this thread has read
-          }
-          tmem_wait_st();
+          uint32_t sv[2][32], pv[2][32];
+          tmem_ld32x2_wait(tS, tS + 64, sv[0], sv[1]);
+          tmem_ld32x2_wait(tP, tP + 64, pv[0], pv[1]);
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(ib.pfull(half)));
+          if (lane == 0) mbar_arrive(bar(ib.read()));  // S and dP may be overwritten now
+          const uint32_t dst = tmem + lane_base + kTmDS + 64 * (j & 1) + 16 * half;
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            // keys of this 32-column slice visible to the row: [0, cnt)
+            const int cnt = lim - t * kBN - 64 * hf - 32 * half;
+            uint32_t pk[16];
+            if (__all_sync(0xffffffffu, !valid || cnt >= 32))
+              bwd_convert<false, false, false>(sv[hf], pv[hf], ss, &nl, &nd, 0, 0, pk, pk);
+            else
+              bwd_convert<false, true, false>(sv[hf], pv[hf], ss, &nl, &nd, 0, cnt, pk, pk);
+            tmem_st16(dst + 32 * hf, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(ib.done(hf)));
+          }
         }
       }
     // ---- epilogue: this CTA's dQ rows; column half h of every row by warps 4h..4h+3
@@ -466,7 +511,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (ok) {
       tc_fence_after();
       constexpr int NC = D / 2;
-      // every product is complete (odone): the tile buffers are free
+      // every product is complete (odone): the tile buffers are free; warps
+      // 4w..4w+3 store column half w of the rows
       float* stage = reinterpret_cast<float*>(smem) + half * kBM * (NC + 4);
       bwd_store_rows<NC>(stage, tmem + lane_base + kTmAcc + half * NC, quad, lane, a.dq + half * NC,
                          (static_cast<long long>(b) * a.S + qs.pos + row0) * a.Hq + h, a.Hq, D, rows, a.scale);
@@ -479,15 +525,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // ----------------------------------------------------------------- dK, dV
-// Same pipeline over the CTA's query tiles j (half h = queries 64h .. 64h + 63):
-//   S^T_h = K Q_h^T, dP^T_h = V dO_h^T; then dV += P^T_h dO_h, dK += dS^T_h Q_h.
+// MMA issue order over the CTA's query tiles j:
+//   S^T(0) dP^T(0); then per j: [tile j read] dP^T(j+1),
+//   [P^T(j), dS^T(j) written] dV += P^T(j) dO(j), dK += dS^T(j) Q(j), S^T(j+1)
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                    const __grid_constant__ BwdArgs a) {
-  using SL = BwdSmem<D>;
-  constexpr int NS = SL::kNS;
+  using SL = BwdKVSmem<D>;
+  constexpr int NQ = SL::kNQ, NO = SL::kNO;
   extern __shared__ uint8_t bsm_raw[];
   uint8_t* smem = bsm_raw + ((1024u - (smem_u32(bsm_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
@@ -526,13 +573,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
   total *= a.groups;
 
-  const BwdBars ib{NS};
+  const BwdBars ib{NQ, NO};
   auto bar = [&](int i) -> uint32_t { return sb + SL::kBar + 8u * i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SL::kAbort);
   if (threadIdx.x == 0) {
     for (int i = 0; i < SL::kNBar; ++i) mbar_init(bar(i), 1);
-    mbar_init(bar(ib.pfull(0)), kBwdElem / 64);
-    mbar_init(bar(ib.pfull(1)), kBwdElem / 64);
+    mbar_init(bar(ib.read()), kBwdElem / 32);
+    mbar_init(bar(ib.done(0)), kBwdElem / 32);  // one arrival per elementwise warp
+    mbar_init(bar(ib.done(1)), kBwdElem / 32);
     *abort_flag = grid_timed_out() ? 1 : 0;
     fence_mbar_init();
   }
@@ -554,8 +602,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tma_load_4d(sb + SL::kX + bx * SL::kBox, &tmK, bx * 64, g, ks.mem + key0, b, bar(ib.kX));
         tma_load_4d(sb + SL::kX + SL::kTile + bx * SL::kBox, &tmV, bx * 64, g, ks.mem + key0, b, bar(ib.kX));
       }
-      int j = 0, issued[NS];
-      for (int s = 0; s < NS; ++s) issued[s] = -1;
+      int j = 0, lastq[NQ], lasto[NO];
+      for (int s = 0; s < NQ; ++s) lastq[s] = -1;
+      for (int s = 0; s < NO; ++s) lasto[s] = -1;
       bool ok = true;
       for (int hh = 0; hh < a.groups && ok; ++hh)
         for (int s_ = 0; s_ < a.nblk && ok; ++s_)
@@ -563,82 +612,103 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             for (int t = 0; t < a.seg_tiles; ++t) {
               int q0, qr;
               if (!q_tile(s_, e_, t, q0, qr)) continue;
-              const int st = j % NS;
-              if (!mbar_wait(bar(ib.yempty(st)), ((j / NS) & 1) ^ 1, abort_flag)) {
+              const int hq = g * a.groups + hh, r = q_mem(s_, e_, t);
+              const int sq = j % NQ, so_ = j % NO;
+              // dO(j) first: dP^T(j) is issued before S^T(j)
+              if (!mbar_wait(bar(ib.empty1(so_)), ((j / NO) & 1) ^ 1, abort_flag)) {
                 ok = false;
                 break;
               }
-              const uint32_t y = sb + SL::kY + st * 2 * SL::kTile;
-              const int hq = g * a.groups + hh, qm = q_mem(s_, e_, t);
-              mbar_expect_tx(bar(ib.yfull(st)), 2 * SL::kTile);
-              for (int bx = 0; bx < D / 64; ++bx) {
-                tma_load_4d(y + bx * SL::kBox, &tmQ, bx * 64, hq, qm, b, bar(ib.yfull(st)));
-                tma_load_4d(y + SL::kTile + bx * SL::kBox, &tmdO, bx * 64, hq, qm, b, bar(ib.yfull(st)));
+              mbar_expect_tx(bar(ib.full1(so_)), SL::kTile);
+              for (int bx = 0; bx < D / 64; ++bx)
+                tma_load_4d(sb + SL::kO + so_ * SL::kTile + bx * SL::kBox, &tmdO, bx * 64, hq, r, b,
+                            bar(ib.full1(so_)));
+              lasto[so_] = j;
+              if (!mbar_wait(bar(ib.empty0(sq)), ((j / NQ) & 1) ^ 1, abort_flag)) {
+                ok = false;
+                break;
               }
-              issued[st] = j;
+              mbar_expect_tx(bar(ib.full0(sq)), SL::kTile);
+              for (int bx = 0; bx < D / 64; ++bx)
+                tma_load_4d(sb + SL::kQ + sq * SL::kTile + bx * SL::kBox, &tmQ, bx * 64, hq, r, b, bar(ib.full0(sq)));
+              lastq[sq] = j;
               ++j;
             }
       mbar_drain(bar(ib.kX), 0);
-      for (int s = 0; s < NS; ++s)
-        if (issued[s] >= 0) mbar_drain(bar(ib.yfull(s)), (issued[s] / NS) & 1);
+      for (int s = 0; s < NQ; ++s)
+        if (lastq[s] >= 0) mbar_drain(bar(ib.full0(s)), (lastq[s] / NQ) & 1);
+      for (int s = 0; s < NO; ++s)
+        if (lasto[s] >= 0) mbar_drain(bar(ib.full1(s)), (lasto[s] / NO) & 1);
     }
   } else if (warp == kBwdMma) {
     if (lane == 0 && work > 0) {
-      constexpr uint32_t kIdescS = idesc_bf16_f32(kBN, 64, false);
+      constexpr uint32_t kIdescS = idesc_bf16_f32(kBN, kBM, false);
       constexpr uint32_t kIdescO = idesc_bf16_f32(kBN, D, true);
-      // S^T_h = K Q_h^T and dP^T_h = V dO_h^T (Q_h, dO_h: rows 64h.. of the tile)
-      auto issue_sdp = [&](int st, int hf) {
-        const uint32_t y = sb + SL::kY + st * 2 * SL::kTile + hf * 64 * 128;
+      // S^T = K Q(j)^T into [0, 128)
+      auto issue_s = [&](int j) -> bool {
+        const int sq = j % NQ;
+        if (!mbar_wait(bar(ib.full0(sq)), (j / NQ) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t yq = sb + SL::kQ + sq * SL::kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
-          mma_ss(tmem + 128 * hf, smem_desc_sw128(sb + SL::kX + off, 16, 1024), smem_desc_sw128(y + off, 16, 1024),
+          mma_ss(tmem + kTmS, smem_desc_sw128(sb + SL::kX + off, 16, 1024), smem_desc_sw128(yq + off, 16, 1024),
                  kIdescS, kk > 0 ? 1u : 0u);
         }
+        return true;
+      };
+      // dP^T = V dO(j)^T into [128, 256)
+      auto issue_dp = [&](int j) -> bool {
+        const int so_ = j % NO;
+        if (!mbar_wait(bar(ib.full1(so_)), (j / NO) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t yo = sb + SL::kO + so_ * SL::kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
-          mma_ss(tmem + 128 * hf + 64, smem_desc_sw128(sb + SL::kX + SL::kTile + off, 16, 1024),
-                 smem_desc_sw128(y + SL::kTile + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + kTmP, smem_desc_sw128(sb + SL::kX + SL::kTile + off, 16, 1024),
+                 smem_desc_sw128(yo + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(ib.sfull(hf)));
+        return true;
       };
-      // dV += P^T_h dO_h and dK += dS^T_h Q_h: A = bf16 in TMEM, B read MN-major
-      auto issue_dkv = [&](int st, int hf, bool acc) {
-        const uint32_t y = sb + SL::kY + st * 2 * SL::kTile;
+      // dV += P^T_h(j) dO_h(j), dK += dS^T_h(j) Q_h(j) over queries 64h .. 64h + 63:
+      // A = bf16 in TMEM (P^T_h at [64h, 64h + 32), dS^T_h at [64h + 32, 64h + 64)),
+      // B = rows of dO(j) / Q(j) read MN-major; after half 1 both tiles are free
+      auto issue_dkv = [&](int j, int hf) {
+        const uint32_t yq = sb + SL::kQ + (j % NQ) * SL::kTile, yo = sb + SL::kO + (j % NO) * SL::kTile;
+        const bool acc = j > 0 || hf > 0;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + kTmAcc, tmem + 128 * hf + kk * 8,
-                 smem_desc_sw128(y + SL::kTile + (hf * 4 + kk) * 2048, SL::kBox, 1024), kIdescO,
-                 (acc || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + kTmAcc, tmem + 64 * hf + 8 * kk, smem_desc_sw128(yo + (4 * hf + kk) * 2048, SL::kBox, 1024),
+                 kIdescO, (acc || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + kTmAcc + 128, tmem + 128 * hf + 64 + kk * 8,
-                 smem_desc_sw128(y + (hf * 4 + kk) * 2048, SL::kBox, 1024), kIdescO, (acc || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + kTmAcc + 128, tmem + 64 * hf + 32 + 8 * kk,
+                 smem_desc_sw128(yq + (4 * hf + kk) * 2048, SL::kBox, 1024), kIdescO, (acc || kk > 0) ? 1u : 0u);
+        if (hf == 1) {
+          tc_commit(bar(ib.empty1(j % NO)));
+          tc_commit(bar(ib.empty0(j % NQ)));
+        }
       };
-      bool ok = mbar_wait(bar(ib.kX), 0, abort_flag) && mbar_wait(bar(ib.yfull(0)), 0, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        issue_sdp(0, 0);
-        issue_sdp(0, 1);
-      }
+      bool ok = mbar_wait(bar(ib.kX), 0, abort_flag) && issue_dp(0) && issue_s(0);
+      if (ok) tc_commit(bar(ib.sfull()));
       for (int j = 0; ok && j < work; ++j) {
-        const int st = j % NS, st1 = (j + 1) % NS;
-        const bool more = j + 1 < work;
+        if (j + 1 < work) {
+          ok = mbar_wait(bar(ib.read()), j & 1, abort_flag) && issue_dp(j + 1);
+          if (!ok) break;
+        }
         for (int hf = 0; hf < 2 && ok; ++hf) {
-          ok = mbar_wait(bar(ib.pfull(hf)), j & 1, abort_flag);
+          ok = mbar_wait(bar(ib.done(hf)), j & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          issue_dkv(st, hf, j > 0 || hf > 0);
-          if (hf == 1) tc_commit(bar(ib.yempty(st)));
-          if (more) {
-            if (hf == 0) {
-              ok = mbar_wait(bar(ib.yfull(st1)), ((j + 1) / NS) & 1, abort_flag);
-              if (!ok) break;
-              tc_fence_after();
-            }
-            issue_sdp(st1, hf);
-          }
+          issue_dkv(j, hf);
+        }
+        if (!ok) break;
+        if (j + 1 < work) {
+          ok = issue_s(j + 1);
+          if (!ok) break;
+          tc_commit(bar(ib.sfull()));
         }
       }
       tc_commit(bar(ib.odone()));
@@ -647,14 +717,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- elementwise
-    // Thread (quad, lane) owns key row quad * 32 + lane; warps 4h..4h+3 own
-    // query half h of every tile.
+    // Thread (quad, lane) owns key row quad * 32 + lane; warps 4w..4w+3 own
+    // query columns 64h + 32w .. 64h + 32w + 31 of column half h = 0, 1.
     const int quad = warp & 3, half = warp >> 2;
     const int row = quad * 32 + lane;
     const int kpos = row < krows ? first_k + row : -1;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_base + 128 * half, tP = tS + 64;
-    float* stat = reinterpret_cast<float*>(smem + SL::kStat);
+    const uint32_t tS = tmem + lane_base + kTmS, tP = tmem + lane_base + kTmP;
+    float* set = reinterpret_cast<float*>(smem + SL::kStat);  // -lse2 x 128 | -delta x 128
     const float ss = a.scale_log2;
     bool ok = work > 0;
     int j = 0;
@@ -664,37 +734,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           for (int t = 0; t < a.seg_tiles; ++t) {
             int q0, qrows;
             if (!q_tile(s_, e_, t, q0, qrows)) continue;
-            // -lse2 (rows 0-63 of the half's warps) and -delta (rows 64-127) of
-            // the half's 64 queries, into the set that tile j - 1 does not read
-            float* set = stat + ((j & 1) * 2 + half) * kBM;
-            {
-              const int c = 64 * half + (row & 63);
-              const long long at = (static_cast<long long>(b) * a.Hq + g * a.groups + hh) * a.S + q0 + c;
-              set[row] = row < 64 ? (c < qrows ? -a.lse2[at] : -INFINITY) : (c < qrows ? -a.delta[at] : 0.f);
-            }
-            const bool w = mbar_wait(bar(ib.sfull(half)), j & 1, abort_flag);
-            ok = bar_and(1 + half, kBM, w);  // one decision for the half's 4 warps; publishes `set`
+            // -lse2 (threads 0-127) and -delta (threads 128-255) of the tile's queries
+            const int c = threadIdx.x & (kBM - 1);
+            const long long at = (static_cast<long long>(b) * a.Hq + g * a.groups + hh) * a.S + q0 + c;
+            const float v = threadIdx.x < kBM ? (c < qrows ? -a.lse2[at] : -INFINITY)
+                                              : (c < qrows ? -a.delta[at] : 0.f);
+            named_barrier_sync(1, kBwdElem);  // every warp is done with tile j - 1's values
+            set[threadIdx.x] = v;
+            const bool w = mbar_wait(bar(ib.sfull()), j & 1, abort_flag);
+            ok = bar_and(1, kBwdElem, w);  // one decision for all 8 warps; publishes `set`
             if (!ok) break;
             tc_fence_after();
-            // when causal, this key sees the half's query columns [lo, 64)
-            const int lo = a.causal && kpos >= 0 ? kpos - q0 - 64 * half : -64;
-            const bool full = __all_sync(0xffffffffu, lo <= 0);
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-              uint32_t sv[32], pv[32], pp[16], pd[16];
-              tmem_ld32x2_wait(tS + 32 * cc, tP + 32 * cc, sv, pv);
-              if (full)
-                bwd_convert<true, false, true>(sv, pv, ss, set + 32 * cc, set + 64 + 32 * cc, 0, 0, pp, pd);
-              else
-                bwd_convert<true, true, true>(sv, pv, ss, set + 32 * cc, set + 64 + 32 * cc, lo - 32 * cc, 64, pp,
-                                              pd);
-              tmem_st16(tS + 16 * cc, pp);  // P^T over columns this thread has read
-              tmem_st16(tP + 16 * cc, pd);  // dS^T likewise
-            }
-            tmem_wait_st();
+            uint32_t sv[2][32], pv[2][32];
+            tmem_ld32x2_wait(tS + 32 * half, tS + 64 + 32 * half, sv[0], sv[1]);
+            tmem_ld32x2_wait(tP + 32 * half, tP + 64 + 32 * half, pv[0], pv[1]);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(ib.pfull(half)));
+            if (lane == 0) mbar_arrive(bar(ib.read()));  // dP^T may be overwritten now
+            named_barrier_sync(1, kBwdElem);             // every warp has read S^T: it may be overwritten
+            tc_fence_after();
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              const int c0 = 64 * hf + 32 * half;
+              // when causal, this key sees the slice's query columns [lo, 32)
+              const int lo = a.causal && kpos >= 0 ? kpos - q0 - c0 : -32;
+              uint32_t pp[16], pd[16];
+              if (__all_sync(0xffffffffu, lo <= 0))
+                bwd_convert<true, false, true>(sv[hf], pv[hf], ss, set + c0, set + kBM + c0, 0, 0, pp, pd);
+              else
+                bwd_convert<true, true, true>(sv[hf], pv[hf], ss, set + c0, set + kBM + c0, lo, 32, pp, pd);
+              tmem_st16(tS + 64 * hf + 16 * half, pp);       // P^T_h
+              tmem_st16(tS + 64 * hf + 32 + 16 * half, pd);  // dS^T_h
+              tmem_wait_st();
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(bar(ib.done(hf)));
+            }
             ++j;
           }
     // ---- epilogue: dV rows by warps 0-3, dK rows by warps 4-7
