@@ -79,8 +79,8 @@ struct BwdQSmem {
   static constexpr int kK = 2 * kTile;
   static constexpr int kV = kK + kNK * kTile;
   static constexpr int kBar = kV + kNV * kTile;
-  // barriers: X, Kfull[NK], Kempty[NK], Vfull[NV], Vempty[NV], Sfull, Read, Done[2], Odone, End
-  static constexpr int kNBar = 1 + 2 * kNK + 2 * kNV + 6;
+  // barriers: X, Kfull[NK], Kempty[NK], Vfull[NV], Vempty[NV], Sfull, Read, Done[2][2], Odone, End
+  static constexpr int kNBar = 1 + 2 * kNK + 2 * kNV + 8;
   static constexpr int kTmemSlot = kBar + kNBar * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4 + 1024;  // + slack to align the base to 1024
@@ -102,8 +102,8 @@ struct BwdKVSmem {
   static constexpr int kO = kQ + kNQ * kTile;
   static constexpr int kStat = kO + kNO * kTile;  // -lse2 x 128 | -delta x 128
   static constexpr int kBar = kStat + 2 * kBM * 4;
-  // barriers: X, Qfull[NQ], Qempty[NQ], Ofull[NO], Oempty[NO], Sfull, Read, Done[2], Odone, End
-  static constexpr int kNBar = 1 + 2 * kNQ + 2 * kNO + 6;
+  // barriers: X, Qfull[NQ], Qempty[NQ], Ofull[NO], Oempty[NO], Sfull, Read, Done[2][2], Odone, End
+  static constexpr int kNBar = 1 + 2 * kNQ + 2 * kNO + 8;
   static constexpr int kTmemSlot = kBar + kNBar * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4 + 1024;
@@ -295,10 +295,16 @@ struct BwdBars {
   __device__ int empty1(int s) const { return 1 + 2 * n0 + n1 + s; }
   __device__ int sfull() const { return 1 + 2 * n0 + 2 * n1; }
   __device__ int read() const { return 2 + 2 * n0 + 2 * n1; }
-  // column half h of the tile converted (P / dS in bf16 written)
-  __device__ int done(int h) const { return 3 + 2 * n0 + 2 * n1 + h; }
-  __device__ int odone() const { return 5 + 2 * n0 + 2 * n1; }
-  __device__ int end() const { return 6 + 2 * n0 + 2 * n1; }
+  // column half h of tile j converted (P / dS in bf16 written).  Tiles of
+  // each parity have their own pair: in the dQ kernel the next tile's scores
+  // are released before the MMA thread waits for this tile's halves, so one
+  // barrier per half could complete twice before it is polled; a second
+  // completion of done(h, j) needs tile j + 2's scores, which the MMA thread
+  // only issues after it has consumed done(h, j).  Polled with parity
+  // (j >> 1) & 1.
+  __device__ int done(int h, int j) const { return 3 + 2 * n0 + 2 * n1 + 2 * (j & 1) + h; }
+  __device__ int odone() const { return 7 + 2 * n0 + 2 * n1; }
+  __device__ int end() const { return 8 + 2 * n0 + 2 * n1; }
 };
 
 // ------------------------------------------------------------------- dQ
@@ -343,8 +349,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < SL::kNBar; ++i) mbar_init(bar(i), 1);
     mbar_init(bar(ib.read()), kBwdElem / 32);  // one arrival per elementwise warp
-    mbar_init(bar(ib.done(0)), kBwdElem / 32);  // one arrival per elementwise warp
-    mbar_init(bar(ib.done(1)), kBwdElem / 32);
+    for (int i = 0; i < 4; ++i) mbar_init(bar(ib.done(i & 1, i >> 1)), kBwdElem / 32);  // one arrival per warp
     *abort_flag = grid_timed_out() ? 1 : 0;
     fence_mbar_init();
   }
@@ -448,7 +453,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (!ok) break;
         }
         for (int hf = 0; hf < 2 && ok; ++hf) {
-          ok = mbar_wait(bar(ib.done(hf)), j & 1, abort_flag);
+          ok = mbar_wait(bar(ib.done(hf, j)), (j >> 1) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
           issue_dq(j, hf);
@@ -502,7 +507,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(ib.done(hf)));
+            if (lane == 0) mbar_arrive(bar(ib.done(hf, j)));
           }
         }
       }
@@ -579,8 +584,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < SL::kNBar; ++i) mbar_init(bar(i), 1);
     mbar_init(bar(ib.read()), kBwdElem / 32);
-    mbar_init(bar(ib.done(0)), kBwdElem / 32);  // one arrival per elementwise warp
-    mbar_init(bar(ib.done(1)), kBwdElem / 32);
+    for (int i = 0; i < 4; ++i) mbar_init(bar(ib.done(i & 1, i >> 1)), kBwdElem / 32);  // one arrival per warp
     *abort_flag = grid_timed_out() ? 1 : 0;
     fence_mbar_init();
   }
@@ -699,7 +703,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (!ok) break;
         }
         for (int hf = 0; hf < 2 && ok; ++hf) {
-          ok = mbar_wait(bar(ib.done(hf)), j & 1, abort_flag);
+          ok = mbar_wait(bar(ib.done(hf, j)), (j >> 1) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
           issue_dkv(j, hf);
@@ -768,7 +772,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               tmem_wait_st();
               tc_fence_before();
               __syncwarp();
-              if (lane == 0) mbar_arrive(bar(ib.done(hf)));
+              if (lane == 0) mbar_arrive(bar(ib.done(hf, j)));
             }
             ++j;
           }
