@@ -186,23 +186,28 @@ def local_gpu_id(dev):
     return f"GPU-{gpu_id}" if not str(gpu_id).startswith("GPU-") else gpu_id
 
 
-def kernel_sha():
+FWD_SOURCES = ["attn_fwd.cuh", "common.cuh", "tmem_ld.cuh", "merge_rule.cuh"]
+BWD_SOURCES = FWD_SOURCES + ["attn_bwd.cuh"]
+
+
+def kernel_sha(files=FWD_SOURCES):
     import hashlib
     h = hashlib.sha256()
     src = os.path.join(ROOT, "blockwise_exact_attention_block_b200", "csrc")
-    for f in ["attn_fwd.cuh", "common.cuh", "tmem_ld.cuh", "merge_rule.cuh"]:
+    for f in files:
         h.update(open(os.path.join(src, f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def attn_traffic(workload):
-    """DRAM bytes per attention launch from the committed ncu capture, or None
-    when there is none for this workload or the kernel changed since."""
-    path = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
+def attn_traffic(workload, record="attn_fwd_traffic.json", files=FWD_SOURCES):
+    """DRAM bytes per launch (per call for the backward's two kernels) from the
+    committed ncu capture, or None when there is none for this workload or the
+    kernel sources changed since."""
+    path = os.path.join(ROOT, "profiles", record)
     if not os.path.exists(path):
         return None
     rec = json.load(open(path)).get(workload)
-    if not rec or rec.get("kernel_sha") != kernel_sha():
+    if not rec or rec.get("kernel_sha") != kernel_sha(files):
         return None
     return rec["dram_bytes_per_launch"]
 
@@ -401,7 +406,8 @@ def run_backward(args):
             "config": dict(workload_config(w, args, f"flushed ({L2_FLUSH_BYTES >> 20} MiB write between calls)"),
                            flops_per_step=2.5 * w.flops),
             "roofline": {"bound": "tensor", "achieved": ktf, "peak": peak, "unit": "TFLOP/s", "frac": ktf / peak,
-                         "traffic": None, "kernel": "bwd_dkv_kernel + bwd_dq_kernel",
+                         "traffic": attn_traffic(w.name, "attn_bwd_traffic.json", BWD_SOURCES),
+                         "kernel": "bwd_dkv_kernel + bwd_dq_kernel",
                          "peak_source": f"{pk_kind} {'sustained' if sustained else 'burst'} bf16 dense"},
             "kernels_ms": kms, "clocks": clk, "gpu_launches": reps * (3 if w.in_dtype == "bf16" else 7),
             "device_status": ra.ra_status_string(status)}
@@ -555,7 +561,8 @@ def run_ours(args):
         bpeak = pk["bf16_tflops_sustained" if bkms > 100.0 else "bf16_tflops"]
         backward = {"kernel": "bwd_dkv_kernel + bwd_dq_kernel (+ bwd_prep_kernel in the call)",
                     "workload": w.name, "flops_per_step": 2.5 * w.flops, "TFLOP/s": tf, "kernels_TFLOP/s": ktf,
-                    "ms": bms, "kernels_ms": bkms, "peak_TFLOP/s": bpeak, "frac": ktf / bpeak}
+                    "ms": bms, "kernels_ms": bkms, "peak_TFLOP/s": bpeak, "frac": ktf / bpeak,
+                    "traffic": attn_traffic(w.name, "attn_bwd_traffic.json", BWD_SOURCES)}
 
     value = replica_throughput(w.flops, world, K, total_ms)
     line = {"metric": "causal-adj attention TFLOP/s (% of dense bf16 peak)", "value": value, "unit": "TFLOP/s",
