@@ -48,6 +48,9 @@ constexpr int kBwdThreads = 320;
 constexpr int kBwdElem = 256;  // elementwise threads (warps 0-7)
 constexpr int kBwdProducer = 8;
 constexpr int kBwdMma = 9;
+// Tiles between drains of the tensor-core accumulators (see bwd_flush_row):
+// bounds every accumulation to 256 x 8 products of 16.  A power of two.
+constexpr int kFlushTiles = 256;
 
 struct BwdArgs {
   int B, S, Hq, Hkv, groups, causal;
@@ -79,8 +82,9 @@ struct BwdQSmem {
   static constexpr int kK = 2 * kTile;
   static constexpr int kV = kK + kNK * kTile;
   static constexpr int kBar = kV + kNV * kTile;
-  // barriers: X, Kfull[NK], Kempty[NK], Vfull[NV], Vempty[NV], Sfull, Read, Done[2][2], Odone, End
-  static constexpr int kNBar = 1 + 2 * kNK + 2 * kNV + 8;
+  // barriers: X, Kfull[NK], Kempty[NK], Vfull[NV], Vempty[NV], Sfull, Read, Done[2][2], Odone, End,
+  // Flush full / empty
+  static constexpr int kNBar = 1 + 2 * kNK + 2 * kNV + 10;
   static constexpr int kTmemSlot = kBar + kNBar * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4 + 1024;  // + slack to align the base to 1024
@@ -102,8 +106,9 @@ struct BwdKVSmem {
   static constexpr int kO = kQ + kNQ * kTile;
   static constexpr int kStat = kO + kNO * kTile;  // -lse2 x 128 | -delta x 128
   static constexpr int kBar = kStat + 2 * kBM * 4;
-  // barriers: X, Qfull[NQ], Qempty[NQ], Ofull[NO], Oempty[NO], Sfull, Read, Done[2][2], Odone, End
-  static constexpr int kNBar = 1 + 2 * kNQ + 2 * kNO + 8;
+  // barriers: X, Qfull[NQ], Qempty[NQ], Ofull[NO], Oempty[NO], Sfull, Read, Done[2][2], Odone, End,
+  // Flush full / empty
+  static constexpr int kNBar = 1 + 2 * kNQ + 2 * kNO + 10;
   static constexpr int kTmemSlot = kBar + kNBar * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4 + 1024;
@@ -209,13 +214,13 @@ __device__ __forceinline__ bool bar_and(int id, int count, bool pred) {
 }
 
 // One warp's 32 rows of an fp32 128 x NC tile in TMEM (columns taddr ..
-// taddr + NC), times `mul`, to global memory: through a padded staging
-// buffer, then whole rows, 16 bytes per lane.  Row r of the tile goes to
+// taddr + NC), times `mul`, to global memory (added to what is there when
+// `add`): through a padded staging buffer, then whole rows, 16 bytes per lane.  Row r of the tile goes to
 // dst + (first_row + r * row_stride) * ld; rows r >= nrows are not written.
 template <int NC>
 __device__ __forceinline__ void bwd_store_rows(float* stage, uint32_t taddr, int quad, int lane, float* dst,
                                                long long first_row, long long row_stride, int ld, int nrows,
-                                               float mul) {
+                                               float mul, bool add) {
   constexpr int kStride = NC + 4;
   const int row = quad * 32 + lane;
 #pragma unroll
@@ -234,11 +239,45 @@ __device__ __forceinline__ void bwd_store_rows(float* stage, uint32_t taddr, int
 #pragma unroll 4
   for (int r0 = 0; r0 < 32; r0 += rpi) {
     const int r = quad * 32 + r0 + rl;
-    if (r < nrows)
-      *reinterpret_cast<float4*>(dst + (first_row + r * row_stride) * ld + 4 * ci) =
-          *reinterpret_cast<const float4*>(stage + r * kStride + 4 * ci);
+    if (r < nrows) {
+      float4* p = reinterpret_cast<float4*>(dst + (first_row + r * row_stride) * ld + 4 * ci);
+      float4 val = *reinterpret_cast<const float4*>(stage + r * kStride + 4 * ci);
+      if (add) {
+        const float4 old = *p;
+        val.x += old.x, val.y += old.y, val.z += old.z, val.w += old.w;
+      }
+      *p = val;
+    }
   }
   __syncwarp();
+}
+
+// The tensor core adds each product into its fp32 accumulator without
+// rounding to nearest, so over very long sums (a key tile at the start of a
+// 1M-token sequence meets ~8,000 query tiles per query head) the error
+// drifts one way.  Every kFlushTiles tiles the accumulator is therefore
+// drained into the fp32 output with ordinary (round-to-nearest) adds and the
+// next product restarts it.  This thread's row, NC columns from taddr:
+// dst[c] (+)= mul * acc[c].
+template <int NC>
+__device__ __forceinline__ void bwd_flush_row(uint32_t taddr, float* dst, bool valid, bool add, float mul) {
+#pragma unroll
+  for (int q = 0; q < NC / 32; ++q) {
+    uint32_t v[32];
+    tmem_ld32_wait(taddr + 32 * q, v);
+    if (valid) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        float4* p = reinterpret_cast<float4*>(dst + 32 * q + i);
+        float4 o = add ? *p : make_float4(0.f, 0.f, 0.f, 0.f);
+        o.x += __uint_as_float(v[i]) * mul;
+        o.y += __uint_as_float(v[i + 1]) * mul;
+        o.z += __uint_as_float(v[i + 2]) * mul;
+        o.w += __uint_as_float(v[i + 3]) * mul;
+        *p = o;
+      }
+    }
+  }
 }
 
 __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
@@ -305,6 +344,10 @@ struct BwdBars {
   __device__ int done(int h, int j) const { return 3 + 2 * n0 + 2 * n1 + 2 * (j & 1) + h; }
   __device__ int odone() const { return 7 + 2 * n0 + 2 * n1; }
   __device__ int end() const { return 8 + 2 * n0 + 2 * n1; }
+  // accumulator drain (see bwd_flush_row): full = the products of the last
+  // kFlushTiles tiles are complete; empty = the warps have read the accumulator
+  __device__ int ffull() const { return 9 + 2 * n0 + 2 * n1; }
+  __device__ int fempty() const { return 10 + 2 * n0 + 2 * n1; }
 };
 
 // ------------------------------------------------------------------- dQ
@@ -350,6 +393,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int i = 0; i < SL::kNBar; ++i) mbar_init(bar(i), 1);
     mbar_init(bar(ib.read()), kBwdElem / 32);  // one arrival per elementwise warp
     for (int i = 0; i < 4; ++i) mbar_init(bar(ib.done(i & 1, i >> 1)), kBwdElem / 32);  // one arrival per warp
+    mbar_init(bar(ib.fempty()), kBwdElem / 32);
     *abort_flag = grid_timed_out() ? 1 : 0;
     fence_mbar_init();
   }
@@ -443,7 +487,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int kk = 0; kk < 4; ++kk)
           mma_ts(tmem + kTmAcc, tmem + kTmDS + 64 * (j & 1) + 32 * hf + kk * 8,
                  smem_desc_sw128(yk + (4 * hf + kk) * 2048, SL::kBox, 1024), kIdescQ,
-                 (j > 0 || hf > 0 || kk > 0) ? 1u : 0u);
+                 (j % kFlushTiles > 0 || hf > 0 || kk > 0) ? 1u : 0u);
         if (hf == 1) tc_commit(bar(ib.empty0(sk)));
       };
       bool ok = mbar_wait(bar(ib.kX), 0, abort_flag) && issue_sdp(0);
@@ -452,12 +496,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           ok = mbar_wait(bar(ib.read()), j & 1, abort_flag) && issue_sdp(j + 1);
           if (!ok) break;
         }
+        constexpr int F = kFlushTiles;
         for (int hf = 0; hf < 2 && ok; ++hf) {
           ok = mbar_wait(bar(ib.done(hf, j)), (j >> 1) & 1, abort_flag);
+          // the accumulator restarts at tile j: the previous sum has been drained
+          if (ok && hf == 0 && j > 0 && j % F == 0) ok = mbar_wait(bar(ib.fempty()), (j / F - 1) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
           issue_dq(j, hf);
         }
+        if (ok && (j + 1) % F == 0 && j + 1 < work) tc_commit(bar(ib.ffull()));
       }
       tc_commit(bar(ib.odone()));
       tc_commit(bar(ib.end()));
@@ -484,6 +532,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int nt = nt_of(s_, e_);
         const int lim = bwd_visible(a, ks, qpos);
         for (int t = 0; t < nt; ++t, ++j) {
+          if (j > 0 && j % kFlushTiles == 0) {
+            // drain the accumulator (tiles j - kFlushTiles .. j - 1) into dq
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(ib.ffull()), (j / kFlushTiles - 1) & 1, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            constexpr int NC = D / 2;
+            bwd_flush_row<NC>(tmem + lane_base + kTmAcc + half * NC,
+                              a.dq + ((static_cast<long long>(b) * a.S + qs.pos + row0 + row) * a.Hq + h) * D +
+                                  half * NC,
+                              valid, j > kFlushTiles, a.scale);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(ib.fempty()));
+          }
           ok = __all_sync(0xffffffffu, mbar_wait(bar(ib.sfull()), j & 1, abort_flag));
           if (!ok) break;
           tc_fence_after();
@@ -520,7 +582,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // 4w..4w+3 store column half w of the rows
       float* stage = reinterpret_cast<float*>(smem) + half * kBM * (NC + 4);
       bwd_store_rows<NC>(stage, tmem + lane_base + kTmAcc + half * NC, quad, lane, a.dq + half * NC,
-                         (static_cast<long long>(b) * a.S + qs.pos + row0) * a.Hq + h, a.Hq, D, rows, a.scale);
+                         (static_cast<long long>(b) * a.S + qs.pos + row0) * a.Hq + h, a.Hq, D, rows, a.scale,
+                         work > kFlushTiles);
     }
   }
   tc_fence_before();
@@ -585,6 +648,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int i = 0; i < SL::kNBar; ++i) mbar_init(bar(i), 1);
     mbar_init(bar(ib.read()), kBwdElem / 32);
     for (int i = 0; i < 4; ++i) mbar_init(bar(ib.done(i & 1, i >> 1)), kBwdElem / 32);  // one arrival per warp
+    mbar_init(bar(ib.fempty()), kBwdElem / 32);
     *abort_flag = grid_timed_out() ? 1 : 0;
     fence_mbar_init();
   }
@@ -681,7 +745,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // B = rows of dO(j) / Q(j) read MN-major; after half 1 both tiles are free
       auto issue_dkv = [&](int j, int hf) {
         const uint32_t yq = sb + SL::kQ + (j % NQ) * SL::kTile, yo = sb + SL::kO + (j % NO) * SL::kTile;
-        const bool acc = j > 0 || hf > 0;
+        const bool acc = j % kFlushTiles > 0 || hf > 0;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_ts(tmem + kTmAcc, tmem + 64 * hf + 8 * kk, smem_desc_sw128(yo + (4 * hf + kk) * 2048, SL::kBox, 1024),
@@ -702,13 +766,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           ok = mbar_wait(bar(ib.read()), j & 1, abort_flag) && issue_dp(j + 1);
           if (!ok) break;
         }
+        constexpr int F = kFlushTiles;
         for (int hf = 0; hf < 2 && ok; ++hf) {
           ok = mbar_wait(bar(ib.done(hf, j)), (j >> 1) & 1, abort_flag);
+          // the accumulators restart at tile j: the previous sums have been drained
+          if (ok && hf == 0 && j > 0 && j % F == 0) ok = mbar_wait(bar(ib.fempty()), (j / F - 1) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
           issue_dkv(j, hf);
         }
         if (!ok) break;
+        if ((j + 1) % F == 0 && j + 1 < work) tc_commit(bar(ib.ffull()));
         if (j + 1 < work) {
           ok = issue_s(j + 1);
           if (!ok) break;
@@ -738,6 +806,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           for (int t = 0; t < a.seg_tiles; ++t) {
             int q0, qrows;
             if (!q_tile(s_, e_, t, q0, qrows)) continue;
+            if (j > 0 && j % kFlushTiles == 0) {
+              // drain the accumulators (tiles j - kFlushTiles .. j - 1): dV by
+              // warps 0-3, dK by warps 4-7
+              // one decision for all 8 warps (they meet at named barriers below)
+              ok = bar_and(1, kBwdElem, mbar_wait(bar(ib.ffull()), (j / kFlushTiles - 1) & 1, abort_flag));
+              if (!ok) break;
+              tc_fence_after();
+              bwd_flush_row<D>(tmem + lane_base + kTmAcc + half * 128,
+                               (half ? a.dk : a.dv) +
+                                   ((static_cast<long long>(b) * a.S + ks.pos + key0 + row) * a.Hkv + g) * D,
+                               row < krows, j > kFlushTiles, half ? a.scale : 1.f);
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(bar(ib.fempty()));
+            }
             // -lse2 (threads 0-127) and -delta (threads 128-255) of the tile's queries
             const int c = threadIdx.x & (kBM - 1);
             const long long at = (static_cast<long long>(b) * a.Hq + g * a.groups + hh) * a.S + q0 + c;
@@ -783,7 +866,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       float* stage = reinterpret_cast<float*>(smem) + half * kBM * (D + 4);
       bwd_store_rows<D>(stage, tmem + lane_base + kTmAcc + half * 128, quad, lane, half ? a.dk : a.dv,
                         (static_cast<long long>(b) * a.S + ks.pos + key0) * a.Hkv + g, a.Hkv, D, krows,
-                        half ? a.scale : 1.f);
+                        half ? a.scale : 1.f, work > kFlushTiles);
     }
   }
   tc_fence_before();

@@ -131,6 +131,37 @@ def test_backward_zero_upstream_gradient(cuda_lib):
         assert int(torch.count_nonzero(g)) == 0
 
 
+def test_backward_accumulator_drains(cuda_lib):
+    """Long walks drain the tensor-core accumulators into the fp32 outputs
+    every 256 tiles.  Here the first key tile meets 64 query tiles of each of
+    8 query heads (512 tiles: one drain in the dK/dV kernel), checked against
+    the whole oracle gradient."""
+    ra = cuda_lib
+    B, S, Hq, Hkv, D, n = 1, 8192, 8, 1, 128, 2
+    q, k, v, do = backward_inputs(B, S, Hq, Hkv, D, "bf16", seed=11)
+    _, _, dq, dk, dv = run(ra, q, k, v, do, n, True, "zigzag", torch.float32)
+    rq, rk, rv = G.attention_backward(q, k, v, do, True, Hq // Hkv)
+    assert_grad_close(to_np(dq), rq, "dq")
+    assert_grad_close(to_np(dk), rk, "dk")
+    assert_grad_close(to_np(dv), rv, "dv")
+    assert ra.ra_get_device_status() == 0
+
+
+def test_backward_accumulator_drains_dq(cuda_lib):
+    """dQ drains: the last query tile of a 40,960-token sequence walks 320 KV
+    tiles (one drain); its rows against the oracle, row by row."""
+    ra = cuda_lib
+    B, S, Hq, Hkv, D, n = 1, 40960, 2, 1, 128, 4
+    q, k, v, do = backward_inputs(B, S, Hq, Hkv, D, "bf16", seed=12)
+    o, l, dq, dk, dv = run(ra, q, k, v, do, n, True, "contiguous", torch.float32)
+    rows = [(0, i, h) for h in range(Hq) for i in (S - 1, S - 60, S - 128, S - 129, 33000, 100)]
+    ref = G.backward_query_rows(q, k, v, do, rows, True, Hq // Hkv)
+    bi, ii, hi = (torch.tensor([r[t] for r in rows]) for t in range(3))
+    assert_grad_close(to_np(dq.cpu()[bi, ii, hi]), ref, "dq rows")
+    check_identities(q, k, v, do, o, dq, dk, dv, Hq // Hkv, "S=40960")
+    assert ra.ra_get_device_status() == 0
+
+
 # ------------------------------------------------------ full-size workloads
 
 def check_identities(q, k, v, do, o, dq, dk, dv, groups, what):
@@ -204,3 +235,34 @@ def test_backward_workload(cuda_lib, name):
     bi, ji, gi = (torch.tensor([r[t] for r in keys]) for t in range(3))
     assert_grad_close(to_np(dk.cpu()[bi, ji, gi]), rk, f"{name} dk late keys")
     assert_grad_close(to_np(dv.cpu()[bi, ji, gi]), rv, f"{name} dv late keys")
+
+
+def test_backward_long1m_workload(cuda_lib):
+    """1,048,576 tokens, 8 zigzag blocks, GQA 8/2, bf16 out: the identities
+    over the whole gradient, sampled dq rows, and dk, dv of late keys (each
+    from the full rows of the few queries that see it).  The oracle gets one
+    query head (or one KV group) at a time, sliced out, so it holds ~1 GB."""
+    ra = cuda_lib
+    w = WORKLOADS["long1m"]
+    q, k, v, do = backward_inputs(w.B, w.S, w.Hq, w.Hkv, w.D, w.in_dtype, seed=10)
+    o, l, dq, dk, dv = run(ra, q, k, v, do, w.n_blocks, w.causal, w.partition, torch.bfloat16)
+    assert ra.ra_get_device_status() == 0
+    check_identities(q, k, v, do, o, dq, dk, dv, w.gqa_groups, "long1m")
+    o = l = None
+    dq, dk, dv = dq.cpu(), dk.cpu(), dv.cpu()
+    torch.cuda.empty_cache()
+    rng = np.random.default_rng(3)
+    G_ = w.gqa_groups
+    for h in (0, w.Hq - 1):  # one query head of each KV group
+        g = h // G_
+        rows = sorted({int(x) for x in rng.integers(0, w.S, 3)} | {w.S - 1})
+        ref = G.backward_query_rows(q[:, :, h:h + 1], k[:, :, g:g + 1], v[:, :, g:g + 1], do[:, :, h:h + 1],
+                                    [(0, i, 0) for i in rows], True, 1)
+        assert_grad_close(to_np(dq[0, rows, h]), ref, f"long1m dq rows head {h}")
+    for g in range(w.Hkv):
+        keys = [w.S - 1 - 5 * g]
+        sl = slice(g * G_, (g + 1) * G_)
+        rk, rv = G.backward_key_rows(q[:, :, sl], k[:, :, g:g + 1], v[:, :, g:g + 1], do[:, :, sl],
+                                     [(0, j, 0) for j in keys], True, G_)
+        assert_grad_close(to_np(dk[0, keys, g]), rk, f"long1m dk late keys group {g}")
+        assert_grad_close(to_np(dv[0, keys, g]), rv, f"long1m dv late keys group {g}")
