@@ -65,6 +65,9 @@ CASES = [
     (1, 1200, 4, 2, 128, 4, True, "zigzag", "bf16", torch.float32, "ring"),         # 150-row chunks
     (1, 512, 2, 1, 128, 16, True, "zigzag", "bf16", torch.float32, "tokenring"),    # 16 blocks, 16-row chunks
     (1, 640, 2, 2, 128, 5, False, "zigzag", "bf16", torch.float32, "ring"),         # non-causal zigzag
+    (1, 32, 2, 1, 64, 16, True, "zigzag", "bf16", torch.float32, "ring"),           # 1-row chunks
+    (2, 200, 2, 2, 128, 1, True, "contiguous", "bf16", torch.bfloat16, "ring"),     # one ragged 200-row block
+    (1, 96, 4, 4, 64, 3, False, "contiguous", "f32", torch.float32, "tokenring"),   # 32-row blocks, fp32
 ]
 
 
