@@ -47,7 +47,7 @@ EXPORTED = ["ra_block_attn", "ra_merge_partial", "ra_merge_partials", "ra_ring_a
 
 class ra_options(ctypes.Structure):
     _fields_ = [("order", ctypes.c_int), ("sched", ctypes.c_int), ("attn_event_begin", ctypes.c_void_p),
-                ("attn_event_end", ctypes.c_void_p), ("tiling", ctypes.c_int)]
+                ("attn_event_end", ctypes.c_void_p), ("tiling", ctypes.c_int), ("fault_inject", ctypes.c_int)]
 
 
 TILINGS = {"auto": 0, "row_pairs": 1, "kv_split": 2, "cluster2": 3}
@@ -132,8 +132,8 @@ def _dtype_code(dt: torch.dtype) -> int:
     raise ValueError(f"unsupported dtype {dt}")
 
 
-def _opts(order: str, sched: str, events=None, tiling: str = "auto") -> ra_options:
-    o = ra_options(ORDERS[order], SCHEDS[sched], None, None, TILINGS[tiling])
+def _opts(order: str, sched: str, events=None, tiling: str = "auto", fault_inject: int = 0) -> ra_options:
+    o = ra_options(ORDERS[order], SCHEDS[sched], None, None, TILINGS[tiling], fault_inject)
     if events is not None:
         for ev in events:
             if ev.cuda_event == 0:  # torch creates the CUDA event on its first record
@@ -198,11 +198,12 @@ def ra_ring_attention_workspace(B, S, Hq, D, n_blocks, gqa_groups, partition="co
 def ra_ring_attention(q, k, v, n_blocks: int, causal: bool, partition: str = "contiguous",
                       gqa_groups: int | None = None, out=None, out_dtype=torch.float32, lse=None,
                       workspace=None, order: str = "ring", sched: str = "auto", stream=None,
-                      attn_events=None, tiling: str = "auto"):
+                      attn_events=None, tiling: str = "auto", fault_inject: int = 0):
     """The whole method on one GPU.  Returns (out [B, S, Hq, D], lse fp32 [B, S, Hq]).
 
     attn_events: optional pair of torch.cuda.Event recorded around the
-    block-attention launches inside the call."""
+    block-attention launches inside the call.  fault_inject=1 is for testing
+    the failure path only (see ra_options in include/ra.h)."""
     B, S, Hq, D = q.shape
     Hkv = k.shape[2]
     if gqa_groups is None:
@@ -216,7 +217,7 @@ def ra_ring_attention(q, k, v, n_blocks: int, causal: bool, partition: str = "co
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    o = _opts(order, sched, attn_events, tiling)
+    o = _opts(order, sched, attn_events, tiling, fault_inject)
     _check(_lib.ra_ring_attention(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q.dtype), B, S, Hq, D, n_blocks,
                                   int(bool(causal)), PARTITIONS[partition], gqa_groups, _ptr(out),
                                   _dtype_code(out.dtype), _ptr(lse), _ptr(workspace), ws_bytes, ctypes.byref(o),

@@ -307,6 +307,7 @@ bool valid_opts(const ra_options* o) {
   if (!o) return true;
   if (o->order != RA_ORDER_RING && o->order != RA_ORDER_TOKENRING) return false;
   if (o->tiling < RA_TILING_AUTO || o->tiling > RA_TILING_CLUSTER2) return false;
+  if (o->fault_inject != 0 && o->fault_inject != 1) return false;
   return o->sched >= RA_SCHED_AUTO && o->sched <= RA_SCHED_PERSISTENT;
 }
 
@@ -687,6 +688,7 @@ ra_status ra_ring_attention(const void* q, const void* k, const void* v, ra_dtyp
   }
   order_segments(a);
   choose_tiling(g, a, opts ? opts->tiling : RA_TILING_AUTO);
+  a.fault_inject = opts ? opts->fault_inject : 0;
 
   if (p.sched == RA_SCHED_PERSISTENT) {
     // a3-a6 in one launch: the running state is carried across block boundaries

@@ -112,6 +112,7 @@ struct AttnArgs {
   void* out;
   float* lse;
   int out_bf16;
+  int fault_inject;       // 1: the producer withholds its second K tile (failure-path tests)
   Seg qseg[kMaxBlocks][2];                      // segments of the i-th query block of the launch
   Seg kvseg[kMaxBlocks][2];                     // segments of KV block r
   signed char kv_list[kMaxBlocks][kMaxBlocks];  // kv_list[i][s]: s-th KV block met by query block i
@@ -440,11 +441,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const Seg ks = seg_tab[use_b ? wb.sg : wa.sg].seg;
         const int sk = g % NSK, sv = g % NSV;
         if (!mbar_wait(bar(BKE(sk)), ((g / NSK) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        mbar_expect_tx(bar(BKF(sk)), SL::kTile);
-        for (int bx = 0; bx < SL::kNBox; ++bx)
-          tma_load_4d(sb + SL::kK + sk * SL::kTile + bx * SL::kBox, &tmK, bx * 64, hk, ks.mem + t * kBN, b,
-                      bar(BKF(sk)));
-        issued_k[sk] = g;
+        if (!(a.fault_inject && g == 1)) {  // an injected fault: this K tile never arrives
+          mbar_expect_tx(bar(BKF(sk)), SL::kTile);
+          for (int bx = 0; bx < SL::kNBox; ++bx)
+            tma_load_4d(sb + SL::kK + sk * SL::kTile + bx * SL::kBox, &tmK, bx * 64, hk, ks.mem + t * kBN, b,
+                        bar(BKF(sk)));
+          issued_k[sk] = g;
+        }
         if (!mbar_wait(bar(BVE(sv)), ((g / NSV) & 1) ^ 1, abort_flag)) { ok = false; break; }
         mbar_expect_tx(bar(BVF(sv)), SL::kTile);
         for (int bx = 0; bx < SL::kNBox; ++bx)

@@ -109,6 +109,14 @@ typedef struct {
   void* attn_event_begin;
   void* attn_event_end;
   ra_tiling tiling; /* default RA_TILING_AUTO */
+  /* Testing the failure path only; 0 (off) in normal use.  1: the TMA
+   * producer of every block-attention CTA withholds the second K tile it
+   * would load, so the tensor-core issuer's bounded wait for it expires
+   * (about 1 s of SM clocks): the kernel records RA_ERR_TIMEOUT in the device
+   * status word, every CTA stops at its next wait, in-flight copies and
+   * products are drained, and the call's outputs are undefined.  The context
+   * stays usable.  Other values: RA_ERR_INVALID_ARG. */
+  int fault_inject;
 } ra_options;
 
 /*
@@ -290,8 +298,8 @@ int ra_decode_splits(int B, int Tq, int Skv, int Hq, int Hkv, int D, int n_split
  *  opts          NULL for defaults; `order` sets the order in which the
  *                block pairs are summed (results agree up to rounding);
  *                attn_event_begin / attn_event_end bracket the two
- *                tensor-core kernels (dK/dV, then dQ).  sched and tiling are
- *                ignored.
+ *                tensor-core kernels (dK/dV, then dQ).  sched, tiling and
+ *                fault_inject are ignored.
  * Every pointer must be 16-byte aligned (else RA_ERR_INVALID_ARG).  Each
  * output row is written by exactly one CTA (no atomics): the result does not
  * depend on scheduling.

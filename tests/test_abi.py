@@ -82,6 +82,8 @@ def test_ring_attention_rejects_bad_arguments(ra):
     assert ring(ra, opts=ctypes.byref(bad)) == E.RA_ERR_INVALID_ARG
     bad_tiling = ra.ra_options(0, 0, None, None, 9)
     assert ring(ra, opts=ctypes.byref(bad_tiling)) == E.RA_ERR_INVALID_ARG
+    bad_fault = ra.ra_options(0, 0, None, None, 0, 2)
+    assert ring(ra, opts=ctypes.byref(bad_fault)) == E.RA_ERR_INVALID_ARG
 
 
 def test_block_attn_rejects_bad_arguments(ra):
