@@ -84,6 +84,29 @@ def test_merge_partial_matches_oracle(cuda_lib, T):
     check_merge(o, l, ref_o, ref_l)
 
 
+def test_merge_partial_full_size_sampled_rows(cuda_lib):
+    """The bench's merge: two [1,048,576, 32, 128] fp32 partials (16 GiB each,
+    drawn on the device from a seeded generator, with the workload's
+    distributions).  Sampled rows, copied out before and after the merge, are
+    checked against the fp64 rule."""
+    ra = cuda_lib
+    T, H, D = 1048576, 32, 128
+    g = torch.Generator(device="cuda").manual_seed(7)
+    out = torch.randn((T, H, D), device="cuda", generator=g)
+    lse = torch.rand((T, H), device="cuda", generator=g) * 20 - 5
+    bo = torch.randn((T, H, D), device="cuda", generator=g)
+    bl = torch.rand((T, H), device="cuda", generator=g) * 20 - 5
+    bl[T - 1, :3] = float("-inf")  # empty partials at the last token
+    rng = np.random.default_rng(8)
+    ti = torch.from_numpy(np.unique(np.concatenate([rng.integers(0, T, 2048), [0, T - 1]])))
+    before = [x[ti.cuda()].double().cpu().numpy() for x in (out, lse, bo, bl)]
+    ra.ra_merge_partial(out, lse, bo, bl)
+    torch.cuda.synchronize()
+    ref_o, ref_l = K.merge_rule(*before)
+    check_merge(out[ti.cuda()], lse[ti.cuda()], ref_o, ref_l)
+    assert ra.ra_get_device_status() == 0
+
+
 @pytest.mark.parametrize("k", [2, 4, 8, 16])
 def test_merge_partials_matches_oracle(cuda_lib, k):
     ra = cuda_lib
