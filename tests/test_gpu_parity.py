@@ -107,6 +107,26 @@ def test_merge_partial_full_size_sampled_rows(cuda_lib):
     assert ra.ra_get_device_status() == 0
 
 
+@pytest.mark.parametrize("T,k", [(1048576, 4), (131072, 16)])
+def test_merge_partials_large_sampled_rows(cuda_lib, T, k):
+    """The k-way merge at the sweep's sizes (16 partials of 1M tokens would
+    need 256 GiB, so k = 16 runs at 131,072 tokens): partials drawn on the
+    device from a seeded generator, sampled rows against the fp64 k-way rule."""
+    ra = cuda_lib
+    H, D = 32, 128
+    g = torch.Generator(device="cuda").manual_seed(9 + k)
+    outs = [torch.randn((T, H, D), device="cuda", generator=g) for _ in range(k)]
+    lses = [torch.rand((T, H), device="cuda", generator=g) * 20 - 5 for _ in range(k)]
+    rng = np.random.default_rng(k)
+    ti = torch.from_numpy(np.unique(np.concatenate([rng.integers(0, T, 1024), [0, T - 1]]))).cuda()
+    ref_o, ref_l = K.merge_partials([o[ti].double().cpu().numpy() for o in outs],
+                                    [l[ti].double().cpu().numpy() for l in lses])
+    go, gl = ra.ra_merge_partials(outs, lses)
+    torch.cuda.synchronize()
+    check_merge(go[ti], gl[ti], ref_o, ref_l)
+    assert ra.ra_get_device_status() == 0
+
+
 @pytest.mark.parametrize("k", [2, 4, 8, 16])
 def test_merge_partials_matches_oracle(cuda_lib, k):
     ra = cuda_lib
