@@ -83,8 +83,8 @@ struct BwdQSmem {
   static constexpr int kV = kK + kNK * kTile;
   static constexpr int kBar = kV + kNV * kTile;
   // barriers: X, Kfull[NK], Kempty[NK], Vfull[NV], Vempty[NV], Sfull, Read, Done[2][2], Odone, End,
-  // Flush full / empty
-  static constexpr int kNBar = 1 + 2 * kNK + 2 * kNV + 10;
+  // Flush full / empty, Sfull of half 1
+  static constexpr int kNBar = 1 + 2 * kNK + 2 * kNV + 11;
   static constexpr int kTmemSlot = kBar + kNBar * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4 + 1024;  // + slack to align the base to 1024
@@ -107,8 +107,8 @@ struct BwdKVSmem {
   static constexpr int kStat = kO + kNO * kTile;  // -lse2 x 128 | -delta x 128
   static constexpr int kBar = kStat + 2 * kBM * 4;
   // barriers: X, Qfull[NQ], Qempty[NQ], Ofull[NO], Oempty[NO], Sfull, Read, Done[2][2], Odone, End,
-  // Flush full / empty
-  static constexpr int kNBar = 1 + 2 * kNQ + 2 * kNO + 10;
+  // Flush full / empty, Sfull of half 1
+  static constexpr int kNBar = 1 + 2 * kNQ + 2 * kNO + 11;
   static constexpr int kTmemSlot = kBar + kNBar * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4 + 1024;
@@ -348,6 +348,9 @@ struct BwdBars {
   // kFlushTiles tiles are complete; empty = the warps have read the accumulator
   __device__ int ffull() const { return 9 + 2 * n0 + 2 * n1; }
   __device__ int fempty() const { return 10 + 2 * n0 + 2 * n1; }
+  // dK/dV kernel: the scores of query half h of the tile are ready (half 0
+  // uses sfull())
+  __device__ int sfull_h(int h) const { return h ? 11 + 2 * n0 + 2 * n1 : sfull(); }
 };
 
 // ------------------------------------------------------------------- dQ
@@ -593,9 +596,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // ----------------------------------------------------------------- dK, dV
-// MMA issue order over the CTA's query tiles j:
-//   S^T(0) dP^T(0); then per j: [tile j read] dP^T(j+1),
-//   [P^T(j), dS^T(j) written] dV += P^T(j) dO(j), dK += dS^T(j) Q(j), S^T(j+1)
+// MMA issue order over the CTA's query tiles j (half h = queries 64h .. 64h + 63):
+//   dP^T(0), S^T_0(0), S^T_1(0); then per j:
+//   [half 0 of tile j converted] dV, dK += half 0,
+//   [tile j's scores read]       dP^T(j+1), S^T_0(j+1),
+//   [half 1 converted]           dV, dK += half 1, S^T_1(j+1)
+// S^T is issued in 64-query halves so that tile j+1's half-0 conversion runs
+// while the tensor core finishes tile j's half 1.
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -712,17 +719,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0 && work > 0) {
       constexpr uint32_t kIdescS = idesc_bf16_f32(kBN, kBM, false);
       constexpr uint32_t kIdescO = idesc_bf16_f32(kBN, D, true);
-      // S^T = K Q(j)^T into [0, 128)
-      auto issue_s = [&](int j) -> bool {
+      // S^T_h = K Q_h(j)^T into [64h, 64h + 64): Q_h = rows 64h.. of the Q tile
+      constexpr uint32_t kIdescS2 = idesc_bf16_f32(kBN, 64, false);
+      auto issue_s = [&](int j, int hf) -> bool {
         const int sq = j % NQ;
         if (!mbar_wait(bar(ib.full0(sq)), (j / NQ) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t yq = sb + SL::kQ + sq * SL::kTile;
+        const uint32_t yq = sb + SL::kQ + sq * SL::kTile + hf * 64 * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
-          mma_ss(tmem + kTmS, smem_desc_sw128(sb + SL::kX + off, 16, 1024), smem_desc_sw128(yq + off, 16, 1024),
-                 kIdescS, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + kTmS + 64 * hf, smem_desc_sw128(sb + SL::kX + off, 16, 1024),
+                 smem_desc_sw128(yq + off, 16, 1024), kIdescS2, kk > 0 ? 1u : 0u);
         }
         return true;
       };
@@ -759,28 +767,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_commit(bar(ib.empty0(j % NQ)));
         }
       };
-      bool ok = mbar_wait(bar(ib.kX), 0, abort_flag) && issue_dp(0) && issue_s(0);
-      if (ok) tc_commit(bar(ib.sfull()));
+      bool ok = mbar_wait(bar(ib.kX), 0, abort_flag) && issue_dp(0) && issue_s(0, 0);
+      if (ok) tc_commit(bar(ib.sfull_h(0)));
+      ok = ok && issue_s(0, 1);
+      if (ok) tc_commit(bar(ib.sfull_h(1)));
+      constexpr int F = kFlushTiles;
       for (int j = 0; ok && j < work; ++j) {
-        if (j + 1 < work) {
-          ok = mbar_wait(bar(ib.read()), j & 1, abort_flag) && issue_dp(j + 1);
-          if (!ok) break;
-        }
-        constexpr int F = kFlushTiles;
-        for (int hf = 0; hf < 2 && ok; ++hf) {
-          ok = mbar_wait(bar(ib.done(hf, j)), (j >> 1) & 1, abort_flag);
-          // the accumulators restart at tile j: the previous sums have been drained
-          if (ok && hf == 0 && j > 0 && j % F == 0) ok = mbar_wait(bar(ib.fempty()), (j / F - 1) & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          issue_dkv(j, hf);
-        }
+        const bool more = j + 1 < work;
+        // half 0 of tile j converted: its products (the accumulators restart
+        // at a drain tile once the previous sums have been drained)
+        ok = mbar_wait(bar(ib.done(0, j)), (j >> 1) & 1, abort_flag);
+        if (ok && j > 0 && j % F == 0) ok = mbar_wait(bar(ib.fempty()), (j / F - 1) & 1, abort_flag);
         if (!ok) break;
-        if ((j + 1) % F == 0 && j + 1 < work) tc_commit(bar(ib.ffull()));
-        if (j + 1 < work) {
-          ok = issue_s(j + 1);
+        tc_fence_after();
+        issue_dkv(j, 0);
+        // tile j's scores are in registers: the next tile's dP^T and S^T half 0
+        if (more) {
+          ok = mbar_wait(bar(ib.read()), j & 1, abort_flag) && issue_dp(j + 1) && issue_s(j + 1, 0);
           if (!ok) break;
-          tc_commit(bar(ib.sfull()));
+          tc_commit(bar(ib.sfull_h(0)));
+        }
+        ok = mbar_wait(bar(ib.done(1, j)), (j >> 1) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_dkv(j, 1);
+        if ((j + 1) % F == 0 && more) tc_commit(bar(ib.ffull()));
+        if (more) {
+          ok = issue_s(j + 1, 1);
+          if (!ok) break;
+          tc_commit(bar(ib.sfull_h(1)));
         }
       }
       tc_commit(bar(ib.odone()));
@@ -828,28 +843,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                               : (c < qrows ? -a.delta[at] : 0.f);
             named_barrier_sync(1, kBwdElem);  // every warp is done with tile j - 1's values
             set[threadIdx.x] = v;
-            const bool w = mbar_wait(bar(ib.sfull()), j & 1, abort_flag);
-            ok = bar_and(1, kBwdElem, w);  // one decision for all 8 warps; publishes `set`
-            if (!ok) break;
-            tc_fence_after();
-            uint32_t sv[2][32], pv[2][32];
-            tmem_ld32x2_wait(tS + 32 * half, tS + 64 + 32 * half, sv[0], sv[1]);
-            tmem_ld32x2_wait(tP + 32 * half, tP + 64 + 32 * half, pv[0], pv[1]);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(ib.read()));  // dP^T may be overwritten now
-            named_barrier_sync(1, kBwdElem);             // every warp has read S^T: it may be overwritten
-            tc_fence_after();
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
+              // the scores of query half hf; the first decision also publishes `set`
+              const bool w = mbar_wait(bar(ib.sfull_h(hf)), j & 1, abort_flag);
+              ok = bar_and(1, kBwdElem, w);  // one decision for all 8 warps
+              if (!ok) break;
+              tc_fence_after();
               const int c0 = 64 * hf + 32 * half;
+              uint32_t sv[32], pv[32];
+              tmem_ld32x2_wait(tS + c0, tP + c0, sv, pv);
+              tc_fence_before();
+              __syncwarp();
+              if (hf == 1 && lane == 0) mbar_arrive(bar(ib.read()));  // dP^T may be overwritten now
+              named_barrier_sync(1, kBwdElem);  // every warp has read half hf of S^T: it may be overwritten
+              tc_fence_after();
               // when causal, this key sees the slice's query columns [lo, 32)
               const int lo = a.causal && kpos >= 0 ? kpos - q0 - c0 : -32;
               uint32_t pp[16], pd[16];
               if (__all_sync(0xffffffffu, lo <= 0))
-                bwd_convert<true, false, true>(sv[hf], pv[hf], ss, set + c0, set + kBM + c0, 0, 0, pp, pd);
+                bwd_convert<true, false, true>(sv, pv, ss, set + c0, set + kBM + c0, 0, 0, pp, pd);
               else
-                bwd_convert<true, true, true>(sv[hf], pv[hf], ss, set + c0, set + kBM + c0, lo, 32, pp, pd);
+                bwd_convert<true, true, true>(sv, pv, ss, set + c0, set + kBM + c0, lo, 32, pp, pd);
               tmem_st16(tS + 64 * hf + 16 * half, pp);       // P^T_h
               tmem_st16(tS + 64 * hf + 32 + 16 * half, pd);  // dS^T_h
               tmem_wait_st();
@@ -857,6 +872,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               __syncwarp();
               if (lane == 0) mbar_arrive(bar(ib.done(hf, j)));
             }
+            if (!ok) break;
             ++j;
           }
     // ---- epilogue: dV rows by warps 0-3, dK rows by warps 4-7
