@@ -38,7 +38,7 @@ ORDERS = {"ring": RA_ORDER_RING, "tokenring": RA_ORDER_TOKENRING}
 SCHEDS = {"auto": RA_SCHED_AUTO, "unfused": RA_SCHED_UNFUSED, "fused": RA_SCHED_EPILOGUE_FUSED,
           "persistent": RA_SCHED_PERSISTENT}
 
-EXPORTED = ["ra_block_attn", "ra_merge_partial", "ra_merge_partials", "ra_ring_attention",
+EXPORTED = ["ra_block_attn", "ra_block_attn_merge", "ra_merge_partial", "ra_merge_partials", "ra_ring_attention",
             "ra_ring_attention_workspace", "ra_zigzag_permute", "ra_get_device_status",
             "ra_status_string", "ra_version", "ra_ring_attention_noalloc", "ra_noalloc_scratch_bytes",
             "ra_decode_attention", "ra_decode_workspace", "ra_decode_splits", "ra_ring_attention_backward",
@@ -56,6 +56,8 @@ TILINGS = {"auto": 0, "row_pairs": 1, "kv_split": 2, "cluster2": 3}
 _vp, _i, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
 _lib.ra_block_attn.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]
 _lib.ra_block_attn.restype = _i
+_lib.ra_block_attn_merge.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]
+_lib.ra_block_attn_merge.restype = _i
 _lib.ra_merge_partial.argtypes = [_vp, _vp, _vp, _vp, _i64, _i, _vp]
 _lib.ra_merge_partial.restype = _i
 _lib.ra_merge_partials.argtypes = [ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i, _vp, _vp, _i64, _i, _vp]
@@ -158,6 +160,19 @@ def ra_block_attn(q, k, v, S: int, n_blocks: int, q_block: int, kv_block: int, c
                               Hq, Hkv, D, int(bool(causal)), PARTITIONS[partition], _ptr(block_out),
                               _ptr(block_lse), _stream(stream)), "ra_block_attn")
     return block_out, block_lse
+
+
+def ra_block_attn_merge(q, k, v, S: int, n_blocks: int, q_block: int, kv_block: int, causal: bool, out, lse,
+                        partition: str = "contiguous", stream=None):
+    """One query block [B, L, Hq, D] against one KV block [B, L, Hkv, D] (bf16),
+    folded by the merge rule into the running (out fp32 [B, L, Hq, D],
+    lse fp32 [B, L, Hq]) in place.  Start from out = 0, lse = -inf."""
+    B, L, Hq, D = q.shape
+    Hkv = k.shape[2]
+    _check(_lib.ra_block_attn_merge(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q.dtype), B, S, n_blocks, q_block,
+                                    kv_block, Hq, Hkv, D, int(bool(causal)), PARTITIONS[partition], _ptr(out),
+                                    _ptr(lse), _stream(stream)), "ra_block_attn_merge")
+    return out, lse
 
 
 def ra_merge_partial(out, lse, block_out, block_lse, stream=None):

@@ -554,6 +554,37 @@ ra_status ra_block_attn(const void* q, const void* k, const void* v, ra_dtype in
   return launch_attn(D, a, mq, mk, mv, static_cast<cudaStream_t>(stream));
 }
 
+ra_status ra_block_attn_merge(const void* q, const void* k, const void* v, ra_dtype in_dtype, int B, int S,
+                              int n_blocks, int q_block, int kv_block, int Hq, int Hkv, int D, int causal,
+                              ra_partition partition, float* out, float* lse, void* stream) {
+  Geom g;
+  ra_status s = check_geom(B, S, n_blocks, Hq, Hkv, D, partition, &g);
+  if (s != RA_OK) return s;
+  if (in_dtype != RA_BF16) return in_dtype == RA_F32 ? RA_ERR_UNSUPPORTED : RA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out || !lse) return RA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return RA_ERR_INVALID_ARG;
+  if (q_block < 0 || q_block >= n_blocks || kv_block < 0 || kv_block >= n_blocks) return RA_ERR_INVALID_ARG;
+  g.causal = causal != 0;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, D, Hq, g.L, B) || !make_map(&mk, k, D, Hkv, g.L, B) || !make_map(&mv, v, D, Hkv, g.L, B))
+    return RA_ERR_CUDA;
+  AttnArgs a = base_args(g);
+  a.nq = 1;
+  a.nkv = 1;
+  block_segments(g, q_block, true, a.qseg[0]);
+  block_segments(g, kv_block, true, a.kvseg[kv_block]);
+  a.kv_list[0][0] = static_cast<signed char>(kv_block);
+  order_segments(a);
+  choose_tiling(g, a, RA_TILING_AUTO);
+  // the epilogue folds this pair's partial into the running rows (merge rule)
+  a.mode = kModeMerge;
+  a.acc_out = out;
+  a.acc_lse = lse;
+  a.acc_brows = g.L;
+  return launch_attn(D, a, mq, mk, mv, static_cast<cudaStream_t>(stream));
+}
+
 ra_status ra_merge_partial(float* out, float* lse, const float* block_out, const float* block_lse, int64_t rows,
                            int D, void* stream) {
   if (rows < 0 || D <= 0) return RA_ERR_INVALID_ARG;

@@ -143,6 +143,29 @@ ra_status ra_block_attn(const void* q, const void* k, const void* v, ra_dtype in
                         float* block_out, float* block_lse, void* stream);
 
 /*
+ * ra_block_attn_merge - one ring step on one device: the block pair's
+ * partial (as ra_block_attn computes it) folded into a running (out, lse) by
+ * the update rule of ra_merge_partial, inside the attention kernel's
+ * epilogue (the partial never reaches HBM).
+ * [RA] SOTA-181: each device keeps its query block and meets one key/value
+ * block per step; [TR] "What carries the argument": the partials are stitched
+ * by the update rule without recomputation.
+ *  q, k, v, in_dtype, B .. partition   as in ra_block_attn.
+ *  out        device, fp32, [B, L, Hq, D], read and written: the running
+ *             output of query block q_block.  Start from out = 0.
+ *  lse        device, fp32, [B, L, Hq], read and written: the running lse;
+ *             start from lse = -inf (no block merged yet).  A row that sees
+ *             no key of this KV block keeps its (out, lse).
+ * Every pointer must be 16-byte aligned (else RA_ERR_INVALID_ARG).  After
+ * the pairs (q_block, 0 .. n_blocks-1) have all been merged, in any order,
+ * (out, lse) is the block's exact attention up to rounding.
+ */
+ra_status ra_block_attn_merge(const void* q, const void* k, const void* v, ra_dtype in_dtype,
+                              int B, int S, int n_blocks, int q_block, int kv_block,
+                              int Hq, int Hkv, int D, int causal, ra_partition partition,
+                              float* out, float* lse, void* stream);
+
+/*
  * ra_merge_partial - one application of the update rule, in place, fp32.
  * [TR] "What carries the argument":
  *     out <- out - sigma(block_lse - lse) * (out - block_out)

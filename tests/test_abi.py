@@ -86,8 +86,11 @@ def test_ring_attention_rejects_bad_arguments(ra):
     assert ring(ra, opts=ctypes.byref(bad_fault)) == E.RA_ERR_INVALID_ARG
 
 
-def test_block_attn_rejects_bad_arguments(ra):
-    f = ra._lib.ra_block_attn
+@pytest.mark.parametrize("entry", ["ra_block_attn", "ra_block_attn_merge"])
+def test_block_attn_rejects_bad_arguments(ra, entry):
+    # ra_block_attn_merge takes the same arguments, with the running (out, lse)
+    # in place of (block_out, block_lse)
+    f = getattr(ra._lib, entry)
     ok = dict(q=FAKE, k=FAKE, v=FAKE, dt=ra.RA_BF16, B=1, S=1024, n=4, qb=0, kb=0, Hq=4, Hkv=2, D=128, causal=1,
               part=ra.RA_PART_ZIGZAG, bo=FAKE, bl=FAKE)
 
@@ -103,6 +106,8 @@ def test_block_attn_rejects_bad_arguments(ra):
     assert call(Hkv=3) == ra.RA_ERR_INVALID_ARG
     assert call(bo=None) == ra.RA_ERR_INVALID_ARG
     assert call(S=1028) == ra.RA_ERR_INVALID_ARG
+    assert call(bl=FAKE + 4) == ra.RA_ERR_INVALID_ARG
+    assert call(D=96) == ra.RA_ERR_UNSUPPORTED
 
 
 def test_merge_and_permute_reject_bad_arguments(ra):

@@ -252,6 +252,71 @@ def test_block_attn_empty_and_full_pairs(cuda_lib):
     assert seen_empty and seen_full
 
 
+@pytest.mark.parametrize("case", BLOCK_CASES, ids=lambda c: f"B{c[0]}S{c[1]}n{c[2]}H{c[3]}/{c[4]}D{c[5]}{c[7]}{'C' if c[6] else ''}")
+def test_block_attn_merge_folds_every_pair(cuda_lib, case):
+    # every query block folds its n pairs, in a shuffled order, into (0, -inf)
+    # with the fused entry point; the blocks gathered back to original order
+    # are the full attention
+    ra = cuda_lib
+    B, S, n, Hq, Hkv, D, causal, part = case
+    q, k, v = attention_inputs(B, S, Hq, Hkv, D, "bf16", seed=9)
+    perm = K.partition_perm(S, n, part)
+    L = S // n
+    pt = torch.from_numpy(perm)
+    qp, kp, vp = q[:, pt].cuda(), k[:, pt].cuda(), v[:, pt].cuda()
+    out = torch.zeros((B, S, Hq, D), dtype=torch.float32, device="cuda")
+    lse = torch.full((B, S, Hq), float("-inf"), dtype=torch.float32, device="cuda")
+    rng = np.random.default_rng(1)
+    for qb in range(n):
+        rows = slice(qb * L, (qb + 1) * L)
+        o, l = out[:, rows].contiguous(), lse[:, rows].contiguous()
+        for kb in rng.permutation(n):
+            before = (o.clone(), l.clone())
+            kv = slice(int(kb) * L, (int(kb) + 1) * L)
+            ra.ra_block_attn_merge(qp[:, rows].contiguous(), kp[:, kv].contiguous(), vp[:, kv].contiguous(), S, n,
+                                   qb, int(kb), causal, o, l, partition=part)
+            if K.pair_is_empty(perm.reshape(n, L)[qb], perm.reshape(n, L)[kb], causal):
+                # a pair that sees no key leaves the running state untouched, bit for bit
+                assert torch.equal(o, before[0]) and torch.equal(l, before[1])
+        out[:, rows], lse[:, rows] = o, l
+    ro, rl = F.full_attention(q, k, v, causal, Hq // Hkv)
+    assert_close_bf16(K.permute_rows(to_np(out), perm, inverse=True), ro, "folded out")
+    assert_close_bf16(K.permute_rows(to_np(lse), perm, inverse=True), rl, "folded lse")
+    assert ra.ra_get_device_status() == 0
+
+
+@pytest.mark.parametrize("order", ["ring", "tokenring"])
+@pytest.mark.parametrize("case", [(1, 2048, 4, 4, 2, 128, True, "zigzag"), (1, 1024, 4, 2, 1, 64, True, "contiguous"),
+                                  (2, 1200, 3, 2, 2, 128, False, "zigzag")],
+                         ids=lambda c: f"B{c[0]}S{c[1]}n{c[2]}D{c[5]}{c[7]}{'C' if c[6] else ''}")
+def test_ring_shards_lockstep_on_cuda(cuda_lib, case, order):
+    # the sequence-parallel rank programs (one block per rank, K/V or Q and
+    # partials exchanged between ranks) with every rank's device work on the
+    # CUDA kernels, all ranks in one process; gathered, the full attention
+    from blockwise_exact_attention_block_b200 import ring
+    ra = cuda_lib
+    B, S, n, Hq, Hkv, D, causal, part = case
+    q, k, v = attention_inputs(B, S, Hq, Hkv, D, "bf16", seed=10)
+
+    def shard(x, r):
+        return torch.cat([x[:, p:p + l] for p, l in ring.block_segments(S, n, part, r)], dim=1).contiguous().cuda()
+
+    res = ring.ring_attention_lockstep([shard(q, r) for r in range(n)], [shard(k, r) for r in range(n)],
+                                       [shard(v, r) for r in range(n)], S, causal, part, order)
+    out = np.empty((B, S, Hq, D))
+    lse = np.empty((B, S, Hq))
+    for r, (o, l) in enumerate(res):
+        row = 0
+        for p, ln in ring.block_segments(S, n, part, r):
+            out[:, p:p + ln] = to_np(o)[:, row:row + ln]
+            lse[:, p:p + ln] = to_np(l)[:, row:row + ln]
+            row += ln
+    ro, rl = F.full_attention(q, k, v, causal, Hq // Hkv)
+    assert_close_bf16(out, ro, f"ring shards out {order}")
+    assert_close_bf16(lse, rl, f"ring shards lse {order}")
+    assert ra.ra_get_device_status() == 0
+
+
 def test_tiny_workload(cuda_lib):
     # fp32 inputs: the library rounds them to bf16 on entry; the attention is
     # judged against the oracle on the same rounded values.
