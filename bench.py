@@ -18,7 +18,10 @@ same workload on its own GPU (replicas, weak scaling; the method needs no
 exchange on one node here) and the slowest rank's time counts.
 
 --impl reference times the CPU fp64 oracle on the host cores instead (a
-bounded sample of the same workload).
+bounded sample of the same workload).  --backward, --decode, --merge-sweep
+and --shards time the gradient, decode over a KV cache, the merge kernels,
+and the sequence-parallel rank programs (one block per rank, all ranks on
+this GPU) instead.
 """
 from __future__ import annotations
 
@@ -63,6 +66,8 @@ def parse():
     p.add_argument("--backward", action="store_true",
                    help="time the backward pass (ra_ring_attention_backward) on --workload instead")
     p.add_argument("--no-backward", action="store_true")
+    p.add_argument("--shards", action="store_true",
+                   help="time the sequence-parallel rank programs (one block per rank), all ranks on one GPU")
     a = p.parse_args()
     if a.steps is None:
         a.steps = DEFAULT_STEPS[a.workload]
@@ -424,6 +429,144 @@ def run_backward(args):
     return 0 if status == 0 else 1
 
 
+# ------------------------------------------------- sequence-parallel programs
+
+def shard_pairs(n, order, s):
+    """(query block, KV block) each rank computes at step s of the order:
+    ring, s = 0..n-1, rank r meets KV block (r - s) mod n; TokenRing,
+    s = 1..n, rank j computes query block (j - s + 1) mod n on its KV j."""
+    if order == "ring":
+        return [(r, (r - s) % n) for r in range(n)]
+    return [((j - s + 1) % n, j) for j in range(n)]
+
+
+def shard_step_estimate(pair_ms, n, order, merge_ms=0.0):
+    """Per-step compute time with one rank per GPU: the slowest rank's pair
+    (plus, under TokenRing, the merge of the partial it receives).  pair_ms
+    maps (query block, KV block) to the pair's kernel time; a pair absent
+    from it ran nothing (causal skip).  Transfers are assumed to overlap."""
+    steps = range(n) if order == "ring" else range(1, n + 1)
+    out = []
+    for s in steps:
+        worst = 0.0
+        for qb, kb in shard_pairs(n, order, s):
+            t = pair_ms.get((qb, kb), 0.0)
+            if order == "tokenring" and s > 1 and (qb, kb) in pair_ms:
+                t += merge_ms
+            worst = max(worst, t)
+        out.append(worst)
+    return out
+
+
+def shard_exchange_bytes(w, order):
+    """Bytes one rank sends per step: the K/V block (ring), or the Q block
+    plus one fp32 partial, block_out and block_lse (TokenRing)."""
+    L = w.S // w.n_blocks
+    if order == "ring":
+        return 2 * w.B * L * w.Hkv * w.D * 2
+    return w.B * L * w.Hq * w.D * 2 + w.B * L * w.Hq * (w.D + 1) * 4
+
+
+def run_shards(args):
+    """The sequence-parallel rank programs (one block per rank) with every
+    rank on this GPU, messages as device copies.  Reports the whole pass, and
+    an estimate for one rank per GPU from each pair's kernel time."""
+    import torch
+    import blockwise_exact_attention_block_b200 as ra
+    from blockwise_exact_attention_block_b200 import ring
+    if int(os.environ.get("WORLD_SIZE", "1")) != 1:
+        raise SystemExit("--shards runs every rank on one GPU (no torchrun)")
+    w = WORKLOADS[args.workload]
+    if w.in_dtype != "bf16":
+        raise SystemExit("--shards needs a bf16 workload")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    pk, pk_kind = peaks()
+    n = w.n_blocks
+    q, k, v = (x.to(dev) for x in workload_inputs(w))
+
+    def shard(x, r):
+        return torch.cat([x[:, p:p + ln] for p, ln in ring.block_segments(w.S, n, w.partition, r)], dim=1).contiguous()
+
+    qs, ks, vs = ([shard(x, r) for r in range(n)] for x in (q, k, v))
+    del q, k, v
+    stream = torch.cuda.current_stream(dev)
+
+    class TimedOps(ring.BlockOps):
+        record = None
+
+        def _timed(self, key, fn, *a):
+            if self.record is None:
+                return fn(*a)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            ev[0].record(stream)
+            fn(*a)
+            ev[1].record(stream)
+            self.record.append((key, ev))
+
+        def attn_merge(self, qq, kk, vv, qb, kb, out, lse):
+            self._timed((qb, kb), super().attn_merge, qq, kk, vv, qb, kb, out, lse)
+
+        def attn(self, qq, kk, vv, qb, kb, bo, bl):
+            self._timed((qb, kb), super().attn, qq, kk, vv, qb, kb, bo, bl)
+
+        def merge(self, out, lse, bo, bl):
+            self._timed("merge", super().merge, out, lse, bo, bl)
+
+    ops = TimedOps(w.S, n, w.causal, w.partition)
+    clocks = Clocks(local_gpu_id(dev))
+    time.sleep(0.3)
+    passes = []
+    for rep in range(args.warmup + args.steps):
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record(stream)
+        ring.ring_attention_lockstep(qs, ks, vs, w.S, w.causal, w.partition, args.order, ops=ops)
+        ev[1].record(stream)
+        ev[1].synchronize()
+        if rep >= args.warmup:
+            passes.append(ev[0].elapsed_time(ev[1]))
+    # one more pass with events around every kernel, for the per-pair times
+    ops.record = []
+    flush.zero_()
+    ring.ring_attention_lockstep(qs, ks, vs, w.S, w.causal, w.partition, args.order, ops=ops)
+    torch.cuda.synchronize()
+    pair_ms, merges = {}, []
+    for key, ev in ops.record:
+        t = ev[0].elapsed_time(ev[1])
+        if key == "merge":
+            merges.append(t)
+        else:
+            pair_ms[key] = t
+    clk = clocks.stop()
+    status = ra.ra_get_device_status()
+    ms = statistics.median(passes)
+    merge_ms = statistics.mean(merges) if merges else 0.0
+    steps = shard_step_estimate(pair_ms, n, args.order, merge_ms)
+    xbytes = shard_exchange_bytes(w, args.order)
+    nvlink_gbs = 770.0  # measured peer copy per direction on this kind of node
+    launches = len(pair_ms) + len(merges)
+    line = {"metric": "sequence-parallel pass TFLOP/s, all ranks on one GPU", "value": w.flops / (ms * 1e-3) / 1e12,
+            "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded randn, bf16-rounded)",
+            "config": dict(workload_config(w, args, f"flushed ({L2_FLUSH_BYTES >> 20} MiB write between passes)"),
+                           parallelism=f"sequence-parallel {n} ranks, lockstep on one GPU"),
+            "ranks": n, "pair_ms": {f"{a},{b}": t for (a, b), t in sorted(pair_ms.items())},
+            "merge_ms": merge_ms,
+            "one_rank_per_gpu_estimate": {
+                "step_compute_ms": steps, "pass_ms": sum(steps),
+                "TFLOP/s": w.flops / (sum(steps) * 1e-3) / 1e12,
+                "exchange_bytes_per_rank_step": xbytes,
+                "exchange_ms_per_step_at_770GBps": xbytes / (nvlink_gbs * 1e9) * 1e3,
+                "note": "transfers assumed hidden under the step's compute when shorter; not measured across GPUs"},
+            "peak_bf16_tflops": pk["bf16_tflops"], "peak_source": pk_kind, "clocks": clk,
+            "gpu_launches": launches * args.steps, "device_status": ra.ra_status_string(status)}
+    print(json.dumps(line))
+    return 0 if status == 0 else 1
+
+
 def launches_per_step(w, sched):
     """Kernels of ours launched by one ra_ring_attention call."""
     cast = 3 if w.in_dtype == "f32" else 0
@@ -674,6 +817,8 @@ def main():
         return run_decode(args)
     if args.backward:
         return run_backward(args)
+    if args.shards:
+        return run_shards(args)
     return run_ours(args)
 
 

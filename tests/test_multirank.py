@@ -1,4 +1,5 @@
-"""The N > 1 path on the CPU: replicas timed by the slowest rank.
+"""The N > 1 path on the CPU: replicas timed by the slowest rank, and the
+per-step estimate of the sequence-parallel bench mode.
 
 bench.py --gpus N runs one replica of the workload per rank (weak scaling,
 no exchange on the data path); the only collectives are the barrier and the
@@ -78,3 +79,48 @@ def test_reference_arm_under_torchrun_two_ranks():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+# ------------------------------------- sequence-parallel estimate (bench --shards)
+
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 8])
+def test_shard_steps_cover_every_pair_once(n):
+    sys.path.insert(0, ROOT)
+    import bench
+    for order, steps in (("ring", range(n)), ("tokenring", range(1, n + 1))):
+        pairs = [p for s in steps for p in bench.shard_pairs(n, order, s)]
+        assert sorted(pairs) == [(i, j) for i in range(n) for j in range(n)]
+        for s in steps:  # one pair per rank and step: ranks own query blocks (ring) or KV blocks (TokenRing)
+            own = [p[0] if order == "ring" else p[1] for p in bench.shard_pairs(n, order, s)]
+            assert own == list(range(n))
+    if n == 4:
+        assert bench.shard_pairs(n, "ring", 1) == [(0, 3), (1, 0), (2, 1), (3, 2)]
+        assert bench.shard_pairs(n, "tokenring", 2) == [(3, 0), (0, 1), (1, 2), (2, 3)]
+
+
+def test_shard_step_estimate_takes_the_slowest_rank():
+    sys.path.insert(0, ROOT)
+    import bench
+    n = 4
+    # contiguous causal: only pairs kv <= q run; pair time grows with the query block
+    pair_ms = {(i, j): 1.0 + i for i in range(n) for j in range(n) if j <= i}
+    ring = bench.shard_step_estimate(pair_ms, n, "ring")
+    # ring step s: rank r meets KV r - s, visible for r >= s; the slowest is rank 3
+    assert ring == [4.0, 4.0, 4.0, 4.0]
+    tok = bench.shard_step_estimate(pair_ms, n, "tokenring", merge_ms=0.5)
+    # TokenRing step s: rank j computes query block j - s + 1 (mod n); visible when j <= it
+    want = []
+    for s in range(1, n + 1):
+        ts = [1.0 + (j - s + 1) % n + (0.5 if s > 1 else 0.0) for j in range(n) if j <= (j - s + 1) % n]
+        want.append(max(ts, default=0.0))
+    assert tok == want
+    assert bench.shard_step_estimate({}, n, "ring") == [0.0] * n
+
+
+def test_shard_exchange_bytes():
+    sys.path.insert(0, ROOT)
+    import bench
+    from seeded_inputs import WORKLOADS
+    w = WORKLOADS["gqa24k"]  # 24,000 tokens, 4 blocks of 6,000, 32 query / 8 KV heads, D = 128
+    assert bench.shard_exchange_bytes(w, "ring") == 2 * 6000 * 8 * 128 * 2
+    assert bench.shard_exchange_bytes(w, "tokenring") == 6000 * 32 * 128 * 2 + 6000 * 32 * 129 * 4
