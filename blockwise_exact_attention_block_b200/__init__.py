@@ -9,6 +9,10 @@ package fails loudly when the library is missing, and every call raises
 Names follow the C ABI (``ra_block_attn``, ``ra_merge_partial``,
 ``ra_ring_attention`` ...).  Layouts: q/out ``[B, S, Hq, D]``, k/v
 ``[B, S, Hkv, D]``, lse ``[B, S, Hq]``, all contiguous.
+
+``ring`` (a submodule, imported on demand) runs the sequence-parallel form
+across ranks, one block of the sequence per rank, on top of these calls and
+torch.distributed point-to-point messages.
 """
 from __future__ import annotations
 
