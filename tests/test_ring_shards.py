@@ -136,7 +136,7 @@ def test_lockstep_ranks_equal_full_attention(n, order, partition, causal):
     assert sorted(ops.computed) == want
 
 
-@pytest.mark.parametrize("n", [2, 3, 4, 5, 8])
+@pytest.mark.parametrize("n", [2, 3, 4, 5, 8, 16])
 def test_steps_follow_the_pages_order(n):
     # Ring: at step s rank r meets KV block (r - s) mod n, folded in that
     # order.  TokenRing: at step s (1-based) rank j computes query block
@@ -279,5 +279,47 @@ def test_gloo_ranks_equal_full_attention(world, order, partition, causal):
     o = gather([torch.from_numpy(x) for x, _ in res], S, world, partition).numpy()
     l = gather([torch.from_numpy(x) for _, x in res], S, world, partition).numpy()
     ro, rl = F.full_attention(q, k, v, causal, 2)
+    assert np.max(np.abs(o - ro)) <= 1e-12
+    assert np.max(np.abs(l - rl)) <= 1e-12
+
+
+def _subgroup_worker(rank, world, port, out):
+    # a ring over ranks {0, 2} of three: block index = rank inside the group
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        group = dist.new_group([0, 2])
+        if rank in (0, 2):
+            S, n, part = 32, 2, "zigzag"
+            q, k, v = inputs(S)
+            r = dist.get_rank(group)
+            ops = OracleOps(S, n, True, part, 2)
+            o, l = R.ring_attention_dist(shard(q, S, n, part, r), shard(k, S, n, part, r), shard(v, S, n, part, r),
+                                         S, True, part, "tokenring", group=group, ops=ops)
+            out[r] = (o.numpy(), l.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gloo_ring_over_a_subgroup():
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = free_port()
+    procs = [ctx.Process(target=_subgroup_worker, args=(r, 3, port, out)) for r in range(3)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    S, n, part = 32, 2, "zigzag"
+    q, k, v = inputs(S)
+    o = gather([torch.from_numpy(out[r][0]) for r in range(n)], S, n, part).numpy()
+    l = gather([torch.from_numpy(out[r][1]) for r in range(n)], S, n, part).numpy()
+    ro, rl = F.full_attention(q, k, v, True, 2)
     assert np.max(np.abs(o - ro)) <= 1e-12
     assert np.max(np.abs(l - rl)) <= 1e-12
