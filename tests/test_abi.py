@@ -216,3 +216,20 @@ def test_backward_workspace_query(ra):
     assert n32 >= n + 24000 * (32 + 8 + 8 + 32) * 128 * 2
     with pytest.raises(ra.RAError):
         ra.ra_ring_attention_backward_workspace(1, 4095, 8, 128, 4, 1, "zigzag")
+
+
+def test_c_caller_links_and_runs(ra, tmp_path):
+    # the boundary from plain C: include/ra.h, a C compiler and the .so
+    import shutil
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    lib_dir = os.path.dirname(ra.LIB_PATH)
+    exe = str(tmp_path / "c_abi_check")
+    build = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                            os.path.join(ROOT, "tests", "c_abi_check.c"), "-L", lib_dir, "-lra_b200",
+                            f"-Wl,-rpath,{lib_dir}", "-o", exe], capture_output=True, text=True)
+    assert build.returncode == 0, build.stderr
+    run = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, run.stderr
+    assert run.stdout.startswith("ok ")
