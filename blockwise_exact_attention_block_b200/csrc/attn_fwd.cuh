@@ -74,10 +74,6 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kAttnThreads * kRegsL
               "register reallocation must fit in the launch allocation");
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-// 1: exponentials as ex2.approx.f16x2 (two per SFU instruction).
-#ifndef RA_EXP_F16X2
-#define RA_EXP_F16X2 0
-#endif
 
 enum AttnMode : int {
   kModePartial = 0,  // write (block_out, block_lse) into acc rows
@@ -642,13 +638,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 f2_fma(f2_pack(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), sl2x2, nbase2);
             float x0, x1;
             f2_unpack(x2, x0, x1);
-#if RA_EXP_F16X2
-            float q0, q1;
-            exp2_f16x2(x0, x1, q0, q1);
-            const uint64_t e2 = f2_pack(q0, q1);
-#else
             const uint64_t e2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
-#endif
             acc[pp & 3] = f2_add(acc[pp & 3], e2);
             float p0, p1;
             f2_unpack(e2, p0, p1);

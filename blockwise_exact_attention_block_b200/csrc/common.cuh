@@ -338,18 +338,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// 2^x for a pair on the SFU in half precision: both values are rounded to
-// fp16 (11-bit significand), exponentiated by one ex2.approx.f16x2, and
-// widened back to fp32.  Results below 2^-24 flush to 0; x = -inf gives 0.
-__device__ __forceinline__ void exp2_f16x2(float x0, float x1, float& p0, float& p1) {
-  uint32_t h2, e2;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h2) : "f"(x1), "f"(x0));
-  asm("ex2.approx.f16x2 %0, %1;" : "=r"(e2) : "r"(h2));
-  asm("{.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tcvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;}"
-      : "=f"(p0), "=f"(p1)
-      : "r"(e2));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);

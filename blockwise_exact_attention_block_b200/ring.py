@@ -96,12 +96,19 @@ def pair_visible(S: int, n: int, partition: str, causal: bool, q_block: int, kv_
 # ------------------------------------------------------------------- ops
 
 class BlockOps:
-    """Device work of a step on the CUDA library (bf16 inputs, fp32 results)."""
+    """Device work of a step on the CUDA library (bf16 inputs, fp32 results).
 
-    def __init__(self, S: int, n: int, causal: bool, partition: str, stream=None):
+    Every launch goes to torch's current stream.  That is the stream the
+    point-to-point operations of `run_dist` are ordered against (NCCL's own
+    stream waits on it when a step is posted, and it waits on NCCL's stream
+    at each Wait), so a receive never overwrites a buffer that a kernel of an
+    earlier step is still reading.  To run on another stream, make it current
+    (`with torch.cuda.stream(s):`) around the whole program."""
+
+    def __init__(self, S: int, n: int, causal: bool, partition: str):
         from . import ra_block_attn, ra_block_attn_merge, ra_merge_partial
         self._attn, self._attn_merge, self._merge = ra_block_attn, ra_block_attn_merge, ra_merge_partial
-        self.S, self.n, self.causal, self.partition, self.stream = S, n, causal, partition, stream
+        self.S, self.n, self.causal, self.partition = S, n, causal, partition
 
     def new_state(self, q):
         """Running (out, lse) of a query block before any pair: (0, -inf)."""
@@ -119,14 +126,14 @@ class BlockOps:
 
     def attn_merge(self, q, k, v, q_block, kv_block, out, lse):
         self._attn_merge(q, k, v, self.S, self.n, q_block, kv_block, self.causal, out, lse,
-                         partition=self.partition, stream=self.stream)
+                         partition=self.partition)
 
     def attn(self, q, k, v, q_block, kv_block, block_out, block_lse):
         self._attn(q, k, v, self.S, self.n, q_block, kv_block, self.causal, partition=self.partition,
-                   block_out=block_out, block_lse=block_lse, stream=self.stream)
+                   block_out=block_out, block_lse=block_lse)
 
     def merge(self, out, lse, block_out, block_lse):
-        self._merge(out, lse, block_out, block_lse, stream=self.stream)
+        self._merge(out, lse, block_out, block_lse)
 
 
 # -------------------------------------------------------------- programs

@@ -247,7 +247,12 @@ ra_status ra_zigzag_permute(const void* src, void* dst, int B, int S, int H, int
  *    default path (bf16 inputs, persistent schedule) needs none.
  *  - The first call on a device looks up the array's device address on the
  *    current device (cudaGetSymbolAddress); make that first call before any
- *    stream capture.  `stream` must belong to the current device.
+ *    stream capture.  `stream` must belong to the current device.  The
+ *    address is kept per device and per context: after cudaDeviceReset, or
+ *    once the device's primary context has been released and created again,
+ *    the next call looks it up anew (the array may then sit elsewhere).
+ *  - Invalid arguments return the same status as ra_ring_attention would
+ *    (RA_ERR_INVALID_ARG or RA_ERR_UNSUPPORTED), before anything runs.
  *  - Every call on a device shares the one array and it keeps the last call's
  *    contents; nothing in it needs to start at zero (every scratch byte the
  *    call reads it first writes).  Calls whose work overlaps on the GPU (on

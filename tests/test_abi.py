@@ -86,6 +86,28 @@ def test_ring_attention_rejects_bad_arguments(ra):
     assert ring(ra, opts=ctypes.byref(bad_fault)) == E.RA_ERR_INVALID_ARG
 
 
+def noalloc(ra, **kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, in_dtype=ra.RA_BF16, B=1, S=4096, Hq=8, D=128, n=4, causal=1,
+                part=ra.RA_PART_ZIGZAG, groups=1, out=FAKE, out_dtype=ra.RA_F32, lse=FAKE, opts=None, stream=None)
+    args.update(kw)
+    return ra._lib.ra_ring_attention_noalloc(args["q"], args["k"], args["v"], args["in_dtype"], args["B"],
+                                             args["S"], args["Hq"], args["D"], args["n"], args["causal"],
+                                             args["part"], args["groups"], args["out"], args["out_dtype"],
+                                             args["lse"], args["opts"], args["stream"])
+
+
+@pytest.mark.parametrize("kw", [dict(S=4100), dict(groups=3), dict(groups=0), dict(D=96), dict(n=17), dict(n=0),
+                                dict(in_dtype=7), dict(out_dtype=9), dict(part=5), dict(q=None),
+                                dict(out=FAKE + 4), dict(B=0)],
+                         ids=lambda kw: ",".join(f"{k}={v}" for k, v in kw.items()))
+def test_noalloc_returns_the_same_status_as_the_workspace_call(ra, kw):
+    # Invalid arguments never reach the scratch lookup or a launch (no GPU
+    # needed); both entry points must name the same cause.
+    expect = ring(ra, **kw)
+    assert expect in (ra.RA_ERR_INVALID_ARG, ra.RA_ERR_UNSUPPORTED)
+    assert noalloc(ra, **kw) == expect
+
+
 @pytest.mark.parametrize("entry", ["ra_block_attn", "ra_block_attn_merge"])
 def test_block_attn_rejects_bad_arguments(ra, entry):
     # ra_block_attn_merge takes the same arguments, with the running (out, lse)

@@ -348,23 +348,64 @@ def test_identity_pin_catches_merge_mutants(mutant, monkeypatch):
     assert max(np.max(np.abs(bo - out)), np.max(np.abs(bl - lse))) > 1e-6
 
 
-def test_brute_force_pin_catches_transposed_and_unscaled():
-    q, k, v = small(1, 12, 1, 1, 4, seed=17)
-    ref_o, ref_l = brute_attention(q, k, v, True, 1)
-    # transposed score operands (k against q) and a missing 1/sqrt(D)
-    t_o, t_l = F.full_attention(k, q, v, True, 1)
-    u_o, u_l = F.full_attention(q * 2.0, k, v, True, 1)  # = scale 1/sqrt(D) dropped for D=4
-    assert np.max(np.abs(t_o - ref_o)) > 1e-6
-    assert np.max(np.abs(u_l - ref_l)) > 1e-6
+def _planted_full_attention(q, k, v, causal, groups, mistake=None):
+    """A copy of the oracle's full attention, step for step, with one planted
+    mistake: "transposed" (scores from k against q), "unscaled" (the 1/sqrt(D)
+    dropped), "strict_mask" (causal keeps j < i instead of j <= i) or
+    "wrong_group" (query head h reads KV head h % Hkv instead of h // groups).
+    With mistake=None it is the oracle's computation."""
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    scale = 1.0 if mistake == "unscaled" else 1.0 / math.sqrt(D)
+    out = np.zeros((B, S, Hq, D))
+    lse = np.zeros((B, S, Hq))
+    for b in range(B):
+        for h in range(Hq):
+            g = h % Hkv if mistake == "wrong_group" else h // groups
+            kk, vv, qq = k[b, :, g, :], v[b, :, g, :], q[b, :, h, :]
+            s = (kk @ qq.T if mistake == "transposed" else qq @ kk.T) * scale
+            if causal:
+                rows, cols = np.arange(S)[:, None], np.arange(S)[None, :]
+                keep = cols < rows if mistake == "strict_mask" else cols <= rows
+                s = np.where(keep, s, -np.inf)
+            with np.errstate(invalid="ignore"):
+                m = s.max(axis=1, keepdims=True)
+                e = np.exp(s - m)
+                tot = e.sum(axis=1, keepdims=True)
+                lse[b, :, h] = (m + np.log(tot))[:, 0]
+                out[b, :, h, :] = (e / tot) @ vv
+    return out, lse
 
 
-def test_causal_pin_catches_off_by_one_mask():
-    # Strict mask (j < i) instead of (j <= i): the single-key closed form fails.
-    q, k, v = small(1, 6, 1, 1, 4, seed=19)
-    out, _ = F.full_attention(q, k, v, True, 1)
-    shifted = np.concatenate([np.zeros_like(v[:, :1]), v[:, :-1]], axis=1)
-    assert np.max(np.abs(out[0, 0, 0] - v[0, 0, 0])) < TOL
-    assert np.max(np.abs(out[0, 0, 0] - shifted[0, 0, 0])) > 1e-6
+def _pin_holds(got, ref):
+    """The brute-force pin's test; NaN (a row left with no key) fails it."""
+    return bool(np.max(np.abs(got[0] - ref[0])) < TOL and np.max(np.abs(got[1] - ref[1])) < TOL)
+
+
+@pytest.mark.parametrize("mistake", [None, "transposed", "unscaled", "strict_mask", "wrong_group"])
+def test_brute_force_pin_catches_planted_mistakes(mistake):
+    # D = 8 (so a dropped 1/sqrt(D) is not a factor a test input could hide),
+    # 4 query heads over 2 KV heads (so the head grouping matters), causal.
+    q, k, v = small(1, 10, 4, 2, 8, seed=17)
+    ref = brute_attention(q, k, v, True, 2)
+    got = _planted_full_attention(q, k, v, True, 2, mistake)
+    if mistake is None:
+        assert _pin_holds(got, ref)  # the copy itself is faithful
+        assert _pin_holds(got, F.full_attention(q, k, v, True, 2))
+    else:
+        assert not _pin_holds(got, ref), mistake
+
+
+def test_strict_mask_changes_every_causal_row():
+    # The off-by-one mask is caught on every row, not only the first (row 0
+    # is left with no key at all; any later row loses its diagonal term).
+    q, k, v = small(1, 8, 1, 1, 4, seed=19)
+    bo, bl = brute_attention(q, k, v, True, 1)
+    po, pl = _planted_full_attention(q, k, v, True, 1, "strict_mask")
+    with np.errstate(invalid="ignore"):
+        for i in range(1, 8):
+            assert abs(pl[0, i, 0] - bl[0, i, 0]) > 1e-6, i
+    assert not np.isfinite(pl[0, 0, 0])
 
 
 # --------------------------------------------------------- decode (KV cache)

@@ -61,9 +61,16 @@ def test_noalloc_matches_workspace_entry_point(cuda_lib, name, inputs, kw):
     for call in range(2):
         out.fill_(float("nan"))
         lse.fill_(float("nan"))
+        torch.cuda.synchronize()
+        # The second call runs with every module already loaded: neither the
+        # device's free memory nor torch's allocator may move across it.
+        free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
         ra.ra_ring_attention_noalloc(q, k, v, kw["n_blocks"], kw["causal"], kw["partition"], out=out, lse=lse,
                                      sched=kw["sched"])
         torch.cuda.synchronize()
+        if call == 1:
+            assert torch.cuda.mem_get_info()[0] == free0, f"{name}: device free memory changed"
+            assert torch.cuda.memory_allocated() == alloc0, f"{name}: torch allocated memory"
         close(out, ref_o, f"{name} out, call {call}")
         close(lse, ref_l, f"{name} lse, call {call}")
     assert ra.ra_get_device_status() == 0
