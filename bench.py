@@ -38,9 +38,30 @@ sys.path.insert(0, ROOT)
 
 from seeded_inputs import WORKLOADS, workload_inputs  # noqa: E402
 
-DEFAULT_WORKLOAD = "zigzag4k"
-DEFAULT_STEPS = {"tiny": 2000, "zigzag4k": 2000, "gqa24k": 400, "long1m": 3}
+DEFAULT_WORKLOAD = "long1m"
+DEFAULT_STEPS = {"tiny": 2000, "zigzag4k": 2000, "gqa24k": 400, "long1m": 5}
+# Workloads timed beside the headline one on the default line, with the
+# steps each runs there (enough for the clock sampler to see the region).
+SIDE_WORKLOADS = {"zigzag4k": 2000, "gqa24k": 200}
+METRIC = "causal-adj attention TFLOP/s (% of dense bf16 peak)"
 L2_FLUSH_BYTES = 256 << 20
+L2_FLUSH_DESC = (f"flushed between steps: a {L2_FLUSH_BYTES >> 20} MiB write, then that buffer read back, "
+                 f"so no input is L2-resident and L2 holds no dirty lines")
+
+
+class L2Flush:
+    """Evicts the inputs of the last step from L2 (126 MB) between timed
+    steps, outside their events.  A write of a buffer twice the size of L2
+    alone would leave up to 126 MB of dirty lines whose write-back the next
+    timed kernel would pay; reading the buffer back leaves only clean lines."""
+
+    def __init__(self, dev):
+        import torch
+        self.buf = torch.empty(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+
+    def __call__(self):
+        self.buf.zero_()
+        self.buf.sum()
 
 
 def parse():
@@ -66,6 +87,9 @@ def parse():
     p.add_argument("--backward", action="store_true",
                    help="time the backward pass (ra_ring_attention_backward) on --workload instead")
     p.add_argument("--no-backward", action="store_true")
+    p.add_argument("--backward-workload", default="gqa24k", choices=sorted(WORKLOADS),
+                   help="workload of the backward object on the default line")
+    p.add_argument("--no-side", action="store_true", help="time only --workload (no other attention workloads)")
     p.add_argument("--shards", action="store_true",
                    help="time the sequence-parallel rank programs (one block per rank), all ranks on one GPU")
     a = p.parse_args()
@@ -93,29 +117,88 @@ def workload_config(w, args, l2):
 
 # ------------------------------------------------------------- CPU oracle
 
-def oracle_sample(w, budget_s: float = 15.0):
-    """Times the oracle's blockwise path (the method in fp64) on a bounded
-    sample: the first h query heads (with their KV heads) of batch 0."""
-    import numpy as np  # noqa: F401
-    from oracle import blockwise as K
-    from seeded_inputs import attention_inputs
-    q, k, v = workload_inputs(w) if w.S <= 24000 else attention_inputs(1, 32768, w.Hq, w.Hkv, w.D, w.in_dtype, 0)
-    S = q.shape[1]
-    n = w.n_blocks
-    g = w.gqa_groups
-    flops_head = 4.0 * w.D * (S * (S + 1) // 2 if w.causal else S * S)
-    t0 = time.perf_counter()
-    K.blockwise_attention(q[:1, :, :1], k[:1, :, :1], v[:1, :, :1], n, w.causal, w.partition, 1)
-    t1 = time.perf_counter() - t0
-    heads = max(1, min(w.Hq, int(budget_s / max(t1, 1e-3)) - 1))
-    t0 = time.perf_counter()
-    nkv = (heads + g - 1) // g
-    K.blockwise_attention(q[:1, :, :heads], k[:1, :, :nkv], v[:1, :, :nkv], n, w.causal, w.partition, g)
-    dt = time.perf_counter() - t0
-    cores = len(os.sched_getaffinity(0))
-    sample = (f"oracle blockwise path (fp64 NumPy) on batch 0, query heads 0..{heads - 1} of {w.Hq}, "
-              f"S={S}" + ("" if S == w.S else f" (sequence shortened from {w.S})"))
-    return flops_head * heads / dt / 1e12, cores, sample, dt
+def blas_threads(n=None):
+    """Pins the oracle's BLAS (OpenBLAS under NumPy) to n threads (default:
+    every core this process may run on) and returns (context, n).  The
+    count is what the baseline reports as `cores`."""
+    import numpy as np  # noqa: F401  (loads the BLAS library threadpoolctl controls)
+    from threadpoolctl import threadpool_limits
+    n = n or len(os.sched_getaffinity(0))
+    return threadpool_limits(limits=n, user_api="blas"), n
+
+
+def sample_rows(w, count, seed=0):
+    """`count` seeded (batch, position, query head) rows of workload w, drawn
+    uniformly over positions and heads (the first and the last position
+    always included)."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    pos = rng.integers(0, w.S, size=count)
+    pos[0], pos[-1] = 0, w.S - 1
+    heads = rng.integers(0, w.Hq, size=count)
+    return [(0, int(i), int(h)) for i, h in zip(pos, heads)]
+
+
+def rows_flops(w, rows):
+    """Causal-adjusted FLOPs of the given query rows: 4 * D per visible key."""
+    return sum(4.0 * w.D * ((i + 1) if w.causal else w.S) for _, i, _ in rows)
+
+
+def oracle_f_sample(w, inputs, budget_s=15.0, threads=None, count=None):
+    """Times the oracle's plain path F (full softmax attention in fp64, the
+    definition the method reproduces) on a bounded sample of workload w, with
+    the BLAS pinned to `threads` threads.  Up to 24,000 tokens the sample is
+    the first h query heads of batch 0 in full, h sized to the budget from a
+    first one-head run; beyond that it is a seeded set of query rows, each
+    computed against every key it sees (oracle.attention.attention_rows):
+    `count` rows, or as many as the budget allows after an 8-row probe (at
+    least 64).  Returns (TFLOP/s, threads, sample description, seconds,
+    rows or heads sampled)."""
+    from oracle import attention as F
+    q, k, v = inputs
+    ctx, n = blas_threads(threads)
+    with ctx:
+        if w.S <= 24000:
+            g = w.gqa_groups
+            per_head = w.flops / (w.B * w.Hq)
+            t0 = time.perf_counter()
+            F.full_attention(q[:1, :, :1], k[:1, :, :1], v[:1, :, :1], w.causal, 1)
+            t1 = time.perf_counter() - t0
+            heads = max(1, min(w.Hq, int(budget_s / max(t1, 1e-3))))
+            nkv = (heads + g - 1) // g
+            t0 = time.perf_counter()
+            F.full_attention(q[:1, :, :heads], k[:1, :, :nkv], v[:1, :, :nkv], w.causal, g)
+            dt = time.perf_counter() - t0
+            return (per_head * heads / dt / 1e12, n,
+                    f"oracle path F (plain fp64 attention, NumPy) on batch 0, query heads 0..{heads - 1} of {w.Hq}, "
+                    f"all {w.S} rows", dt, heads)
+        if count is None:
+            probe = sample_rows(w, 8, seed=1)
+            t0 = time.perf_counter()
+            F.attention_rows(q, k, v, probe, w.causal, w.gqa_groups)
+            t1 = time.perf_counter() - t0
+            count = int(max(64, min(4096, 8 * budget_s / max(t1, 1e-3))))
+        rows = sample_rows(w, count, seed=2)
+        t0 = time.perf_counter()
+        F.attention_rows(q, k, v, rows, w.causal, w.gqa_groups)
+        dt = time.perf_counter() - t0
+        return (rows_flops(w, rows) / dt / 1e12, n,
+                f"oracle path F rows (plain fp64 attention per query row, NumPy): {count} seeded rows of batch 0 "
+                f"over all positions and query heads, each against every key it sees", dt, count)
+
+
+def cpu_baseline(w, inputs, budget_s=15.0):
+    """The `cpu_baseline` object: path F on every core of this process, and
+    a per-core figure (path F, one BLAS thread, one head of the 4k zigzag
+    workload)."""
+    v_, n, sample, dt, _ = oracle_f_sample(w, inputs, budget_s)
+    w4 = WORKLOADS["zigzag4k"]
+    one = workload_inputs(w4) if w.name != "zigzag4k" else inputs
+    v1, _, s1, dt1, _ = oracle_f_sample(w4, one, budget_s=0.0, threads=1)
+    return {"value": v_, "unit": "TFLOP/s", "cores": n, "kind": "oracle", "sample": sample, "seconds": dt,
+            "blas_threads": n,
+            "per_core": {"value": v1, "unit": "TFLOP/s", "cores": 1, "workload": "zigzag4k", "sample": s1,
+                         "seconds": dt1}}
 
 
 def run_reference(args):
@@ -123,19 +206,26 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = WORKLOADS[args.workload]
+    inputs = workload_inputs(w)
     per_step = []
     budget = max(1.0, 120.0 / max(args.steps + args.warmup, 1))
+    row_mode = w.S > 24000
     for _ in range(args.warmup):  # untimed
-        oracle_sample(w, budget_s=0.0)
+        oracle_f_sample(w, inputs, budget_s=0.0, count=8 if row_mode else None)
+    cores, sample, count = None, None, None
     for _ in range(args.steps):
-        v, cores, sample, dt = oracle_sample(w, budget_s=budget)
+        # every step samples the same amount: the first step sizes it
+        v, cores, sample, dt, got = oracle_f_sample(w, inputs, budget_s=budget, count=count)
+        if row_mode:
+            count = got
         per_step.append(v)
     value = statistics.median(per_step)
-    line = {"impl": "reference", "metric": "causal-adj attention TFLOP/s (% of dense bf16 peak)", "value": value,
+    line = {"impl": "reference", "metric": METRIC, "value": value,
             "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded randn, bf16-rounded)", "config": workload_config(w, args, "n/a (CPU)"),
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample,
+                             "blas_threads": cores},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
     return 0
@@ -205,16 +295,16 @@ def kernel_sha(files=FWD_SOURCES):
 
 
 def attn_traffic(workload, record="attn_fwd_traffic.json", files=FWD_SOURCES):
-    """DRAM bytes per launch (per call for the backward's two kernels) from the
-    committed ncu capture, or None when there is none for this workload or the
-    kernel sources changed since."""
+    """The committed ncu record of this workload: DRAM bytes per launch (per
+    call for the backward's two kernels) and a note on what they count; None
+    when there is none for this workload or the kernel sources changed since."""
     path = os.path.join(ROOT, "profiles", record)
     if not os.path.exists(path):
         return None
     rec = json.load(open(path)).get(workload)
     if not rec or rec.get("kernel_sha") != kernel_sha(files):
         return None
-    return rec["dram_bytes_per_launch"]
+    return rec
 
 
 # ------------------------------------------------------------- multi-rank
@@ -240,41 +330,54 @@ def replica_throughput(flops_per_step: float, world: int, steps: int, max_ms: fl
 
 # ------------------------------------------------------------ merge kernels
 
+MERGE_HBM_BUDGET = 140 << 30  # device bytes the k-way sweep may hold in partials
+
+
 def bench_merge(ra, dev, T, k, reps, flush, kway=False):
     """GB/s of merging k partials of [T, 32, 128] fp32 (+ lse [T, 32]).
 
-    Pairwise: k-1 ra_merge_partial calls, 12*D+12 bytes per row each.
-    k-way: one ra_merge_partials call, (k+1)*(4*D+4) bytes per row.
-    At most 4 distinct partial buffers are allocated and cycled (16 partials
-    of 16 GiB do not fit in HBM); the bytes moved per merge are unchanged."""
+    Pairwise: k-1 ra_merge_partial launches into one accumulator, 12*D+12
+    bytes per row each; every launch is timed on its own, after an L2 flush,
+    and the GB/s is that of the median launch (the bytes of one launch do not
+    depend on k).  The partials cycle through at most 4 buffers: each launch
+    reads one of them once, so nothing it reads was left in L2 by the launch
+    before.
+    k-way: one ra_merge_partials call over k distinct partial buffers (a
+    repeated buffer inside one call would be read from L2, since the kernel
+    reads every partial of a row together), (k+1)*(4*D+4) bytes per row.
+    Returns (GB/s, ms), or (None, None) when k distinct partials of this size
+    do not fit in the device memory set aside for them."""
     import torch
     H, D = 32, 128
     rows = T * H
-    nb = min(max(k - 1, 1), 4) if not kway else min(k, 4)
+    part_bytes = rows * (D + 1) * 4
+    if kway and k * part_bytes > MERGE_HBM_BUDGET:
+        return None, None
+    nb = k if kway else min(max(k - 1, 1), 4)
     g = torch.Generator(device=dev).manual_seed(1)
     out = torch.randn((T, H, D), device=dev, generator=g)
     lse = torch.rand((T, H), device=dev, generator=g) * 20 - 5
-    bos = [torch.randn((T, H, D), device=dev, generator=g) for _ in range(nb)]
-    bls = [torch.rand((T, H), device=dev, generator=g) * 20 - 5 for _ in range(nb)]
+    n_extra = k - 1 if kway else nb
+    bos = [torch.randn((T, H, D), device=dev, generator=g) for _ in range(n_extra)]
+    bls = [torch.rand((T, H), device=dev, generator=g) * 20 - 5 for _ in range(n_extra)]
     stream = torch.cuda.current_stream(dev)
     times = []
     for rep in range(reps + 2):
-        if rows * (D + 1) * 4 * 2 < 4 * (256 << 20):
-            flush.zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        if kway:
-            ra.ra_merge_partials([out] + [bos[j % nb] for j in range(k - 1)],
-                                 [lse] + [bls[j % nb] for j in range(k - 1)], out=out, lse=lse)
-        else:
-            for j in range(k - 1):
+        launches = [None] if kway else list(range(k - 1))
+        for j in launches:
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            if kway:
+                ra.ra_merge_partials([out] + bos, [lse] + bls, out=out, lse=lse)
+            else:
                 ra.ra_merge_partial(out, lse, bos[j % nb], bls[j % nb])
-        e1.record(stream)
-        e1.synchronize()
-        if rep >= 2:
-            times.append(e0.elapsed_time(e1))
+            e1.record(stream)
+            e1.synchronize()
+            if rep >= 2:
+                times.append(e0.elapsed_time(e1))
     ms = statistics.median(times)
-    nbytes = rows * ((k + 1) * (4 * D + 4) if kway else (k - 1) * (12 * D + 12))
+    nbytes = rows * ((k + 1) * (4 * D + 4) if kway else (12 * D + 12))
     del out, lse, bos, bls
     torch.cuda.empty_cache()
     return nbytes / (ms * 1e-3) / 1e9, ms
@@ -301,7 +404,7 @@ def bench_decode(ra, dev, w, reps, flush):
     stream = torch.cuda.current_stream(dev)
     times = []
     for rep in range(reps + 3):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         ra.ra_decode_attention(q, k, v, w.causal, 0, out=out, lse=lse, workspace=ws)
@@ -322,7 +425,7 @@ def run_decode(args):
     from seeded_inputs import DECODE_WORKLOADS
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     pk, pk_kind = peaks()
     lines = []
     clocks = Clocks(local_gpu_id(dev))
@@ -338,7 +441,7 @@ def run_decode(args):
                 "dtype": "bf16", "data": "synthetic (device randn, bf16-rounded)",
                 "config": {"workload": name, "B": w.B, "Tq": w.Tq, "Skv": w.Skv, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
                            "causal": w.causal, "chunks": splits, "bytes_per_call": w.bytes,
-                           "l2": f"flushed ({L2_FLUSH_BYTES >> 20} MiB write between calls)"},
+                           "l2": L2_FLUSH_DESC},
                 "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                              "frac": gbs / pk["hbm_gbs"], "traffic": None, "kernel": "decode_partial_kernel",
                              "peak_source": f"{pk_kind} copy bandwidth"},
@@ -380,7 +483,7 @@ def bench_backward(ra, dev, w, reps, flush, order="ring"):
     # library records around them) in a second pass
     for timed, out_list in ((False, call), (True, kern)):
         for rep in range(reps + 3):
-            flush.zero_()
+            flush()
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
             if timed:
                 one(tuple(ev))
@@ -403,7 +506,7 @@ def run_backward(args):
     import blockwise_exact_attention_block_b200 as ra
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     w = WORKLOADS[args.workload]
     pk, pk_kind = peaks()
     clocks = Clocks(local_gpu_id(dev))
@@ -417,10 +520,11 @@ def run_backward(args):
     line = {"metric": "backward causal-adj TFLOP/s (2.5x forward FLOPs)", "value": tf, "unit": "TFLOP/s",
             "n_gpus": 1, "steps": reps, "warmup": 3, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded randn, bf16-rounded)",
-            "config": dict(workload_config(w, args, f"flushed ({L2_FLUSH_BYTES >> 20} MiB write between calls)"),
+            "config": dict(workload_config(w, args, L2_FLUSH_DESC),
                            flops_per_step=2.5 * w.flops),
             "roofline": {"bound": "tensor", "achieved": ktf, "peak": peak, "unit": "TFLOP/s", "frac": ktf / peak,
-                         "traffic": attn_traffic(w.name, "attn_bwd_traffic.json", BWD_SOURCES),
+                         "traffic": (attn_traffic(w.name, "attn_bwd_traffic.json", BWD_SOURCES) or {}).get(
+                             "dram_bytes_per_launch"),
                          "kernel": "bwd_dkv_kernel + bwd_dq_kernel",
                          "peak_source": f"{pk_kind} {'sustained' if sustained else 'burst'} bf16 dense"},
             "kernels_ms": kms, "clocks": clk, "gpu_launches": reps * (3 if w.in_dtype == "bf16" else 7),
@@ -481,7 +585,7 @@ def run_shards(args):
         raise SystemExit("--shards needs a bf16 workload")
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     pk, pk_kind = peaks()
     n = w.n_blocks
     q, k, v = (x.to(dev) for x in workload_inputs(w))
@@ -519,7 +623,7 @@ def run_shards(args):
     time.sleep(0.3)
     passes = []
     for rep in range(args.warmup + args.steps):
-        flush.zero_()
+        flush()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         ev[0].record(stream)
         ring.ring_attention_lockstep(qs, ks, vs, w.S, w.causal, w.partition, args.order, ops=ops)
@@ -529,7 +633,7 @@ def run_shards(args):
             passes.append(ev[0].elapsed_time(ev[1]))
     # one more pass with events around every kernel, for the per-pair times
     ops.record = []
-    flush.zero_()
+    flush()
     ring.ring_attention_lockstep(qs, ks, vs, w.S, w.causal, w.partition, args.order, ops=ops)
     torch.cuda.synchronize()
     pair_ms, merges = {}, []
@@ -551,7 +655,7 @@ def run_shards(args):
             "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded randn, bf16-rounded)",
-            "config": dict(workload_config(w, args, f"flushed ({L2_FLUSH_BYTES >> 20} MiB write between passes)"),
+            "config": dict(workload_config(w, args, L2_FLUSH_DESC),
                            parallelism=f"sequence-parallel {n} ranks, lockstep on one GPU"),
             "ranks": n, "pair_ms": {f"{a},{b}": t for (a, b), t in sorted(pair_ms.items())},
             "merge_ms": merge_ms,
@@ -578,6 +682,158 @@ def launches_per_step(w, sched):
     return cast + w.n_blocks + (w.n_blocks - 1) + out_cast
 
 
+def forward_roofline(w, attn_ms, pk, pk_kind):
+    """Roofline object of the attention kernel: achieved = the workload's
+    causal-adjusted FLOPs over the kernel's mean launch time, against the
+    measured dense bf16 peak (the sustained figure for launches over 100 ms,
+    the burst one otherwise)."""
+    sustained = attn_ms > 100.0
+    peak = pk["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    achieved = w.flops / (attn_ms * 1e-3) / 1e12
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": None, "kernel": "attn_fwd_kernel",
+            "peak_source": f"{pk_kind} {'sustained' if sustained else 'burst'} bf16 dense"}
+    rec = attn_traffic(w.name)
+    if rec is not None:
+        roof["traffic"] = rec["dram_bytes_per_launch"]
+        if rec.get("note"):
+            roof["traffic_note"] = rec["note"]
+    return roof
+
+
+def time_forward(ra, dev, w, args, steps, warmup, flush, world, inputs=None):
+    """Times `steps` ra_ring_attention calls on workload w, inputs resident in
+    HBM, L2 flushed between calls (outside the events).  Returns a dict with
+    the per-step device times, the slowest rank's total, the attention
+    kernel's mean time, the clocks seen, and the device tensors."""
+    import torch
+    import torch.distributed as dist
+    q_h, k_h, v_h = inputs if inputs is not None else workload_inputs(w)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    odt = torch.bfloat16 if w.out_dtype == "bf16" else torch.float32
+    out = torch.empty((w.B, w.S, w.Hq, w.D), dtype=odt, device=dev)
+    lse = torch.empty((w.B, w.S, w.Hq), dtype=torch.float32, device=dev)
+    need = ra.ra_ring_attention_workspace(w.B, w.S, w.Hq, w.D, w.n_blocks, w.gqa_groups, w.partition, q.dtype,
+                                          args.order, args.sched, odt)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(events=None):
+        ra.ra_ring_attention(q, k, v, w.n_blocks, w.causal, w.partition, w.gqa_groups, out=out, lse=lse,
+                             workspace=ws, order=args.order, sched=args.sched, attn_events=events,
+                             tiling=args.tiling)
+
+    for _ in range(warmup):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    if ra.ra_get_device_status() != 0:
+        raise SystemExit(f"{w.name}: device status not OK after warm-up")
+    # The timed steps carry only their bracketing events (events the library
+    # records inside the call cost about 10 us of GPU time per step).
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = Clocks(local_gpu_id(dev))
+    time.sleep(0.3)
+    for i in range(steps):
+        flush()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = max_over_ranks(sum(step_ms), dev)
+    one_launch = args.sched in ("auto", "persistent") and w.in_dtype == "bf16"
+    if one_launch:
+        # the call is the one attention launch: the step events time it
+        attn_ms = statistics.mean(step_ms)
+    else:
+        # the attention launches alone: events the library records around them
+        Ka = min(steps, 200)
+        av = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ka)]
+        for i in range(Ka):
+            flush()
+            step(av[i])
+        torch.cuda.synchronize()
+        attn_ms = statistics.mean(a.elapsed_time(b) for a, b in av)
+    status = ra.ra_get_device_status()
+    return {"step_ms": step_ms, "total_ms": total_ms, "attn_ms": attn_ms, "clocks": clk, "status": status,
+            "tensors": (q, k, v, out, lse, ws), "host": (q_h, k_h, v_h), "stream": stream}
+
+
+def time_e2e(ra, dev, w, args, fw, steps, world):
+    """The same call end to end through the public API with host buffers:
+    every step copies its Q, K, V from pinned host memory, makes the call
+    and reads out and lse back.  Two sets of device buffers and three streams
+    let step i+1's upload, step i's call and step i-1's download overlap
+    (PCIe is full duplex), as a caller streaming batches through the library
+    would."""
+    import torch
+    import torch.distributed as dist
+    q, k, v, out, lse, ws = fw["tensors"]
+    q_h, k_h, v_h = fw["host"]
+    stream = fw["stream"]
+    qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+    bufs = [(q, k, v, out, lse, ws),
+            (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(out),
+             torch.empty_like(lse), torch.empty_like(ws))]
+    host_out = [(torch.empty(out.shape, dtype=out.dtype).pin_memory(),
+                 torch.empty(lse.shape, dtype=lse.dtype).pin_memory()) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def e2e_steps(n, e_begin=None, e_end=None):
+        ev_c, ev_o = [], []
+        if e_begin is not None:
+            e_begin.record(s_in)
+        for i in range(n):
+            qd, kd, vd, od, ld, wd = bufs[i % 2]
+            if i >= 2:
+                s_in.wait_event(ev_c[i - 2])  # step i-2's call has read these inputs
+            with torch.cuda.stream(s_in):
+                qd.copy_(qp, non_blocking=True)
+                kd.copy_(kp, non_blocking=True)
+                vd.copy_(vp, non_blocking=True)
+            e_in = torch.cuda.Event()
+            e_in.record(s_in)
+            stream.wait_event(e_in)
+            if i >= 2:
+                stream.wait_event(ev_o[i - 2])  # step i-2's results are on the host
+            ra.ra_ring_attention(qd, kd, vd, w.n_blocks, w.causal, w.partition, w.gqa_groups, out=od, lse=ld,
+                                 workspace=wd, order=args.order, sched=args.sched, tiling=args.tiling,
+                                 stream=stream)
+            ev_c.append(torch.cuda.Event())
+            ev_c[-1].record(stream)
+            s_out.wait_event(ev_c[-1])
+            with torch.cuda.stream(s_out):
+                host_out[i % 2][0].copy_(od, non_blocking=True)
+                host_out[i % 2][1].copy_(ld, non_blocking=True)
+            ev_o.append(torch.cuda.Event())
+            ev_o[-1].record(s_out)
+        if e_end is not None:
+            e_end.record(s_out)
+
+    e2e_steps(3)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e2e_steps(steps, e0, e1)
+    torch.cuda.synchronize()
+    e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
+    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+    del bufs, host_out, qp, kp, vp
+    return {"value": replica_throughput(w.flops, world, steps, e_ms), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps, "warmup": 3,
+            "ms_per_step": e_ms / steps,
+            "pipelining": "uploads, calls and downloads on three streams, two buffer sets"}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -590,146 +846,53 @@ def run_ours(args):
     torch.cuda.set_device(local)
     if world > 1:
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
     import blockwise_exact_attention_block_b200 as ra
 
     w = WORKLOADS[args.workload]
     dev = torch.device("cuda", local)
-    q_h, k_h, v_h = workload_inputs(w)
-    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
-    odt = torch.bfloat16 if w.out_dtype == "bf16" else torch.float32
-    out = torch.empty((w.B, w.S, w.Hq, w.D), dtype=odt, device=dev)
-    lse = torch.empty((w.B, w.S, w.Hq), dtype=torch.float32, device=dev)
-    need = ra.ra_ring_attention_workspace(w.B, w.S, w.Hq, w.D, w.n_blocks, w.gqa_groups, w.partition, q.dtype,
-                                          args.order, args.sched, odt)
-    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
-    stream = torch.cuda.current_stream(dev)
-
-    def step(events=None):
-        ra.ra_ring_attention(q, k, v, w.n_blocks, w.causal, w.partition, w.gqa_groups, out=out, lse=lse,
-                             workspace=ws, order=args.order, sched=args.sched, attn_events=events,
-                             tiling=args.tiling)
-
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    if ra.ra_get_device_status() != 0:
-        raise SystemExit("device status not OK after warm-up")
-
-    # The timed steps: only the bracketing events on the stream (events the
-    # library records inside the call cost about 10 us of GPU time per step,
-    # so the kernel-only timing is a separate pass below).
+    l2 = f"{L2_FLUSH_DESC} (L2 {l2_bytes >> 20} MiB)"
+    pk, pk_kind = peaks()
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    clocks = Clocks(local_gpu_id(dev))
-    time.sleep(0.3)
-    for i in range(K):
-        flush.zero_()
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clk = clocks.stop()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = max_over_ranks(sum(step_ms), dev)
-    # The attention kernel(s) alone: events the library records around its
-    # block-attention launches, over up to 200 more steps.  With the
-    # persistent schedule a step is that one launch, and the step events
-    # above already time it.
-    Ka = min(K, 200)
-    av = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ka)]
-    for i in range(Ka):
-        flush.zero_()
-        step(av[i])
-    torch.cuda.synchronize()
-    attn_ms = [a.elapsed_time(b) for a, b in av]
-    status = ra.ra_get_device_status()
 
-    # end to end through the public call with host buffers: every step copies
-    # its Q, K, V from pinned host memory, makes the call and reads out and lse
-    # back.  Two sets of device buffers and three streams let step i+1's
-    # upload, step i's call and step i-1's download overlap (PCIe is full
-    # duplex), as a caller streaming batches through the library would.
+    fw = time_forward(ra, dev, w, args, K, args.warmup, flush, world)
+    status = fw["status"]
+    roof = forward_roofline(w, fw["attn_ms"], pk, pk_kind)
     e2e = None
     if not args.no_e2e:
-        qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
-        Ke = max(3, min(K, 200))
-        bufs = [(q, k, v, out, lse, ws),
-                (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(out),
-                 torch.empty_like(lse), torch.empty_like(ws))]
-        host_out = [(torch.empty(out.shape, dtype=out.dtype).pin_memory(),
-                     torch.empty(lse.shape, dtype=lse.dtype).pin_memory()) for _ in range(2)]
-        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-
-        def e2e_steps(n, e_begin=None, e_end=None):
-            ev_c, ev_o = [], []
-            if e_begin is not None:
-                e_begin.record(s_in)
-            for i in range(n):
-                qd, kd, vd, od, ld, wd = bufs[i % 2]
-                if i >= 2:
-                    s_in.wait_event(ev_c[i - 2])  # step i-2's call has read these inputs
-                with torch.cuda.stream(s_in):
-                    qd.copy_(qp, non_blocking=True)
-                    kd.copy_(kp, non_blocking=True)
-                    vd.copy_(vp, non_blocking=True)
-                e_in = torch.cuda.Event()
-                e_in.record(s_in)
-                stream.wait_event(e_in)
-                if i >= 2:
-                    stream.wait_event(ev_o[i - 2])  # step i-2's results are on the host
-                ra.ra_ring_attention(qd, kd, vd, w.n_blocks, w.causal, w.partition, w.gqa_groups, out=od, lse=ld,
-                                     workspace=wd, order=args.order, sched=args.sched, tiling=args.tiling,
-                                     stream=stream)
-                ev_c.append(torch.cuda.Event())
-                ev_c[-1].record(stream)
-                s_out.wait_event(ev_c[-1])
-                with torch.cuda.stream(s_out):
-                    host_out[i % 2][0].copy_(od, non_blocking=True)
-                    host_out[i % 2][1].copy_(ld, non_blocking=True)
-                ev_o.append(torch.cuda.Event())
-                ev_o[-1].record(s_out)
-            if e_end is not None:
-                e_end.record(s_out)
-
-        e2e_steps(3)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            dist.barrier()
-        e2e_steps(Ke, e0, e1)
-        torch.cuda.synchronize()
-        e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
-        h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
-        d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
-        e2e = {"value": replica_throughput(w.flops, world, Ke, e_ms), "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke,
-               "pipelining": "uploads, calls and downloads on three streams, two buffer sets"}
-
-    pk, pk_kind = peaks()
-    one_launch = args.sched in ("auto", "persistent") and w.in_dtype == "bf16"
-    attn_mean = statistics.mean(step_ms) if one_launch else statistics.mean(attn_ms)
-    sustained = attn_mean > 100.0
-    peak = pk["bf16_tflops_sustained" if sustained else "bf16_tflops"]
-    achieved = w.flops / (attn_mean * 1e-3) / 1e12
-    traffic = attn_traffic(w.name)
-    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-            "traffic": traffic, "kernel": "attn_fwd_kernel",
-            "peak_source": f"{pk_kind} {'sustained' if sustained else 'burst'} bf16 dense"}
+        # long calls: a few steps are enough for the pipeline's steady state
+        Ke = max(3, min(K, 200 if fw["attn_ms"] < 100.0 else 3))
+        e2e = time_e2e(ra, dev, w, args, fw, Ke, world)
+    host = fw["host"]
+    total_ms, attn_ms, clk = fw["total_ms"], fw["attn_ms"], fw["clocks"]
+    del fw
+    torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v_, cores, sample, _ = oracle_sample(w)
-        cpu = {"value": v_, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample}
+        cpu = cpu_baseline(w, host)
+    del host
+
+    # The other attention workloads, each timed the same way (its own steps,
+    # warm-up, clocks and roofline).
+    side = {}
+    if not args.no_side:
+        for name, steps in SIDE_WORKLOADS.items():
+            if name == w.name:
+                continue
+            ws_ = WORKLOADS[name]
+            r = time_forward(ra, dev, ws_, args, steps, 5, flush, world)
+            status = status or r["status"]
+            side[name] = {"value": replica_throughput(ws_.flops, world, steps, r["total_ms"]), "unit": "TFLOP/s",
+                          "ms_per_step": r["total_ms"] / steps, "steps": steps, "warmup": 5,
+                          "config": workload_config(ws_, args, l2),
+                          "roofline": forward_roofline(ws_, r["attn_ms"], pk, pk_kind), "clocks": r["clocks"],
+                          "gpu_launches": steps * launches_per_step(ws_, args.sched)}
+            del r
+            torch.cuda.empty_cache()
 
     merge = None
     if not args.no_merge:
@@ -749,24 +912,24 @@ def run_ours(args):
 
     backward = None
     if not args.no_backward and world == 1:
-        tf, ktf, bms, bkms = bench_backward(ra, dev, w, 20 if w.S <= 32768 else 2, flush, args.order)
+        bw = WORKLOADS[args.backward_workload]
+        tf, ktf, bms, bkms = bench_backward(ra, dev, bw, 20 if bw.S <= 32768 else 2, flush, args.order)
         bpeak = pk["bf16_tflops_sustained" if bkms > 100.0 else "bf16_tflops"]
+        brec = attn_traffic(bw.name, "attn_bwd_traffic.json", BWD_SOURCES)
         backward = {"kernel": "bwd_dkv_kernel + bwd_dq_kernel (+ bwd_prep_kernel in the call)",
-                    "workload": w.name, "flops_per_step": 2.5 * w.flops, "TFLOP/s": tf, "kernels_TFLOP/s": ktf,
+                    "workload": bw.name, "flops_per_step": 2.5 * bw.flops, "TFLOP/s": tf, "kernels_TFLOP/s": ktf,
                     "ms": bms, "kernels_ms": bkms, "peak_TFLOP/s": bpeak, "frac": ktf / bpeak,
-                    "traffic": attn_traffic(w.name, "attn_bwd_traffic.json", BWD_SOURCES)}
+                    "traffic": brec["dram_bytes_per_launch"] if brec else None}
+    status = status or ra.ra_get_device_status()
 
     value = replica_throughput(w.flops, world, K, total_ms)
-    line = {"metric": "causal-adj attention TFLOP/s (% of dense bf16 peak)", "value": value, "unit": "TFLOP/s",
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded randn, bf16-rounded)",
-            "config": workload_config(w, args, f"flushed ({L2_FLUSH_BYTES >> 20} MiB write between steps, "
-                                               f"L2 {l2_bytes >> 20} MiB)"),
-            "pct_of_peak": 100.0 * value / peak, "attn_kernel_ms": attn_mean,
-            "attn_kernel_ms_inner_events": statistics.mean(attn_ms), "roofline": roof,
+            "data": "synthetic (seeded randn, bf16-rounded)", "config": workload_config(w, args, l2),
+            "pct_of_peak": 100.0 * roof["frac"], "attn_kernel_ms": attn_ms, "roofline": roof,
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "gpu_launches": K * launches_per_step(w, args.sched),
-            "merge": merge, "decode": decode, "backward": backward,
+            "configs": side, "merge": merge, "decode": decode, "backward": backward,
             "device_status": ra.ra_status_string(status)}
     if rank == 0:
         print(json.dumps(line))
@@ -782,7 +945,7 @@ def run_merge_sweep(args):
     from seeded_inputs import MERGE_PARTIALS, MERGE_TOKENS
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     pk, pk_kind = peaks()
     sweep = []
     Ts = args.merge_T or MERGE_TOKENS
@@ -792,13 +955,16 @@ def run_merge_sweep(args):
             reps = 10 if T <= 262144 else 3
             pw, pw_ms = bench_merge(ra, dev, T, k, reps, flush)
             kw, kw_ms = bench_merge(ra, dev, T, k, reps, flush, kway=True)
-            sweep.append({"T": T, "k": k, "pairwise_GB/s": pw, "pairwise_ms": pw_ms, "kway_GB/s": kw, "kway_ms": kw_ms})
+            sweep.append({"T": T, "k": k, "pairwise_GB/s": pw, "pairwise_ms_per_launch": pw_ms,
+                          "pairwise_frac": pw / pk["hbm_gbs"], "kway_GB/s": kw, "kway_ms": kw_ms,
+                          "kway_frac": None if kw is None else kw / pk["hbm_gbs"],
+                          "bytes_per_pairwise_launch": T * 32 * (12 * 128 + 12)})
     top = max(sweep, key=lambda r: (r["T"], -r["k"]))
     line = {"metric": "merge GB/s (% of HBM peak)", "value": top["pairwise_GB/s"], "unit": "GB/s", "n_gpus": 1,
             "steps": None, "warmup": 2, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic (device randn / rand)",
             "config": {"workload": "merge sweep [T,32,128] fp32", "T": Ts, "k": ks,
-                       "headline": {"T": top["T"], "k": top["k"]}},
+                       "headline": {"T": top["T"], "k": top["k"]}, "l2": L2_FLUSH_DESC},
             "roofline": {"bound": "hbm", "achieved": top["pairwise_GB/s"], "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": top["pairwise_GB/s"] / pk["hbm_gbs"], "traffic": None,
                          "peak_source": f"{pk_kind} copy bandwidth"},

@@ -396,6 +396,43 @@ def test_gqa24k_workload_sampled_rows(cuda_lib, sched):
     assert ra.ra_get_device_status() == 0
 
 
+def whole_tile_rows(w, seed=0):
+    """Every row of whole 128-row query tiles, per head: the ragged last tile
+    of chunk h mod 2n and one seeded interior tile of chunk (h + 3) mod 2n.
+    Query tiles start at their chunk's first token (zigzag chunks of c tokens,
+    tiles never straddle one), so these are exactly the rows one CTA's tile
+    writes; across the heads every chunk's tail and many interior tiles are
+    covered."""
+    rng = np.random.default_rng(seed)
+    nch = 2 * w.n_blocks
+    c = w.S // nch
+    ntiles = (c + 127) // 128
+    rows = []
+    for b in range(w.B):
+        for h in range(w.Hq):
+            tail = (h % nch) * c + (ntiles - 1) * 128
+            rows.extend((b, i, h) for i in range(tail, (h % nch) * c + c))
+            t = int(rng.integers(0, ntiles - 1))
+            first = ((h + 3) % nch) * c + 128 * t
+            rows.extend((b, i, h) for i in range(first, first + 128))
+    return rows
+
+
+def test_gqa24k_whole_tiles(cuda_lib):
+    # Sampled rows could miss a fault confined to one tile of one head; here
+    # every row of two whole tiles per head (32 heads, 5,888 rows) is checked
+    # against the fp64 oracle, the ragged 56-row chunk tails included.
+    ra = cuda_lib
+    w = WORKLOADS["gqa24k"]
+    q, k, v = workload_inputs(w)
+    o, l = ra.ra_ring_attention(q.cuda(), k.cuda(), v.cuda(), w.n_blocks, w.causal, w.partition,
+                                out_dtype=torch.float32)
+    rows = whole_tile_rows(w)
+    assert len(rows) == w.Hq * ((w.S // 8) % 128 + 128)
+    check_sampled(w, q, k, v, o, l, rows, "gqa24k whole tiles")
+    assert ra.ra_get_device_status() == 0
+
+
 def test_long1m_workload_sampled_rows(cuda_lib):
     ra = cuda_lib
     w = WORKLOADS["long1m"]
