@@ -221,12 +221,52 @@ int grid_for(long long work, int per_block) {
   return static_cast<int>(need < 1 ? 1 : (need < cap ? need : cap));
 }
 
+// Grid of a merge kernel: one block per 8 warp sweeps, at most 16 blocks
+// per SM (the kernels stride over the rest).
+int merge_grid(long long sweeps) {
+  const long long need = (sweeps + (kMergeThreads / 32) - 1) / (kMergeThreads / 32);
+  const long long cap = static_cast<long long>(sm_count()) * 16;
+  return static_cast<int>(need < 1 ? 1 : (need < cap ? need : cap));
+}
+
 ra_status launch_merge(float* out, float* lse, const float* bo, const float* bl, long long rows, int D,
                        cudaStream_t st) {
   const long long nvec = rows * (D / 4);
-  merge_partial_kernel<<<grid_for(nvec, kMergeThreads * kMergeUnroll), kMergeThreads, 0, st>>>(
+  merge_partial_kernel<<<merge_grid((nvec + 32 * kMergeUnroll - 1) / (32 * kMergeUnroll)), kMergeThreads, 0, st>>>(
       out, lse, bo, bl, rows, D / 4);
   return cuda_status(cudaGetLastError());
+}
+
+template <int K>
+ra_status launch_merge_k(const MergeList& ml, float* out, float* lse, long long rows, int D, cudaStream_t st) {
+  constexpr int V = K <= 4 ? 2 : 1;
+  const long long nvec = rows * (D / 4);
+  merge_partials_kernel<K><<<merge_grid((nvec + 32 * V - 1) / (32 * V)), kMergeThreads, 0, st>>>(ml, out, lse, rows,
+                                                                                               D / 4);
+  return cuda_status(cudaGetLastError());
+}
+
+ra_status launch_merge_partials(const MergeList& ml, int k, float* out, float* lse, long long rows, int D,
+                                cudaStream_t st) {
+  switch (k) {
+    case 1: return launch_merge_k<1>(ml, out, lse, rows, D, st);
+    case 2: return launch_merge_k<2>(ml, out, lse, rows, D, st);
+    case 3: return launch_merge_k<3>(ml, out, lse, rows, D, st);
+    case 4: return launch_merge_k<4>(ml, out, lse, rows, D, st);
+    case 5: return launch_merge_k<5>(ml, out, lse, rows, D, st);
+    case 6: return launch_merge_k<6>(ml, out, lse, rows, D, st);
+    case 7: return launch_merge_k<7>(ml, out, lse, rows, D, st);
+    case 8: return launch_merge_k<8>(ml, out, lse, rows, D, st);
+    case 9: return launch_merge_k<9>(ml, out, lse, rows, D, st);
+    case 10: return launch_merge_k<10>(ml, out, lse, rows, D, st);
+    case 11: return launch_merge_k<11>(ml, out, lse, rows, D, st);
+    case 12: return launch_merge_k<12>(ml, out, lse, rows, D, st);
+    case 13: return launch_merge_k<13>(ml, out, lse, rows, D, st);
+    case 14: return launch_merge_k<14>(ml, out, lse, rows, D, st);
+    case 15: return launch_merge_k<15>(ml, out, lse, rows, D, st);
+    case 16: return launch_merge_k<16>(ml, out, lse, rows, D, st);
+  }
+  return RA_ERR_UNSUPPORTED;
 }
 
 // Row move between original and block order, bit-exact, for rows and base
@@ -612,10 +652,7 @@ ra_status ra_merge_partials(const float* const* outs, const float* const* lses, 
     ml.outs[j] = outs[j];
     ml.lses[j] = lses[j];
   }
-  const long long nvec = rows * (D / 4);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  merge_partials_kernel<<<grid_for(nvec, kMergeThreads), kMergeThreads, 0, st>>>(ml, k, out, lse, rows, D / 4);
-  return cuda_status(cudaGetLastError());
+  return launch_merge_partials(ml, k, out, lse, rows, D, static_cast<cudaStream_t>(stream));
 }
 
 ra_status ra_zigzag_permute(const void* src, void* dst, int B, int S, int H, int D, int elem_bytes, int n_blocks,

@@ -14,27 +14,35 @@
 namespace ra {
 
 constexpr int kMergeThreads = 256;
-constexpr int kMergeUnroll = 2;
+constexpr int kMergeUnroll = 2;  // float4 vectors per lane and warp sweep (pairwise)
 constexpr int kMaxMergeInputs = 16;
 
+// Work split of the merge kernels: the vectors are cut into sweeps of one
+// warp (32 * V vectors, whole rows since D / 4 divides 32), and the warps of
+// the grid take the sweeps in turn (grid stride).  The grid holds many more
+// blocks than are resident at once, so the block scheduler keeps every SM fed
+// to the end even though SMs do not all stream at the same rate.
 // out, lse <- merge(out, lse; block_out, block_lse), in place.
 __global__ void __launch_bounds__(kMergeThreads)
     merge_partial_kernel(float* __restrict__ out, float* __restrict__ lse,
                          const float* __restrict__ block_out, const float* __restrict__ block_lse,
                          long long rows, int vpr /* D / 4 */) {
+  constexpr int V = kMergeUnroll;
   const long long nvec = rows * vpr;
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x * kMergeUnroll;
-  const long long base0 = (static_cast<long long>(blockIdx.x) * blockDim.x * kMergeUnroll) + threadIdx.x;
+  const long long sweeps = (nvec + 32 * V - 1) / (32 * V);
+  const long long nw = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
   float4* o4 = reinterpret_cast<float4*>(out);
   const float4* b4 = reinterpret_cast<const float4*>(block_out);
-  for (long long base = base0 - threadIdx.x % 32; base < nvec; base += stride) {
-    // `base` is warp-uniform here: the warp's first vector of this sweep
-    float4 ov[kMergeUnroll], bv[kMergeUnroll];
-    float la[kMergeUnroll], lb[kMergeUnroll];
-    long long iv[kMergeUnroll];
+  for (long long g = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); g < sweeps;
+       g += nw) {
+    const long long base = g * 32 * V;  // the warp's first vector of this sweep
+    float4 ov[V], bv[V];
+    float la[V], lb[V];
+    long long iv[V];
 #pragma unroll
-    for (int u = 0; u < kMergeUnroll; ++u) {
-      iv[u] = base + threadIdx.x % 32 + static_cast<long long>(u) * blockDim.x;
+    for (int u = 0; u < V; ++u) {
+      iv[u] = base + 32 * u + lane;
       if (iv[u] < nvec) {
         const long long row = iv[u] / vpr;
         ov[u] = o4[iv[u]];
@@ -45,7 +53,7 @@ __global__ void __launch_bounds__(kMergeThreads)
     }
     __syncwarp();  // every lane has read lse[row] before any lane rewrites it
 #pragma unroll
-    for (int u = 0; u < kMergeUnroll; ++u) {
+    for (int u = 0; u < V; ++u) {
       if (iv[u] < nvec) {
         const MergeWeights mw = merge_weights(la[u], lb[u]);
         float4 r;
@@ -65,40 +73,58 @@ struct MergeList {
   const float* lses[kMaxMergeInputs];
 };
 
-// k partials folded left to right on chip; one write of the result.
+// k = K partials folded left to right on chip; one write of the result.
+// K is a compile-time constant so that every partial's load is issued before
+// the first one is folded in (K loads in flight per vector); V vectors per
+// lane and sweep (2 for K <= 4, where K alone keeps few loads in flight).
 // out / lse may alias outs[0] / lses[0]: every lane reads its row's lse before
 // the warp rewrites it (the lanes of a row share a warp; see the top note).
+template <int K>
 __global__ void __launch_bounds__(kMergeThreads)
-    merge_partials_kernel(const __grid_constant__ MergeList in, int k, float* out, float* lse,
-                          long long rows, int vpr) {
+    merge_partials_kernel(const __grid_constant__ MergeList in, float* out, float* lse, long long rows, int vpr) {
+  constexpr int V = K <= 4 ? 2 : 1;
   const long long nvec = rows * vpr;
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  const int lane = threadIdx.x % 32;
-  for (long long base = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x - lane; base < nvec;
-       base += stride) {
-    const long long i = base + lane;
-    const bool act = i < nvec;
-    const long long row = act ? i / vpr : 0;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float l = -INFINITY;
-    if (act) {
-      acc = reinterpret_cast<const float4*>(in.outs[0])[i];
-      l = in.lses[0][row];
-      for (int j = 1; j < k; ++j) {
-        const float4 bo = __ldcs(reinterpret_cast<const float4*>(in.outs[j]) + i);
-        const float bl = in.lses[j][row];
-        const MergeWeights mw = merge_weights(l, bl);
-        acc.x = merge_out(acc.x, bo.x, mw.w);
-        acc.y = merge_out(acc.y, bo.y, mw.w);
-        acc.z = merge_out(acc.z, bo.z, mw.w);
-        acc.w = merge_out(acc.w, bo.w, mw.w);
-        l = mw.lse;
+  const long long sweeps = (nvec + 32 * V - 1) / (32 * V);
+  const long long nw = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  for (long long g = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); g < sweeps;
+       g += nw) {
+    const long long base = g * 32 * V;
+    long long iv[V], row[V];
+    bool act[V];
+    float4 v[V][K];
+    float l[V][K];
+#pragma unroll
+    for (int u = 0; u < V; ++u) {
+      iv[u] = base + 32 * u + lane;
+      act[u] = iv[u] < nvec;
+      row[u] = act[u] ? iv[u] / vpr : 0;
+      if (act[u]) {
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+          v[u][j] = j == 0 ? reinterpret_cast<const float4*>(in.outs[0])[iv[u]]
+                           : __ldcs(reinterpret_cast<const float4*>(in.outs[j]) + iv[u]);
+          l[u][j] = in.lses[j][row[u]];
+        }
       }
     }
     __syncwarp();
-    if (act) {
-      reinterpret_cast<float4*>(out)[i] = acc;
-      if (i % vpr == 0) lse[row] = l;
+#pragma unroll
+    for (int u = 0; u < V; ++u) {
+      if (!act[u]) continue;
+      float4 acc = v[u][0];
+      float la = l[u][0];
+#pragma unroll
+      for (int j = 1; j < K; ++j) {
+        const MergeWeights mw = merge_weights(la, l[u][j]);
+        acc.x = merge_out(acc.x, v[u][j].x, mw.w);
+        acc.y = merge_out(acc.y, v[u][j].y, mw.w);
+        acc.z = merge_out(acc.z, v[u][j].z, mw.w);
+        acc.w = merge_out(acc.w, v[u][j].w, mw.w);
+        la = mw.lse;
+      }
+      reinterpret_cast<float4*>(out)[iv[u]] = acc;
+      if (iv[u] % vpr == 0) lse[row[u]] = la;
     }
   }
 }
