@@ -63,9 +63,6 @@ constexpr int kBM = 128;        // query rows per tile = TMEM lanes
 constexpr int kCtaRows = 256;   // two tiles per CTA
 constexpr int kBN = 128;        // keys per KV tile
 constexpr int kMaxBlocks = 16;  // ring size limit
-// Largest row sum of a tile's exponentials accepted on the common softmax path
-// (every value is then <= 2^15).
-constexpr float kFastSumLimit = 32768.f;
 constexpr int kAttnThreads = 384;
 constexpr int kRegsLaunch = 168;  // per thread at launch (__launch_bounds__(384, 1))
 constexpr int kRegsSoftmax = 216;
@@ -116,22 +113,25 @@ struct AttnArgs {
 };
 
 // Shared memory: the Q tiles (two for row pairs, one for KV-split), then a
-// ring of K tiles and a ring of V tiles sized to fill the 227 KB: K is
-// needed first (S = Q K^T), so its ring is at least as deep as V's.
+// ring of K tiles and a ring of V tiles sized to fill the 227 KB.  A stage of
+// either ring is refilled once the products of its step have read it, and
+// V(g) is needed at the start of step g while K(g + 1) is needed only after
+// P_A V(g) has been issued, so V gets the deeper ring where they differ.
 template <int D, bool SPLIT>
 struct AttnSmem {
   static constexpr int kBox = kBM * 64 * 2;  // one TMA box: 128 rows x 64 bf16 (128 B) = 16 KB
   static constexpr int kNBox = D / 64;
   static constexpr int kTile = kBox * kNBox;
   static constexpr int kQTiles = SPLIT ? 1 : 2;
-  static constexpr int kNSK = D == 128 ? 3 : 6;
-  static constexpr int kNSV = D == 128 ? (SPLIT ? 3 : 2) : (SPLIT ? 6 : 4);
+  static constexpr int kNSK = D == 128 ? (SPLIT ? 3 : 2) : (SPLIT ? 6 : 5);
+  static constexpr int kNSV = D == 128 ? 3 : 6;
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kQTiles * kTile;
   static constexpr int kV = kK + kNSK * kTile;
   static constexpr int kBar = kV + kNSV * kTile;
-  // barriers: Q, Kfull[NSK], Kempty[NSK], Vfull[NSV], Vempty[NSV], Sfull[2], Pfull[2], Odone[2], End
-  static constexpr int kNBar = 1 + 2 * kNSK + 2 * kNSV + 2 + 2 + 2 + 1;
+  // barriers: Q, Kfull[NSK], Kempty[NSK], Vfull[NSV], Vempty[NSV], Sfull[2], Pfull[2] (first
+  // half of P), Odone[2], End, Phalf[2] (second half of P)
+  static constexpr int kNBar = 1 + 2 * kNSK + 2 * kNSV + 2 + 2 + 2 + 1 + 2;
   static constexpr int kTmemSlot = kBar + kNBar * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kTotal = kAbort + 4;               // KV tiles of the CTA's sequence
@@ -274,12 +274,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   auto BPF = [&](int x) { return 3 + 2 * NSK + 2 * NSV + x; };
   auto BOD = [&](int x) { return 5 + 2 * NSK + 2 * NSV + x; };
   const int BEND = 7 + 2 * NSK + 2 * NSV;
+  auto BPH = [&](int x) { return 8 + 2 * NSK + 2 * NSV + x; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SL::kAbort);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < SL::kNBar; ++i) mbar_init(bar(i), 1);
     mbar_init(bar(BPF(0)), kBM / 32);  // one arrival per softmax warp
     mbar_init(bar(BPF(1)), kBM / 32);
+    mbar_init(bar(BPH(0)), kBM / 32);
+    mbar_init(bar(BPH(1)), kBM / 32);
     *abort_flag = grid_timed_out() ? 1 : 0;  // after a timeout elsewhere, do no work
     fence_mbar_init();
   }
@@ -371,7 +374,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           o.y = pack_bf16x2(lo4.z, lo4.w);
           o.z = pack_bf16x2(hi4.x, hi4.y);
           o.w = pack_bf16x2(hi4.z, hi4.w);
-          *reinterpret_cast<uint4*>(dst0 + r * rstride) = o;
+          __stcs(reinterpret_cast<uint4*>(dst0 + r * rstride), o);
         }
       }
       return;
@@ -384,8 +387,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int r0 = 0; r0 < per; r0 += rpi) {
         const int r = r0 + rl;
         if (r < per && wr0 + r < my_rows)
-          *reinterpret_cast<float4*>(dst0 + r * rstride) =
-              *reinterpret_cast<const float4*>(stage + (wr0 + r) * kStride + 4 * ci);
+          __stcs(reinterpret_cast<float4*>(dst0 + r * rstride),
+                 *reinterpret_cast<const float4*>(stage + (wr0 + r) * kStride + 4 * ci));
       }
       return;
     }
@@ -430,8 +433,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int issued_k[NSK], issued_v[NSV];
       for (int s = 0; s < NSK; ++s) issued_k[s] = -1;
       for (int s = 0; s < NSV; ++s) issued_v[s] = -1;
+      // L2 prefetch: when load g2 is issued into its ring stage, load
+      // g2 + kL2Ahead is prefetched into L2, so that by the time its own stage
+      // frees, its ring load reads L2 rather than HBM.  A second cursor walks
+      // the load order kL2Ahead loads ahead of the ring loads.
+      constexpr int kL2Ahead = 2;
+      KvWalk pa = wa, pb = wb;
+      int g_pf = 0;
+      auto prefetch_next = [&]() {
+        const bool pub = split && (g_pf & 1);
+        KvWalk& pw = pub ? pb : pa;
+        const int row = seg_tab[pw.sg].seg.mem + pw.t * kBN;
+        for (int bx = 0; bx < SL::kNBox; ++bx) {
+          tma_prefetch_l2_4d(&tmK, bx * 64, hk, row, b);
+          tma_prefetch_l2_4d(&tmV, bx * 64, hk, row, b);
+        }
+        walk_next(pw);
+        ++g_pf;
+      };
+      for (int i = 0; i < kL2Ahead && g_pf < work; ++i) walk_next(split && (g_pf & 1) ? pb : pa), ++g_pf;
       // load order: the CTA's sequence (row pairs), or A0, B0, A1, B1, ... (KV-split)
       for (int g2 = 0; g2 < work && ok; ++g2) {
+        if (g_pf < work) prefetch_next();
         const bool use_b = split && (g2 & 1);
         const int t = use_b ? wb.t : wa.t;
         const Seg ks = seg_tab[use_b ? wb.sg : wa.sg].seg;
@@ -468,23 +491,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, D, true);
       const int qslot1 = split ? 0 : 1;  // Q tile of B
+      // The tensor core takes 64 cycles for a 128 x 128 x 16 product and this
+      // one thread shares its scheduler with two softmax warps, so its work per
+      // product decides how close the products run to that rate.  Every
+      // descriptor is therefore a base computed here plus a compile-time
+      // offset added to its low half (see mma_ss_lo); the descriptors share
+      // their high half (the 1024-byte atom stride and the swizzle mode).
+      const uint64_t dq0 = smem_desc_sw128(sb + SL::kQ, 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(sb + SL::kK, 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(sb + SL::kV, SL::kBox, 1024);
+      const uint32_t hi_qk = static_cast<uint32_t>(dq0 >> 32), hi_v = static_cast<uint32_t>(dv0 >> 32);
+      const uint32_t lo_q0 = static_cast<uint32_t>(dq0);
+      const uint32_t lo_q1 = lo_q0 + static_cast<uint32_t>((qslot1 * SL::kTile) >> 4);
+      const uint32_t lo_k = static_cast<uint32_t>(dk0), lo_v = static_cast<uint32_t>(dv0);
       auto issue_s = [&](int x, int st) {
+        const uint32_t a = x ? lo_q1 : lo_q0;
+        const uint32_t bk = lo_k + static_cast<uint32_t>(st) * (SL::kTile >> 4);
+        const uint32_t td = tmem + x * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
-          const uint64_t ad = smem_desc_sw128(sb + SL::kQ + (x ? qslot1 : 0) * SL::kTile + off, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sb + SL::kK + st * SL::kTile + off, 16, 1024);
-          mma_ss(tmem + x * 128, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk / 4) * SL::kBox + (kk % 4) * 32) >> 4;
+          mma_ss_lo(td, a + off, bk + off, hi_qk, kIdescS, kk > 0 ? 1u : 0u);
         }
         tc_commit(bar(BSF(x)));
       };
-      auto issue_pv = [&](int x, int st, bool acc) {
+      // O_X += P_X V in two halves of the keys: the first as soon as the
+      // softmax has written P's first 64 columns (Pfull), the second once it
+      // has written the rest (Phalf).  Returns false when a wait gave up.
+      auto issue_pv = [&](int x, int st, bool acc, uint32_t parity) -> bool {
+        const uint32_t bv = lo_v + static_cast<uint32_t>(st) * (SL::kTile >> 4);
+        const uint32_t to = tmem + 256 + x * 128, tp = tmem + x * 128;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bd = smem_desc_sw128(sb + SL::kV + st * SL::kTile + kk * 2048, SL::kBox, 1024);
-          mma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, bd, kIdescO, (acc || kk > 0) ? 1u : 0u);
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait_spin(bar(h ? BPH(x) : BPF(x)), parity, abort_flag)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
+            mma_ts_lo(to, tp + kk * 8, bv + ((kk * 2048) >> 4), hi_v, kIdescO, (acc || kk > 0) ? 1u : 0u);
         }
-        tc_commit(bar(BOD(x)));
+        return true;
       };
 
       if (split) {
@@ -504,9 +549,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (j >= n_of[x]) continue;
             const int ld = 2 * j + x, st = ld % NSV;
             if (!mbar_wait(bar(BVF(st)), (ld / NSV) & 1, abort_flag)) { okk = false; break; }
-            if (!mbar_wait_spin(bar(BPF(x)), j & 1, abort_flag)) { okk = false; break; }
-            tc_fence_after();
-            issue_pv(x, st, j > 0);
+            if (!issue_pv(x, st, j > 0, j & 1)) { okk = false; break; }
             tc_commit(bar(BVE(st)));
             if (j + 1 < n_of[x]) {
               const int ld1 = ld + 2, st1 = ld1 % NSK;
@@ -517,6 +560,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
           }
         }
+        tc_commit(bar(BOD(0)));  // O_A and O_B are complete once every product is
+        tc_commit(bar(BOD(1)));
         tc_commit(bar(BEND));
         mbar_drain(bar(BEND), 0);
       } else {
@@ -544,12 +589,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         if (!mbar_wait(bar(BVF(st)), (g / NSV) & 1, abort_flag)) break;
         bool k_ready = false;
+        const int last_pv = act[1] ? 1 : 0;  // the step's last P V product reads V(g) last
         for (int x = 0; x < 2; ++x) {
           if (act[x]) {
-            if (!mbar_wait_spin(bar(BPF(x)), cnt[x] & 1, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            issue_pv(x, st, cnt[x] > 0);
+            if (!issue_pv(x, st, cnt[x] > 0, cnt[x] & 1)) { ok = false; break; }
             ++cnt[x];
+            if (x == last_pv) tc_commit(bar(BVE(st)));  // V(g) is free once that product is done
           }
           if (act1[x]) {
             if (!k_ready) {
@@ -561,12 +606,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
         if (!ok) break;
-        tc_commit(bar(BVE(st)));
         if (has_next) tc_commit(bar(BKE(sk1)));
         cur = nxt;
         act[0] = act1[0];
         act[1] = act1[1];
       }
+      tc_commit(bar(BOD(0)));  // O_A and O_B are complete once every product is
+      tc_commit(bar(BOD(1)));
       // nothing may still write tensor memory when it is released
       tc_commit(bar(BEND));
       mbar_drain(bar(BEND), 0);
@@ -586,8 +632,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t tS = tmem + lane_base + x * 128;
     const uint32_t tO = tmem + lane_base + 256 + x * 128;
     const float sl2 = a.scale_log2;
-    // Padding rows (beyond the segment) see no key; a finite base keeps their
-    // warp on the common path (their exponentials are all 0).
+    // Padding rows (beyond the segment) see no key: all their scores are
+    // masked and, with a finite base, their exponentials are 0.
     float m_use = valid ? -INFINITY : 0.f;
     float l_sum = 0.f;
     bool ok = work > 0;
@@ -610,27 +656,63 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_after();
       uint32_t sv[kBN];
       const int cnt = lim - t * kBN;
-      const bool masked = __any_sync(0xffffffffu, cnt < kBN);  // warp-uniform: full tiles skip the masking code
       // S of this row from TMEM, with the keys it may not see set to -inf
-      auto load_s = [&]() {
-        tmem_ld128_wait(tS, sv);
-        if (masked) {
+      // (warp-uniform test: full tiles skip the masking code)
+      tmem_ld128_wait(tS, sv);
+      if (__any_sync(0xffffffffu, cnt < kBN)) {
 #pragma unroll
-          for (int j = 0; j < kBN; ++j) sv[j] = j < cnt ? sv[j] : __float_as_uint(-INFINITY);
+        for (int j = 0; j < kBN; ++j) sv[j] = j < cnt ? sv[j] : __float_as_uint(-INFINITY);
+      }
+      // The row maximum first (3-input max, 8 independent chains of depth 8),
+      // so that the base of the exponentials is settled before any of them is
+      // taken: P can then go to the tensor core in two halves.  The base is
+      // raised only when the tile maximum exceeds it by more than 8 (log2
+      // units; every P value then stays <= 2^8), and O is rescaled in TMEM.
+      float m8[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) m8[q] = fmaxf(__uint_as_float(sv[2 * q]), __uint_as_float(sv[2 * q + 1]));
+#pragma unroll
+      for (int j = 16; j < kBN; j += 16)
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          m8[q] = fmax3(m8[q], __uint_as_float(sv[j + 2 * q]), __uint_as_float(sv[j + 2 * q + 1]));
+      const float mt =
+          fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * sl2;
+      float alpha = 1.f;
+      bool resc = false;
+      if (mt > m_use + 8.f) {  // also a row's first visible keys (m_use = -inf)
+        if (m_use != -INFINITY) {
+          alpha = fast_exp2(m_use - mt);
+          resc = true;
         }
-      };
-      load_s();
+        m_use = mt;
+      }
+      // O of this tile is stable here: S_X(c) was committed after the P V
+      // product of tile c-1, so its completion implies that one's.
+      if (c > 0 && __any_sync(0xffffffffu, resc)) {
+#pragma unroll
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t ov[32];
+          tmem_ld32_wait(tO + 32 * q, ov);
+#pragma unroll
+          for (int i2 = 0; i2 < 32; ++i2) ov[i2] = __float_as_uint(__uint_as_float(ov[i2]) * alpha);
+          tmem_st32(tO + 32 * q, ov);
+        }
+      }
       // P = 2^(scale * S - base) as packed bf16 pairs, on the SFU (ex2.approx),
-      // two per pair of scores, into pk (when given) or straight into the
-      // tile's TMEM columns (over S); returns the row sum of the fp32 values.
-      auto exps = [&](float base, uint32_t* pk_out) -> float {
-        const uint64_t sl2x2 = f2_pack(sl2, sl2);
-        const uint64_t nbase2 = f2_pack(-base, -base);
+      // over the score columns [64h, 64h + 64), stored over S in this tile's
+      // TMEM columns [32h, 32h + 32); returns the row sum of the fp32 values.
+      // Each half is handed to the MMA thread as soon as it is in TMEM.
+      const float base = m_use == -INFINITY ? 0.f : m_use;
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      const uint64_t nbase2 = f2_pack(-base, -base);
+      float psum = 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
         uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-        for (int ch = 0; ch < kBN / 32; ++ch) {  // 32 scores -> 16 packed bf16 pairs per store
-          uint32_t pk_local[16];
-          uint32_t* pk = pk_out ? pk_out + ch * 16 : pk_local;
+        for (int ch = 2 * h; ch < 2 * h + 2; ++ch) {  // 32 scores -> 16 packed bf16 pairs per store
+          uint32_t pk[16];
 #pragma unroll
           for (int pp = 0; pp < 16; ++pp) {
             const int j = ch * 32 + 2 * pp;
@@ -644,75 +726,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             f2_unpack(e2, p0, p1);
             pk[pp] = pack_bf16x2(p0, p1);
           }
-          if (!pk_out) tmem_st16(tS + ch * 16, pk);
+          tmem_st16(tS + ch * 16, pk);
         }
         const uint64_t acc2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
         float ps0, ps1;
         f2_unpack(acc2, ps0, ps1);
-        return ps0 + ps1;
-      };
-      // Common case: the exponentials against the running base m_use, with no
-      // tile maximum.  Kept when every value stays <= 2^15 (their sum does),
-      // which bf16 P and the fp32 sums hold exactly as well as values <= 1:
-      // out = O / l and lse = ln 2 * (m_use + log2 l) are exact for any base.
-      float psum = 0.f;
-      bool done = false;
-      if (__all_sync(0xffffffffu, m_use != -INFINITY)) {
-        uint32_t pk[kBN / 2];
-        psum = exps(m_use, pk);
-        done = __all_sync(0xffffffffu, psum <= kFastSumLimit);
-        if (done) {
-#pragma unroll
-          for (int ch = 0; ch < kBN / 32; ++ch) tmem_st16(tS + ch * 16, pk + ch * 16);
-        } else {
-          load_s();  // S is still in TMEM: nothing was stored over it
-        }
-      }
-      // Otherwise (a row's first tile, or a score that rose more than about 8
-      // above the base): the tile maximum; the base is raised when the tile
-      // maximum exceeds it by more than 8, and the exponentials redone.
-      float alpha = 1.f;
-      bool resc = false;
-      if (!done) {
-        // row maximum: 3-input max, 8 independent chains of depth 8
-        float m8[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) m8[q] = fmaxf(__uint_as_float(sv[2 * q]), __uint_as_float(sv[2 * q + 1]));
-#pragma unroll
-        for (int j = 16; j < kBN; j += 16)
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            m8[q] = fmax3(m8[q], __uint_as_float(sv[j + 2 * q]), __uint_as_float(sv[j + 2 * q + 1]));
-        const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-        const float mt = mx * sl2;
-        if (mt > m_use + 8.f) {
-          if (m_use != -INFINITY) {
-            alpha = fast_exp2(m_use - mt);
-            resc = true;
-          }
-          m_use = mt;
-        }
-        psum = exps(m_use == -INFINITY ? 0.f : m_use, nullptr);
+        psum += ps0 + ps1;
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(h ? BPH(x) : BPF(x)));
       }
       l_sum = l_sum * alpha + psum;
-      tmem_wait_st();
-      // O of this tile is stable here: S_X(c) was committed after the
-      // P V product of tile c-1, so its completion implies that one's.
-      if (c > 0 && __any_sync(0xffffffffu, resc)) {
-        tc_fence_after();
-#pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
-          uint32_t ov[32];
-          tmem_ld32_wait(tO + 32 * q, ov);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tmem_st32(tO + 32 * q, ov);
-        }
-        tmem_wait_st();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BPF(x)));
       ++c;
     }
 
@@ -722,7 +747,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // rings hold the staging buffers: they are idle once the last P V products
     // of both tiles have landed (barrier below).
     if (ok && c > 0) {
-      ok = mbar_wait(bar(BOD(x)), (c - 1) & 1, abort_flag);
+      ok = mbar_wait(bar(BOD(x)), 0, abort_flag);  // one commit, after the last product
       ok = __all_sync(0xffffffffu, ok);
     }
     const bool has = ok && l_sum > 0.f;
