@@ -457,6 +457,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0 && work > 0) {
       constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t kIdescQ = idesc_bf16_f32(kBM, D, true);
+      // Descriptors as bases plus compile-time offsets (one add per operand
+      // and product: this one thread's work per product bounds how close the
+      // products run to the tensor core's rate).
+      const uint32_t dhi = desc_sw128_hi();
+      const uint32_t lo_q = desc_sw128_lo(sb + SL::kX, 16), lo_do = desc_sw128_lo(sb + SL::kX + SL::kTile, 16);
+      const uint32_t lo_k = desc_sw128_lo(sb + SL::kK, 16), lo_v = desc_sw128_lo(sb + SL::kV, 16);
+      const uint32_t lo_kmn = desc_sw128_lo(sb + SL::kK, SL::kBox);
       // S = Q K(j)^T into [0, 128), dP = dO V(j)^T into [128, 256): K-major operands
       auto issue_sdp = [&](int j) -> bool {
         const int sk = j % NK, sv = j % NV;
@@ -464,18 +471,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             !mbar_wait(bar(ib.full1(sv)), (j / NV) & 1, abort_flag))
           return false;
         tc_fence_after();
-        const uint32_t yk = sb + SL::kK + sk * SL::kTile, yv = sb + SL::kV + sv * SL::kTile;
+        const uint32_t bk = lo_k + static_cast<uint32_t>(sk) * (SL::kTile >> 4);
+        const uint32_t bv = lo_v + static_cast<uint32_t>(sv) * (SL::kTile >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
-          mma_ss(tmem + kTmS, smem_desc_sw128(sb + SL::kX + off, 16, 1024), smem_desc_sw128(yk + off, 16, 1024),
-                 kIdescS, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk / 4) * SL::kBox + (kk % 4) * 32) >> 4;
+          mma_ss_lo(tmem + kTmS, lo_q + off, bk + off, dhi, kIdescS, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
-          mma_ss(tmem + kTmP, smem_desc_sw128(sb + SL::kX + SL::kTile + off, 16, 1024),
-                 smem_desc_sw128(yv + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk / 4) * SL::kBox + (kk % 4) * 32) >> 4;
+          mma_ss_lo(tmem + kTmP, lo_do + off, bv + off, dhi, kIdescS, kk > 0 ? 1u : 0u);
         }
         tc_commit(bar(ib.empty1(sv)));  // V(j) is read only by dP(j)
         tc_commit(bar(ib.sfull()));
@@ -485,12 +491,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // B = rows of K(j) read MN-major; after half 1, K(j) is free
       auto issue_dq = [&](int j, int hf) {
         const int sk = j % NK;
-        const uint32_t yk = sb + SL::kK + sk * SL::kTile;
+        const uint32_t bk = lo_kmn + static_cast<uint32_t>(sk) * (SL::kTile >> 4);
+        const uint32_t ta = tmem + kTmDS + 64 * (j & 1) + 32 * hf;
+        const bool acc = j % kFlushTiles > 0 || hf > 0;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + kTmAcc, tmem + kTmDS + 64 * (j & 1) + 32 * hf + kk * 8,
-                 smem_desc_sw128(yk + (4 * hf + kk) * 2048, SL::kBox, 1024), kIdescQ,
-                 (j % kFlushTiles > 0 || hf > 0 || kk > 0) ? 1u : 0u);
+          mma_ts_lo(tmem + kTmAcc, ta + kk * 8, bk + (((4 * hf + kk) * 2048) >> 4), dhi, kIdescQ,
+                    (acc || kk > 0) ? 1u : 0u);
         if (hf == 1) tc_commit(bar(ib.empty0(sk)));
       };
       bool ok = mbar_wait(bar(ib.kX), 0, abort_flag) && issue_sdp(0);
@@ -721,16 +728,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       constexpr uint32_t kIdescO = idesc_bf16_f32(kBN, D, true);
       // S^T_h = K Q_h(j)^T into [64h, 64h + 64): Q_h = rows 64h.. of the Q tile
       constexpr uint32_t kIdescS2 = idesc_bf16_f32(kBN, 64, false);
+      // Descriptors as bases plus compile-time offsets (see the dQ kernel).
+      const uint32_t dhi = desc_sw128_hi();
+      const uint32_t lo_k = desc_sw128_lo(sb + SL::kX, 16), lo_v = desc_sw128_lo(sb + SL::kX + SL::kTile, 16);
+      const uint32_t lo_q = desc_sw128_lo(sb + SL::kQ, 16), lo_o = desc_sw128_lo(sb + SL::kO, 16);
+      const uint32_t lo_qmn = desc_sw128_lo(sb + SL::kQ, SL::kBox), lo_omn = desc_sw128_lo(sb + SL::kO, SL::kBox);
       auto issue_s = [&](int j, int hf) -> bool {
         const int sq = j % NQ;
         if (!mbar_wait(bar(ib.full0(sq)), (j / NQ) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t yq = sb + SL::kQ + sq * SL::kTile + hf * 64 * 128;
+        const uint32_t bq = lo_q + static_cast<uint32_t>(sq) * (SL::kTile >> 4) + ((hf * 64 * 128) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
-          mma_ss(tmem + kTmS + 64 * hf, smem_desc_sw128(sb + SL::kX + off, 16, 1024),
-                 smem_desc_sw128(yq + off, 16, 1024), kIdescS2, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk / 4) * SL::kBox + (kk % 4) * 32) >> 4;
+          mma_ss_lo(tmem + kTmS + 64 * hf, lo_k + off, bq + off, dhi, kIdescS2, kk > 0 ? 1u : 0u);
         }
         return true;
       };
@@ -739,12 +750,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int so_ = j % NO;
         if (!mbar_wait(bar(ib.full1(so_)), (j / NO) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t yo = sb + SL::kO + so_ * SL::kTile;
+        const uint32_t bo = lo_o + static_cast<uint32_t>(so_) * (SL::kTile >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * SL::kBox + (kk % 4) * 32;
-          mma_ss(tmem + kTmP, smem_desc_sw128(sb + SL::kX + SL::kTile + off, 16, 1024),
-                 smem_desc_sw128(yo + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk / 4) * SL::kBox + (kk % 4) * 32) >> 4;
+          mma_ss_lo(tmem + kTmP, lo_v + off, bo + off, dhi, kIdescS, kk > 0 ? 1u : 0u);
         }
         return true;
       };
@@ -752,16 +762,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // A = bf16 in TMEM (P^T_h at [64h, 64h + 32), dS^T_h at [64h + 32, 64h + 64)),
       // B = rows of dO(j) / Q(j) read MN-major; after half 1 both tiles are free
       auto issue_dkv = [&](int j, int hf) {
-        const uint32_t yq = sb + SL::kQ + (j % NQ) * SL::kTile, yo = sb + SL::kO + (j % NO) * SL::kTile;
+        const uint32_t bq = lo_qmn + static_cast<uint32_t>(j % NQ) * (SL::kTile >> 4);
+        const uint32_t bo = lo_omn + static_cast<uint32_t>(j % NO) * (SL::kTile >> 4);
         const bool acc = j % kFlushTiles > 0 || hf > 0;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + kTmAcc, tmem + 64 * hf + 8 * kk, smem_desc_sw128(yo + (4 * hf + kk) * 2048, SL::kBox, 1024),
-                 kIdescO, (acc || kk > 0) ? 1u : 0u);
+          mma_ts_lo(tmem + kTmAcc, tmem + 64 * hf + 8 * kk, bo + (((4 * hf + kk) * 2048) >> 4), dhi, kIdescO,
+                    (acc || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + kTmAcc + 128, tmem + 64 * hf + 32 + 8 * kk,
-                 smem_desc_sw128(yq + (4 * hf + kk) * 2048, SL::kBox, 1024), kIdescO, (acc || kk > 0) ? 1u : 0u);
+          mma_ts_lo(tmem + kTmAcc + 128, tmem + 64 * hf + 32 + 8 * kk, bq + (((4 * hf + kk) * 2048) >> 4), dhi,
+                    kIdescO, (acc || kk > 0) ? 1u : 0u);
         if (hf == 1) {
           tc_commit(bar(ib.empty1(j % NO)));
           tc_commit(bar(ib.empty0(j % NQ)));

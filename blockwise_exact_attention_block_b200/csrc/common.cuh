@@ -332,6 +332,15 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// Low half of smem_desc_sw128(saddr, lbo, 1024): the start address and the
+// leading byte offset.  The high half is the same for every such descriptor
+// (desc_sw128_hi): stepping a descriptor through a tile is one add of
+// (offset >> 4) to its low half (see mma_ss_lo).
+__device__ __forceinline__ uint32_t desc_sw128_lo(uint32_t saddr, uint32_t lbo) {
+  return static_cast<uint32_t>(smem_desc_sw128(saddr, lbo, 1024));
+}
+__device__ __forceinline__ uint32_t desc_sw128_hi() { return static_cast<uint32_t>(smem_desc_sw128(0, 16, 1024) >> 32); }
+
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator.
 //   b_mn_major: B operand is MN-major (N contiguous) instead of K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
