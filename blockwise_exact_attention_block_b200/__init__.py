@@ -22,11 +22,15 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libra_b200.so")
+# RA_DEBUG_BOUNDS=1 selects the checked build (every run-time-indexed global
+# access checked on the device; see ra_debug_build in include/ra.h).
+DEBUG_BOUNDS = os.environ.get("RA_DEBUG_BOUNDS", "0") == "1"
+LIB_PATH = os.path.join(_PKG, "libra_b200_debug.so" if DEBUG_BOUNDS else "libra_b200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python blockwise_exact_attention_block_b200/build.py`")
+        f"{LIB_PATH} is missing: build it with `python blockwise_exact_attention_block_b200/build.py"
+        f"{' --debug-bounds' if DEBUG_BOUNDS else ''}`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -46,7 +50,7 @@ EXPORTED = ["ra_block_attn", "ra_block_attn_merge", "ra_merge_partial", "ra_merg
             "ra_ring_attention_workspace", "ra_zigzag_permute", "ra_get_device_status",
             "ra_status_string", "ra_version", "ra_ring_attention_noalloc", "ra_noalloc_scratch_bytes",
             "ra_decode_attention", "ra_decode_workspace", "ra_decode_splits", "ra_ring_attention_backward",
-            "ra_ring_attention_backward_workspace"]
+            "ra_ring_attention_backward_workspace", "ra_debug_build", "ra_get_bounds_record"]
 
 
 class ra_options(ctypes.Structure):
@@ -95,6 +99,10 @@ _lib.ra_ring_attention_backward.argtypes = [_vp, _vp, _vp, _i, _vp, _i, _vp, _vp
 _lib.ra_ring_attention_backward.restype = _i
 _lib.ra_ring_attention_backward_workspace.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
 _lib.ra_ring_attention_backward_workspace.restype = _sz
+_lib.ra_debug_build.argtypes = []
+_lib.ra_debug_build.restype = _i
+_lib.ra_get_bounds_record.argtypes = [ctypes.POINTER(ctypes.c_int64)]
+_lib.ra_get_bounds_record.restype = _i
 
 
 class RAError(RuntimeError):
@@ -114,6 +122,19 @@ def ra_status_string(status: int) -> str:
 
 def ra_version() -> str:
     return _lib.ra_version().decode()
+
+
+def ra_debug_build() -> bool:
+    """True when the loaded library is the checked build (RA_DEBUG_BOUNDS)."""
+    return _lib.ra_debug_build() == 1
+
+
+def ra_get_bounds_record() -> tuple[int, int, int]:
+    """(source line, index, limit) of the first failed device index check
+    since the last read (zeros if none), then cleared."""
+    rec = (ctypes.c_int64 * 3)()
+    _check(_lib.ra_get_bounds_record(rec), "ra_get_bounds_record")
+    return int(rec[0]), int(rec[1]), int(rec[2])
 
 
 def _stream(stream=None) -> int:

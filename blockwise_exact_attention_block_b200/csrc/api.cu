@@ -347,7 +347,8 @@ bool valid_opts(const ra_options* o) {
   if (!o) return true;
   if (o->order != RA_ORDER_RING && o->order != RA_ORDER_TOKENRING) return false;
   if (o->tiling < RA_TILING_AUTO || o->tiling > RA_TILING_CLUSTER2) return false;
-  if (o->fault_inject != 0 && o->fault_inject != 1) return false;
+  // 2: the checked build's injected out-of-range row (see AttnArgs)
+  if (o->fault_inject != 0 && o->fault_inject != 1 && !(kDebugBounds && o->fault_inject == 2)) return false;
   return o->sched >= RA_SCHED_AUTO && o->sched <= RA_SCHED_PERSISTENT;
 }
 
@@ -549,6 +550,21 @@ const char* ra_status_string(ra_status s) {
 
 const char* ra_version(void) { return "ra_b200 0.1 (sm_100a)"; }
 
+int ra_debug_build(void) { return kDebugBounds ? 1 : 0; }
+
+ra_status ra_get_bounds_record(int64_t record[3]) {
+  if (!record) return RA_ERR_INVALID_ARG;
+  record[0] = record[1] = record[2] = 0;
+#ifdef RA_DEBUG_BOUNDS
+  long long r[3];
+  if (cudaMemcpyFromSymbol(r, g_bounds_record, sizeof(r)) != cudaSuccess) return RA_ERR_CUDA;
+  const long long z[3] = {0, 0, 0};
+  if (cudaMemcpyToSymbol(g_bounds_record, z, sizeof(z)) != cudaSuccess) return RA_ERR_CUDA;
+  for (int i = 0; i < 3; ++i) record[i] = r[i];
+#endif
+  return RA_OK;
+}
+
 ra_status ra_get_device_status(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int v = 0;
@@ -591,6 +607,7 @@ ra_status ra_block_attn(const void* q, const void* k, const void* v, ra_dtype in
   a.acc_out = block_out;
   a.acc_lse = block_lse;
   a.acc_brows = g.L;
+  a.q_rows = a.kv_rows = g.L;  // the maps cover block-local tensors
   return launch_attn(D, a, mq, mk, mv, static_cast<cudaStream_t>(stream));
 }
 
@@ -622,6 +639,7 @@ ra_status ra_block_attn_merge(const void* q, const void* k, const void* v, ra_dt
   a.acc_out = out;
   a.acc_lse = lse;
   a.acc_brows = g.L;
+  a.q_rows = a.kv_rows = g.L;  // the maps cover block-local tensors
   return launch_attn(D, a, mq, mk, mv, static_cast<cudaStream_t>(stream));
 }
 
@@ -757,6 +775,7 @@ ra_status ra_ring_attention(const void* q, const void* k, const void* v, ra_dtyp
   order_segments(a);
   choose_tiling(g, a, opts ? opts->tiling : RA_TILING_AUTO);
   a.fault_inject = opts ? opts->fault_inject : 0;
+  a.q_rows = a.kv_rows = S;  // the maps cover the tensors in original order
 
   if (p.sched == RA_SCHED_PERSISTENT) {
     // a3-a6 in one launch: the running state is carried across block boundaries

@@ -164,8 +164,10 @@ __global__ void __launch_bounds__(256)
       const long long bs = r / Hq;
       const int s = static_cast<int>(bs % S), b = static_cast<int>(bs / S);
       const long long t = (static_cast<long long>(b) * Hq + h) * S + s;
-      delta[t] = acc;
-      lse2[t] = lse[r] * 1.4426950408889634f;
+      if (RA_IN_BOUNDS(t, rows)) {
+        delta[t] = acc;
+        lse2[t] = lse[r] * 1.4426950408889634f;
+      }
     }
   }
 }
@@ -220,7 +222,7 @@ __device__ __forceinline__ bool bar_and(int id, int count, bool pred) {
 template <int NC>
 __device__ __forceinline__ void bwd_store_rows(float* stage, uint32_t taddr, int quad, int lane, float* dst,
                                                long long first_row, long long row_stride, int ld, int nrows,
-                                               float mul, bool add) {
+                                               float mul, bool add, long long dst_rows) {
   constexpr int kStride = NC + 4;
   const int row = quad * 32 + lane;
 #pragma unroll
@@ -239,7 +241,7 @@ __device__ __forceinline__ void bwd_store_rows(float* stage, uint32_t taddr, int
 #pragma unroll 4
   for (int r0 = 0; r0 < 32; r0 += rpi) {
     const int r = quad * 32 + r0 + rl;
-    if (r < nrows) {
+    if (r < nrows && RA_IN_BOUNDS(first_row + r * row_stride, dst_rows)) {
       float4* p = reinterpret_cast<float4*>(dst + (first_row + r * row_stride) * ld + 4 * ci);
       float4 val = *reinterpret_cast<const float4*>(stage + r * kStride + 4 * ci);
       if (add) {
@@ -413,10 +415,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmdO);
-      mbar_expect_tx(bar(ib.kX), 2 * SL::kTile);
-      for (int bx = 0; bx < D / 64; ++bx) {
-        tma_load_4d(sb + SL::kX + bx * SL::kBox, &tmQ, bx * 64, h, qs.mem + row0, b, bar(ib.kX));
-        tma_load_4d(sb + SL::kX + SL::kTile + bx * SL::kBox, &tmdO, bx * 64, h, qs.mem + row0, b, bar(ib.kX));
+      // checked build: the CTA's rows and heads must lie inside the tensors
+      const bool x_ok = RA_IN_BOUNDS(qs.mem + row0, a.S) && RA_IN_BOUNDS(h, a.Hq) && RA_IN_BOUNDS(hk, a.Hkv);
+      if (!x_ok) *abort_flag = 1;
+      if (x_ok) {
+        mbar_expect_tx(bar(ib.kX), 2 * SL::kTile);
+        for (int bx = 0; bx < D / 64; ++bx) {
+          tma_load_4d(sb + SL::kX + bx * SL::kBox, &tmQ, bx * 64, h, qs.mem + row0, b, bar(ib.kX));
+          tma_load_4d(sb + SL::kX + SL::kTile + bx * SL::kBox, &tmdO, bx * 64, h, qs.mem + row0, b, bar(ib.kX));
+        }
       }
       int j = 0, lastk[NK], lastv[NV];
       for (int s = 0; s < NK; ++s) lastk[s] = -1;
@@ -428,7 +435,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const int nt = nt_of(s_, e_);
           for (int t = 0; t < nt; ++t, ++j) {
             const int sk = j % NK, sv = j % NV, r = ks.mem + t * kBN;
-            if (!mbar_wait(bar(ib.empty0(sk)), ((j / NK) & 1) ^ 1, abort_flag)) {
+            if (!mbar_wait(bar(ib.empty0(sk)), ((j / NK) & 1) ^ 1, abort_flag) || !RA_IN_BOUNDS(r, a.S)) {
+              *abort_flag = 1;
               ok = false;
               break;
             }
@@ -447,7 +455,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
         }
       // every copy issued lands before the CTA can release its shared memory
-      mbar_drain(bar(ib.kX), 0);
+      if (x_ok) mbar_drain(bar(ib.kX), 0);
       for (int s = 0; s < NK; ++s)
         if (lastk[s] >= 0) mbar_drain(bar(ib.full0(s)), (lastk[s] / NK) & 1);
       for (int s = 0; s < NV; ++s)
@@ -551,7 +559,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             bwd_flush_row<NC>(tmem + lane_base + kTmAcc + half * NC,
                               a.dq + ((static_cast<long long>(b) * a.S + qs.pos + row0 + row) * a.Hq + h) * D +
                                   half * NC,
-                              valid, j > kFlushTiles, a.scale);
+                              valid && RA_IN_BOUNDS((static_cast<long long>(b) * a.S + qs.pos + row0 + row) * a.Hq + h,
+                                                    static_cast<long long>(a.B) * a.S * a.Hq),
+                              j > kFlushTiles, a.scale);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(ib.fempty()));
@@ -593,7 +603,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       float* stage = reinterpret_cast<float*>(smem) + half * kBM * (NC + 4);
       bwd_store_rows<NC>(stage, tmem + lane_base + kTmAcc + half * NC, quad, lane, a.dq + half * NC,
                          (static_cast<long long>(b) * a.S + qs.pos + row0) * a.Hq + h, a.Hq, D, rows, a.scale,
-                         work > kFlushTiles);
+                         work > kFlushTiles, static_cast<long long>(a.B) * a.S * a.Hq);
     }
   }
   tc_fence_before();
@@ -679,10 +689,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmdO);
-      mbar_expect_tx(bar(ib.kX), 2 * SL::kTile);
-      for (int bx = 0; bx < D / 64; ++bx) {
-        tma_load_4d(sb + SL::kX + bx * SL::kBox, &tmK, bx * 64, g, ks.mem + key0, b, bar(ib.kX));
-        tma_load_4d(sb + SL::kX + SL::kTile + bx * SL::kBox, &tmV, bx * 64, g, ks.mem + key0, b, bar(ib.kX));
+      // checked build: the CTA's keys and KV head must lie inside the tensors
+      const bool x_ok = RA_IN_BOUNDS(ks.mem + key0, a.S) && RA_IN_BOUNDS(g, a.Hkv);
+      if (!x_ok) *abort_flag = 1;
+      if (x_ok) {
+        mbar_expect_tx(bar(ib.kX), 2 * SL::kTile);
+        for (int bx = 0; bx < D / 64; ++bx) {
+          tma_load_4d(sb + SL::kX + bx * SL::kBox, &tmK, bx * 64, g, ks.mem + key0, b, bar(ib.kX));
+          tma_load_4d(sb + SL::kX + SL::kTile + bx * SL::kBox, &tmV, bx * 64, g, ks.mem + key0, b, bar(ib.kX));
+        }
       }
       int j = 0, lastq[NQ], lasto[NO];
       for (int s = 0; s < NQ; ++s) lastq[s] = -1;
@@ -697,7 +712,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               const int hq = g * a.groups + hh, r = q_mem(s_, e_, t);
               const int sq = j % NQ, so_ = j % NO;
               // dO(j) first: dP^T(j) is issued before S^T(j)
-              if (!mbar_wait(bar(ib.empty1(so_)), ((j / NO) & 1) ^ 1, abort_flag)) {
+              if (!mbar_wait(bar(ib.empty1(so_)), ((j / NO) & 1) ^ 1, abort_flag) || !RA_IN_BOUNDS(r, a.S) ||
+                  !RA_IN_BOUNDS(hq, a.Hq)) {
+                *abort_flag = 1;
                 ok = false;
                 break;
               }
@@ -716,7 +733,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               lastq[sq] = j;
               ++j;
             }
-      mbar_drain(bar(ib.kX), 0);
+      if (x_ok) mbar_drain(bar(ib.kX), 0);
       for (int s = 0; s < NQ; ++s)
         if (lastq[s] >= 0) mbar_drain(bar(ib.full0(s)), (lastq[s] / NQ) & 1);
       for (int s = 0; s < NO; ++s)
@@ -842,7 +859,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               bwd_flush_row<D>(tmem + lane_base + kTmAcc + half * 128,
                                (half ? a.dk : a.dv) +
                                    ((static_cast<long long>(b) * a.S + ks.pos + key0 + row) * a.Hkv + g) * D,
-                               row < krows, j > kFlushTiles, half ? a.scale : 1.f);
+                               row < krows && RA_IN_BOUNDS((static_cast<long long>(b) * a.S + ks.pos + key0 + row) * a.Hkv + g,
+                                                           static_cast<long long>(a.B) * a.S * a.Hkv),
+                               j > kFlushTiles, half ? a.scale : 1.f);
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(bar(ib.fempty()));
@@ -893,7 +912,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       float* stage = reinterpret_cast<float*>(smem) + half * kBM * (D + 4);
       bwd_store_rows<D>(stage, tmem + lane_base + kTmAcc + half * 128, quad, lane, half ? a.dk : a.dv,
                         (static_cast<long long>(b) * a.S + ks.pos + key0) * a.Hkv + g, a.Hkv, D, krows,
-                        half ? a.scale : 1.f, work > kFlushTiles);
+                        half ? a.scale : 1.f, work > kFlushTiles, static_cast<long long>(a.B) * a.S * a.Hkv);
     }
   }
   tc_fence_before();

@@ -105,7 +105,9 @@ struct AttnArgs {
   void* out;
   float* lse;
   int out_bf16;
-  int fault_inject;       // 1: the producer withholds its second K tile (failure-path tests)
+  int fault_inject;       // 1: the producer withholds its second K tile (failure-path tests);
+                          // 2 (checked build only): its second K tile's row is checked out of range
+  int q_rows, kv_rows;    // rows per batch of the Q and K / V tensors the maps cover
   Seg qseg[kMaxBlocks][2];                      // segments of the i-th query block of the launch
   Seg kvseg[kMaxBlocks][2];                     // segments of KV block r
   signed char kv_list[kMaxBlocks][kMaxBlocks];  // kv_list[i][s]: s-th KV block met by query block i
@@ -336,7 +338,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int my_rows = x ? rows_b : rows_a;
     const long long row_base = a.mode == kModeFinal ? static_cast<long long>(b) * a.S + qs.pos + my_row0
                                                     : static_cast<long long>(b) * a.acc_brows + qs.mem + my_row0;
-    if (row < my_rows) {
+    const long long out_rows = a.mode == kModeFinal ? static_cast<long long>(a.B) * a.S
+                                                    : static_cast<long long>(a.B) * a.acc_brows;
+    (void)out_rows;  // read by the checks of the checked build only
+    if (row < my_rows && RA_IN_BOUNDS(row_base + row, out_rows) && RA_IN_BOUNDS(h, a.Hq)) {
       float* lse_ptr = (a.mode == kModeFinal ? a.lse : a.acc_lse) + (row_base + row) * a.Hq + h;
       if (a.mode == kModeMerge) {
         const MergeWeights mw = merge_weights(*lse_ptr, stage_l[row]);
@@ -357,6 +362,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int per = kBM / nw;
     const int wr0 = wi * per;
     const long long first = (row_base + wr0) * a.Hq + h;  // output row index of row wr0
+    if (kDebugBounds) {  // checked build: this warp's rows must lie inside the output
+      const long long out_rows = a.mode == kModeFinal ? static_cast<long long>(a.B) * a.S
+                                                      : static_cast<long long>(a.B) * a.acc_brows;
+      const int last = min(per, my_rows - wr0) - 1;
+      (void)out_rows;
+      if (last >= 0 && !(RA_IN_BOUNDS(row_base + wr0, out_rows) && RA_IN_BOUNDS(row_base + wr0 + last, out_rows) &&
+                         RA_IN_BOUNDS(h, a.Hq)))
+        return;
+    }
     const long long rstride = static_cast<long long>(a.Hq) * D;  // elements between consecutive rows
     if (a.mode == kModeFinal && a.out_bf16) {
       constexpr int lpr = D / 8, rpi = 32 / lpr;  // 16 B (8 bf16) per lane
@@ -419,11 +433,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       const int nqt = split ? 1 : 2;  // KV-split: both tiles read Q_A
-      mbar_expect_tx(bar(BQ), nqt * SL::kTile);
-      for (int x = 0; x < nqt; ++x)
-        for (int bx = 0; bx < SL::kNBox; ++bx)
-          tma_load_4d(sb + SL::kQ + x * SL::kTile + bx * SL::kBox, &tmQ, bx * 64, h, qs.mem + (x ? row0_b : row0_a), b,
-                      bar(BQ));
+      // checked build: the rows a tile uses must lie inside the Q tensor (a
+      // tile with no rows, past a short segment's end, reads TMA's zero fill)
+      bool q_ok = RA_IN_BOUNDS(h, a.Hq) && RA_IN_BOUNDS(b, a.B);
+      for (int x = 0; x < nqt; ++x) {
+        const int r0 = qs.mem + (x ? row0_b : row0_a), nr = x ? rows_b : rows_a;
+        if (nr > 0) q_ok = q_ok && RA_IN_BOUNDS(r0, a.q_rows) && RA_IN_BOUNDS(r0 + nr - 1, a.q_rows);
+        (void)r0;
+      }
+      if (!q_ok) *abort_flag = 1;  // checked build: the load is skipped and the CTA gives up
+      if (q_ok) {
+        mbar_expect_tx(bar(BQ), nqt * SL::kTile);
+        for (int x = 0; x < nqt; ++x)
+          for (int bx = 0; bx < SL::kNBox; ++bx)
+            tma_load_4d(sb + SL::kQ + x * SL::kTile + bx * SL::kBox, &tmQ, bx * 64, h,
+                        qs.mem + (x ? row0_b : row0_a), b, bar(BQ));
+      }
       int g = 0;
       bool ok = true;
       // row pairs: one walk over [lo, hi); KV-split: A's tiles [0, half) and B's
@@ -460,7 +485,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const Seg ks = seg_tab[use_b ? wb.sg : wa.sg].seg;
         const int sk = g % NSK, sv = g % NSV;
         if (!mbar_wait(bar(BKE(sk)), ((g / NSK) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        if (!(a.fault_inject && g == 1)) {  // an injected fault: this K tile never arrives
+        // checked build: the tile's row and heads must lie inside the K / V tensors
+        const int row_chk = ks.mem + t * kBN + (kDebugBounds && a.fault_inject == 2 && g == 1 ? a.kv_rows : 0);
+        (void)row_chk;
+        if (!(RA_IN_BOUNDS(row_chk, a.kv_rows) && RA_IN_BOUNDS(hk, a.Hkv) && RA_IN_BOUNDS(use_b ? wb.sg : wa.sg, nsg))) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        if (!(a.fault_inject == 1 && g == 1)) {  // an injected fault: this K tile never arrives
           mbar_expect_tx(bar(BKF(sk)), SL::kTile);
           for (int bx = 0; bx < SL::kNBox; ++bx)
             tma_load_4d(sb + SL::kK + sk * SL::kTile + bx * SL::kBox, &tmK, bx * 64, hk, ks.mem + t * kBN, b,
@@ -478,7 +511,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         else walk_next(wa);
       }
       if (!ok) {  // let every copy already issued land before shared memory is released
-        mbar_drain(bar(BQ), 0);
+        if (q_ok) mbar_drain(bar(BQ), 0);
         for (int s = 0; s < NSK; ++s)
           if (issued_k[s] >= 0) mbar_drain(bar(BKF(s)), (issued_k[s] / NSK) & 1);
         for (int s = 0; s < NSV; ++s)

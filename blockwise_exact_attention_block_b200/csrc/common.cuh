@@ -18,6 +18,30 @@ __device__ int g_status;
 
 __device__ __forceinline__ void set_status(int s) { atomicCAS(&g_status, 0, s); }
 
+// Index checks of the checked build (compiled with -DRA_DEBUG_BOUNDS): a
+// failed check records RA_ERR_DEVICE_BOUNDS in the status word (the first
+// error wins) with the source line, the index and its limit, and the caller
+// skips the access.  The release build compiles every check to `true`.
+#ifdef RA_DEBUG_BOUNDS
+__device__ long long g_bounds_record[3];  // line, index, limit of the first failed check
+__device__ __noinline__ bool bounds_failed(long long idx, long long limit, int line) {
+  if (atomicCAS(&g_status, 0, RA_ERR_DEVICE_BOUNDS) == 0) {
+    g_bounds_record[0] = line;
+    g_bounds_record[1] = idx;
+    g_bounds_record[2] = limit;
+  }
+  return false;
+}
+#define RA_IN_BOUNDS(idx, limit)                                                                          \
+  ((static_cast<long long>(idx) >= 0 && static_cast<long long>(idx) < static_cast<long long>(limit)) \
+       ? true                                                                                             \
+       : ::ra::bounds_failed(static_cast<long long>(idx), static_cast<long long>(limit), __LINE__))
+constexpr bool kDebugBounds = true;
+#else
+#define RA_IN_BOUNDS(idx, limit) true
+constexpr bool kDebugBounds = false;
+#endif
+
 // A bounded wait gives up after this many SM clock cycles (about one second
 // at the B200's 1.9 GHz boost clock) and reports RA_ERR_TIMEOUT.
 constexpr long long kWaitLimitCycles = 2000000000LL;

@@ -40,10 +40,12 @@ __global__ void __launch_bounds__(kMergeThreads)
     float4 ov[V], bv[V];
     float la[V], lb[V];
     long long iv[V];
+    bool act[V];
 #pragma unroll
     for (int u = 0; u < V; ++u) {
       iv[u] = base + 32 * u + lane;
-      if (iv[u] < nvec) {
+      act[u] = iv[u] < nvec && RA_IN_BOUNDS(iv[u] / vpr, rows);
+      if (act[u]) {
         const long long row = iv[u] / vpr;
         ov[u] = o4[iv[u]];
         bv[u] = __ldcs(b4 + iv[u]);
@@ -54,7 +56,7 @@ __global__ void __launch_bounds__(kMergeThreads)
     __syncwarp();  // every lane has read lse[row] before any lane rewrites it
 #pragma unroll
     for (int u = 0; u < V; ++u) {
-      if (iv[u] < nvec) {
+      if (act[u]) {
         const MergeWeights mw = merge_weights(la[u], lb[u]);
         float4 r;
         r.x = merge_out(ov[u].x, bv[u].x, mw.w);
@@ -97,7 +99,7 @@ __global__ void __launch_bounds__(kMergeThreads)
 #pragma unroll
     for (int u = 0; u < V; ++u) {
       iv[u] = base + 32 * u + lane;
-      act[u] = iv[u] < nvec;
+      act[u] = iv[u] < nvec && RA_IN_BOUNDS(iv[u] / vpr, rows);
       row[u] = act[u] ? iv[u] / vpr : 0;
       if (act[u]) {
 #pragma unroll

@@ -115,7 +115,10 @@ typedef struct {
    * (about 1 s of SM clocks): the kernel records RA_ERR_TIMEOUT in the device
    * status word, every CTA stops at its next wait, in-flight copies and
    * products are drained, and the call's outputs are undefined.  The context
-   * stays usable.  Other values: RA_ERR_INVALID_ARG. */
+   * stays usable.  2 (checked build only, see ra_debug_build): the producer
+   * checks its second K tile's row as if it lay past the end of the tensor;
+   * the check records RA_ERR_DEVICE_BOUNDS, the copy is skipped and the CTA
+   * stops.  Other values: RA_ERR_INVALID_ARG. */
   int fault_inject;
 } ra_options;
 
@@ -353,6 +356,23 @@ const char* ra_status_string(ra_status s);
 
 /* Library version string. */
 const char* ra_version(void);
+
+/*
+ * The checked build.  libra_b200_debug.so is this library compiled with
+ * -DRA_DEBUG_BOUNDS: before every run-time-indexed global access (the rows
+ * and heads of TMA copies, output rows, lse and Delta entries, merge rows) and
+ * every segment-table read, the kernels check the index against the extent it
+ * must lie in.  A failed check records RA_ERR_DEVICE_BOUNDS in the device
+ * status word (ra_get_device_status), skips the access and ends the CTA's work;
+ * nothing traps.  Not part of the method on the pages: a debugging aid.
+ *
+ * ra_debug_build: 1 in the checked build, 0 otherwise.
+ * ra_get_bounds_record: the first failed check since the last read (source
+ *   line, index, limit; zeros if none, and always zeros in the release
+ *   build), then clears it.  Synchronous.  record: host, 3 entries.
+ */
+int ra_debug_build(void);
+ra_status ra_get_bounds_record(int64_t record[3]);
 
 #ifdef __cplusplus
 }

@@ -255,3 +255,22 @@ def test_c_caller_links_and_runs(ra, tmp_path):
     run = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert run.returncode == 0, run.stderr
     assert run.stdout.startswith("ok ")
+
+
+def test_release_build_is_not_the_checked_build(ra):
+    # the checked build is a separate library (libra_b200_debug.so); the
+    # release one reports 0, has no bounds record, and rejects the checked
+    # build's injected out-of-range row before any launch
+    assert ra.ra_debug_build() is False
+    assert ra.ra_get_bounds_record() == (0, 0, 0)
+    inj = ra.ra_options(0, ra.RA_SCHED_AUTO, None, None, 0, 2)
+    assert ring(ra, opts=ctypes.byref(inj)) == ra.RA_ERR_INVALID_ARG
+
+
+def test_checked_build_exports_the_same_symbols(ra):
+    import __graft_entry__
+    mod = __graft_entry__._build_module()
+    path = mod.build(debug_bounds=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (ra_\w+)", out))
+    assert not [n for n in declared_functions() if n not in exported]
