@@ -75,10 +75,18 @@ struct MergeList {
   const float* lses[kMaxMergeInputs];
 };
 
-// k = K partials folded left to right on chip; one write of the result.
+// k = K partials merged on chip; one write of the result.  Folding the
+// update rule left to right k - 1 times gives, for every row,
+//     lse = ln sum_j exp(lse_j),   out = sum_j exp(lse_j - lse) * out_j,
+// the softmax merge of the k partials; this kernel evaluates that closed
+// form (maximum, sum of exponentials, one logarithm, weighted sum), whose k
+// exponentials are independent, instead of a chain of k - 1 dependent rule
+// applications (the chain left the k = 16 kernel bound by instruction
+// latency).  Partials with lse = -inf get weight 0; when every partial is
+// empty the state stays partial 0, as the fold leaves it.
 // K is a compile-time constant so that every partial's load is issued before
-// the first one is folded in (K loads in flight per vector); V vectors per
-// lane and sweep (2 for K <= 4, where K alone keeps few loads in flight).
+// any is used (K loads in flight per vector); V vectors per lane and sweep (2
+// for K <= 4, where K alone keeps few loads in flight).
 // out / lse may alias outs[0] / lses[0]: every lane reads its row's lse before
 // the warp rewrites it (the lanes of a row share a warp; see the top note).
 template <int K>
@@ -114,16 +122,31 @@ __global__ void __launch_bounds__(kMergeThreads)
 #pragma unroll
     for (int u = 0; u < V; ++u) {
       if (!act[u]) continue;
-      float4 acc = v[u][0];
-      float la = l[u][0];
+      float m = l[u][0];
 #pragma unroll
-      for (int j = 1; j < K; ++j) {
-        const MergeWeights mw = merge_weights(la, l[u][j]);
-        acc.x = merge_out(acc.x, v[u][j].x, mw.w);
-        acc.y = merge_out(acc.y, v[u][j].y, mw.w);
-        acc.z = merge_out(acc.z, v[u][j].z, mw.w);
-        acc.w = merge_out(acc.w, v[u][j].w, mw.w);
-        la = mw.lse;
+      for (int j = 1; j < K; ++j) m = fmaxf(m, l[u][j]);
+      float4 acc = v[u][0];
+      float la = -INFINITY;
+      if (m != -INFINITY) {
+        float e[K], ssum = 0.f;
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+          e[j] = expf(l[u][j] - m);  // 0 for an empty partial
+          ssum += e[j];
+        }
+        const float inv = 1.f / ssum;
+        acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+          const float w = e[j] * inv;
+          if (w != 0.f) {
+            acc.x = fmaf(w, v[u][j].x, acc.x);
+            acc.y = fmaf(w, v[u][j].y, acc.y);
+            acc.z = fmaf(w, v[u][j].z, acc.z);
+            acc.w = fmaf(w, v[u][j].w, acc.w);
+          }
+        }
+        la = m + logf(ssum);
       }
       reinterpret_cast<float4*>(out)[iv[u]] = acc;
       if (iv[u] % vpr == 0) lse[row[u]] = la;
