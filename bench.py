@@ -7,15 +7,16 @@
 
 One step = one ra_ring_attention call over the workload (partition of Q, K, V
 into block order, block attention over every (query block, KV block) pair in
-schedule order with the merge rule, output in original order).  The metric is
-causal-adjusted attention throughput, 4 * B * Hq * D * P FLOPs per step with P
-the number of visible (query, key) pairs.  Inputs are resident in HBM when the
-timed region starts; L2 is flushed (a 256 MiB write) between timed steps,
-outside the timed events.  Each step is timed on the device with CUDA events;
-the attention kernel inside the call is timed with a second pair of events
-recorded by the library around its launch.  With N GPUs each rank runs the
-same workload on its own GPU (replicas, weak scaling; the method needs no
-exchange on one node here) and the slowest rank's time counts.
+schedule order with the merge rule, output in original order).  The default
+workload is the 1M-token one (the largest that fits one GPU); the 4k and 24k
+workloads are timed the same way beside it, each in its own sub-object.  The
+metric is causal-adjusted attention throughput, 4 * B * Hq * D * P FLOPs per
+step with P the number of visible (query, key) pairs.  Inputs are resident in
+HBM when the timed region starts; L2 is flushed between timed steps (a
+256 MiB write, then read back), outside the timed events.  Each step is timed
+on the device with CUDA events on the launching stream.  With N GPUs each rank
+runs the same workload on its own GPU (replicas, weak scaling; the method needs
+no exchange on one node here) and the slowest rank's time counts.
 
 --impl reference times the CPU fp64 oracle on the host cores instead (a
 bounded sample of the same workload).  --backward, --decode, --merge-sweep
