@@ -91,6 +91,9 @@ def parse():
     p.add_argument("--backward-workload", default="gqa24k", choices=sorted(WORKLOADS),
                    help="workload of the backward object on the default line")
     p.add_argument("--no-side", action="store_true", help="time only --workload (no other attention workloads)")
+    p.add_argument("--cta-timeline", action="store_true",
+                   help="record where every CTA of the forward (and with --backward, of the two backward "
+                        "kernels) ran, once, after warm-up; print a per-kernel summary instead")
     p.add_argument("--shards", action="store_true",
                    help="time the sequence-parallel rank programs (one block per rank), all ranks on one GPU")
     a = p.parse_args()
@@ -897,30 +900,35 @@ def run_ours(args):
 
     merge = None
     if not args.no_merge:
+        mclk = Clocks(local_gpu_id(dev))
         gbs, mms = bench_merge(ra, dev, 1048576, 2, 10, flush)
         merge = {"kernel": "merge_partial_kernel", "tokens": 1048576, "heads": 32, "D": 128, "partials": 2,
                  "GB/s": gbs, "ms": mms, "peak_GB/s": pk["hbm_gbs"], "frac": gbs / pk["hbm_gbs"],
-                 "bytes_per_row": 12 * 128 + 12}
+                 "bytes_per_row": 12 * 128 + 12, "clocks": mclk.stop()}
 
     decode = None
     if not args.no_decode and world == 1:
         from seeded_inputs import DECODE_WORKLOADS
         dw = DECODE_WORKLOADS["decode1m"]
+        dclk = Clocks(local_gpu_id(dev))
         gbs, dms, splits = bench_decode(ra, dev, dw, 10, flush)
         decode = {"kernel": "decode_partial_kernel + decode_combine_kernel", "workload": "decode1m", "B": dw.B,
                   "Tq": dw.Tq, "Skv": dw.Skv, "Hq": dw.Hq, "Hkv": dw.Hkv, "D": dw.D, "chunks": splits,
-                  "GB/s": gbs, "ms": dms, "peak_GB/s": pk["hbm_gbs"], "frac": gbs / pk["hbm_gbs"]}
+                  "GB/s": gbs, "ms": dms, "peak_GB/s": pk["hbm_gbs"], "frac": gbs / pk["hbm_gbs"],
+                  "clocks": dclk.stop()}
 
     backward = None
     if not args.no_backward and world == 1:
         bw = WORKLOADS[args.backward_workload]
+        bclk = Clocks(local_gpu_id(dev))
         tf, ktf, bms, bkms = bench_backward(ra, dev, bw, 20 if bw.S <= 32768 else 2, flush, args.order)
+        bclk = bclk.stop()
         bpeak = pk["bf16_tflops_sustained" if bkms > 100.0 else "bf16_tflops"]
         brec = attn_traffic(bw.name, "attn_bwd_traffic.json", BWD_SOURCES)
         backward = {"kernel": "bwd_dkv_kernel + bwd_dq_kernel (+ bwd_prep_kernel in the call)",
                     "workload": bw.name, "flops_per_step": 2.5 * bw.flops, "TFLOP/s": tf, "kernels_TFLOP/s": ktf,
                     "ms": bms, "kernels_ms": bkms, "peak_TFLOP/s": bpeak, "frac": ktf / bpeak,
-                    "traffic": brec["dram_bytes_per_launch"] if brec else None}
+                    "traffic": brec["dram_bytes_per_launch"] if brec else None, "clocks": bclk}
     status = status or ra.ra_get_device_status()
 
     value = replica_throughput(w.flops, world, K, total_ms)
@@ -974,10 +982,102 @@ def run_merge_sweep(args):
     return 0
 
 
+def timeline_summary(rec, event_ms):
+    """Summary of one launch's per-CTA records (start ns, end ns, SM id | work
+    units << 32, SM cycles): span, the heaviest CTA, a least-squares fit of
+    CTA duration to work units, how many CTAs started after the first wave,
+    and the SM clock the CTAs ran at (cycles over time)."""
+    import numpy as np
+    r = rec[rec[:, 1] > 0]
+    t0 = int(r[:, 0].min())
+    start, end = (r[:, 0] - t0) / 1e3, (r[:, 1] - t0) / 1e3
+    sm = r[:, 2] & 0xFFFFFFFF
+    dur, work = end - start, (r[:, 2] >> 32).astype(float)
+    mhz = float(r[:, 3].sum()) / max(float(dur.sum()), 1e-9)
+    span = float(end.max())
+    i = int(np.argmax(dur))
+    A = np.stack([np.ones_like(work), work], 1)
+    fit = np.linalg.lstsq(A, dur, rcond=None)[0]
+    later = start > 2.0
+    n_sm = len(set(sm.tolist()))
+    return {"ctas": int(len(r)), "sms": n_sm, "event_us": event_ms * 1e3, "span_us": span,
+            "launch_overhead_us": event_ms * 1e3 - span,
+            "heaviest_cta": {"work": int(work[i]), "us": float(dur[i]), "of_span": float(dur[i]) / span},
+            "fit_us": {"fixed": float(fit[0]), "per_unit": float(fit[1])},
+            "ctas_after_first_wave": int(later.sum()),
+            "last_end_of_first_wave_us": float(end[~later].max()),
+            "mean_sm_busy_us": float(dur.sum()) / n_sm,
+            "work_units": int(work.sum()),
+            "sm_mhz_in_ctas": mhz,
+            "cycles_per_unit": float(fit[1]) * mhz}
+
+
+def run_cta_timeline(args):
+    """--cta-timeline: after warm-up, one launch of each kernel with the
+    per-CTA timeline on (ra_set_cta_timeline), summarised.  Times in us."""
+    import torch
+    import blockwise_exact_attention_block_b200 as ra
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    flush = L2Flush(dev)
+    w = WORKLOADS[args.workload]
+    q, k, v = (x.to(dev) for x in workload_inputs(w))
+    odt = torch.bfloat16 if w.out_dtype == "bf16" else torch.float32
+    rec = torch.zeros((1 << 16, 4), dtype=torch.int64, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd(events=None):
+        return ra.ra_ring_attention(q, k, v, w.n_blocks, w.causal, w.partition, w.gqa_groups, out_dtype=odt,
+                                    order=args.order, sched=args.sched, tiling=args.tiling, attn_events=events)
+
+    calls = {"attn_fwd": fwd}
+    if args.backward:
+        from seeded_inputs import backward_inputs
+        _, _, _, do = backward_inputs(w.B, w.S, w.Hq, w.Hkv, w.D, w.in_dtype, seed=10)
+        do = do.to(dev)
+        o, l = fwd()
+
+        def bwd(events=None):
+            return ra.ra_ring_attention_backward(q, k, v, o, l, do, w.n_blocks, w.causal, w.partition, w.gqa_groups,
+                                                 order=args.order, attn_events=events)
+        calls["bwd_dkv"] = calls["bwd_dq"] = bwd
+    clocks = Clocks(local_gpu_id(dev))
+    out = {}
+    for name, fn in calls.items():
+        for _ in range(args.warmup + args.steps):  # warm-up, and clocks up to their load level
+            flush()
+            fn()
+        best = None
+        for _ in range(3):
+            flush()
+            rec.zero_()
+            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            ra.ra_set_cta_timeline(rec, name)
+            try:
+                fn(ev)
+                torch.cuda.synchronize()
+            finally:
+                ra.ra_set_cta_timeline(None)
+            summ = timeline_summary(rec.cpu().numpy(), ev[0].elapsed_time(ev[1]))
+            if best is None or summ["span_us"] < best["span_us"]:
+                best = summ
+        out[name] = best
+    clk = clocks.stop()
+    status = ra.ra_get_device_status()
+    line = {"metric": "per-CTA timeline", "config": workload_config(w, args, L2_FLUSH_DESC), "kernels": out,
+            "note": "the launch with the shortest CTA span of three; event_us from events the library records "
+                    "around the kernels (the backward's pair of kernels for both backward entries)",
+            "clocks": clk, "device_status": ra.ra_status_string(status)}
+    print(json.dumps(line))
+    return 0 if status == 0 else 1
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.cta_timeline:
+        return run_cta_timeline(args)
     if args.merge_sweep:
         return run_merge_sweep(args)
     if args.decode:

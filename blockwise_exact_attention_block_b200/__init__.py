@@ -50,7 +50,11 @@ EXPORTED = ["ra_block_attn", "ra_block_attn_merge", "ra_merge_partial", "ra_merg
             "ra_ring_attention_workspace", "ra_zigzag_permute", "ra_get_device_status",
             "ra_status_string", "ra_version", "ra_ring_attention_noalloc", "ra_noalloc_scratch_bytes",
             "ra_decode_attention", "ra_decode_workspace", "ra_decode_splits", "ra_ring_attention_backward",
-            "ra_ring_attention_backward_workspace", "ra_debug_build", "ra_get_bounds_record"]
+            "ra_ring_attention_backward_workspace", "ra_debug_build", "ra_get_bounds_record",
+            "ra_set_cta_timeline"]
+
+RA_TIMELINE_ATTN_FWD, RA_TIMELINE_BWD_DKV, RA_TIMELINE_BWD_DQ = 0, 1, 2
+TIMELINE_KERNELS = {"attn_fwd": RA_TIMELINE_ATTN_FWD, "bwd_dkv": RA_TIMELINE_BWD_DKV, "bwd_dq": RA_TIMELINE_BWD_DQ}
 
 
 class ra_options(ctypes.Structure):
@@ -103,6 +107,8 @@ _lib.ra_debug_build.argtypes = []
 _lib.ra_debug_build.restype = _i
 _lib.ra_get_bounds_record.argtypes = [ctypes.POINTER(ctypes.c_int64)]
 _lib.ra_get_bounds_record.restype = _i
+_lib.ra_set_cta_timeline.argtypes = [_vp, _i64, _i]
+_lib.ra_set_cta_timeline.restype = _i
 
 
 class RAError(RuntimeError):
@@ -135,6 +141,24 @@ def ra_get_bounds_record() -> tuple[int, int, int]:
     rec = (ctypes.c_int64 * 3)()
     _check(_lib.ra_get_bounds_record(rec), "ra_get_bounds_record")
     return int(rec[0]), int(rec[1]), int(rec[2])
+
+
+def ra_set_cta_timeline(records: torch.Tensor | None, kernel: str = "attn_fwd") -> None:
+    """Per-CTA timeline of one kernel's following launches (tracing).
+
+    records: a contiguous int64 CUDA tensor [max_ctas, 4] that receives, per
+    CTA, (start ns, end ns, SM id, work units); None turns the timeline off.
+    kernel: "attn_fwd", "bwd_dkv" or "bwd_dq".  The tensor must stay alive
+    until the launches that write it have completed."""
+    if kernel not in TIMELINE_KERNELS:
+        raise ValueError(f"unknown kernel {kernel!r}")
+    if records is None:
+        _check(_lib.ra_set_cta_timeline(None, 0, TIMELINE_KERNELS[kernel]), "ra_set_cta_timeline")
+        return
+    if records.dtype != torch.int64 or records.dim() != 2 or records.shape[1] != 4:
+        raise ValueError("records must be an int64 tensor [max_ctas, 4]")
+    _check(_lib.ra_set_cta_timeline(_ptr(records), records.shape[0], TIMELINE_KERNELS[kernel]),
+           "ra_set_cta_timeline")
 
 
 def _stream(stream=None) -> int:

@@ -118,9 +118,24 @@ void choose_tiling(const Geom& g, AttnArgs& a, ra_tiling tiling) {
   a.seg_tiles = (len + (a.kv_split ? kBM : kCtaRows) - 1) / (a.kv_split ? kBM : kCtaRows);
 }
 
+// The per-CTA timeline set by ra_set_cta_timeline (process-wide; off while
+// rec is null): the one kernel it is recorded for, its records and their count.
+struct TimelineState {
+  unsigned long long* rec;
+  int max_ctas;
+  int kernel;
+};
+TimelineState g_timeline = {nullptr, 0, 0};
+
+CtaTimeline timeline_for(int kernel) {
+  if (g_timeline.rec == nullptr || g_timeline.kernel != kernel) return CtaTimeline{nullptr, 0};
+  return CtaTimeline{g_timeline.rec, g_timeline.max_ctas};
+}
+
 AttnArgs base_args(const Geom& g) {
   AttnArgs a;
   memset(&a, 0, sizeof(a));
+  a.timeline = timeline_for(RA_TIMELINE_ATTN_FWD);
   a.B = g.B;
   a.S = g.S;
   a.Hq = g.Hq;
@@ -552,6 +567,20 @@ const char* ra_version(void) { return "ra_b200 0.1 (sm_100a)"; }
 
 int ra_debug_build(void) { return kDebugBounds ? 1 : 0; }
 
+ra_status ra_set_cta_timeline(uint64_t* records, int64_t max_ctas, ra_timeline_kernel kernel) {
+  if (kernel != RA_TIMELINE_ATTN_FWD && kernel != RA_TIMELINE_BWD_DKV && kernel != RA_TIMELINE_BWD_DQ)
+    return RA_ERR_INVALID_ARG;
+  if (records == nullptr) {
+    g_timeline = TimelineState{nullptr, 0, 0};
+    return RA_OK;
+  }
+  if (max_ctas < 1 || max_ctas > (int64_t{1} << 24) || (reinterpret_cast<uintptr_t>(records) & 7u) != 0)
+    return RA_ERR_INVALID_ARG;
+  g_timeline = TimelineState{reinterpret_cast<unsigned long long*>(records), static_cast<int>(max_ctas),
+                             static_cast<int>(kernel)};
+  return RA_OK;
+}
+
 ra_status ra_get_bounds_record(int64_t record[3]) {
   if (!record) return RA_ERR_INVALID_ARG;
   record[0] = record[1] = record[2] = 0;
@@ -979,6 +1008,8 @@ ra_status ra_ring_attention_backward(const void* q, const void* k, const void* v
   // forward); dK/dV: KV block j meets the query blocks that meet it there
   const ra_order order = opts ? opts->order : RA_ORDER_RING;
   BwdArgs adq = a, adkv = a;
+  adq.timeline = timeline_for(RA_TIMELINE_BWD_DQ);
+  adkv.timeline = timeline_for(RA_TIMELINE_BWD_DKV);
   for (int r = 0; r < g.n; ++r)
     for (int t = 0; t < g.n; ++t) {
       const int fwd = order == RA_ORDER_RING ? r - t : r + t;

@@ -67,6 +67,7 @@ struct BwdArgs {
   Seg seg[kMaxBlocks][2];                     // segments of block r (queries and keys alike)
   signed char order[kMaxBlocks][kMaxBlocks];  // order[r][s]: s-th block that block r meets
   signed char seg_order[2 * kMaxBlocks];      // (r * nseg + e) of the CTA segments, heaviest first
+  CtaTimeline timeline;  // per-CTA tracing (rec == nullptr: off); work units = tiles walked
 };
 
 // Shared memory of the dQ kernel: Q and dO stay; K and V stream through
@@ -369,6 +370,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* smem = bsm_raw + ((1024u - (smem_u32(bsm_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  timeline_begin(a.timeline);
 
   // tile: heads fastest, then batch, then query segments heaviest first,
   // then tiles of the segment, latest first
@@ -408,6 +410,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + SL::kTmemSlot);
   const int work = *abort_flag || rows == 0 ? 0 : total;
+  timeline_work(a.timeline, work);
 
   if (warp == kBwdProducer) {
     if (lane == 0 && work > 0) {
@@ -610,6 +613,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == kBwdMma) tmem_dealloc(tmem, 512);
+  timeline_end(a.timeline);
 }
 
 // ----------------------------------------------------------------- dK, dV
@@ -631,6 +635,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* smem = bsm_raw + ((1024u - (smem_u32(bsm_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  timeline_begin(a.timeline);
 
   // tile: KV heads fastest, then batch, then key segments heaviest first,
   // then tiles of the segment, earliest first
@@ -682,6 +687,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + SL::kTmemSlot);
   const int work = *abort_flag || krows == 0 ? 0 : total;
+  timeline_work(a.timeline, work);
 
   if (warp == kBwdProducer) {
     if (lane == 0 && work > 0) {
@@ -919,6 +925,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == kBwdMma) tmem_dealloc(tmem, 512);
+  timeline_end(a.timeline);
 }
 
 }  // namespace ra

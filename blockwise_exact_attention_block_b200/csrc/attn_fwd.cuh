@@ -108,6 +108,7 @@ struct AttnArgs {
   int fault_inject;       // 1: the producer withholds its second K tile (failure-path tests);
                           // 2 (checked build only): its second K tile's row is checked out of range
   int q_rows, kv_rows;    // rows per batch of the Q and K / V tensors the maps cover
+  CtaTimeline timeline;   // per-CTA tracing (rec == nullptr: off); work units = KV tiles
   Seg qseg[kMaxBlocks][2];                      // segments of the i-th query block of the launch
   Seg kvseg[kMaxBlocks][2];                     // segments of KV block r
   signed char kv_list[kMaxBlocks][kMaxBlocks];  // kv_list[i][s]: s-th KV block met by query block i
@@ -205,6 +206,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  timeline_begin(a.timeline);
 
   // ---- tile decode: heads fastest (heads of one KV group share K/V in L2),
   // then batch, then query tiles in decreasing position (heaviest first).
@@ -314,6 +316,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int lo = kCl > 1 ? crank * total / kCl : 0;
   const int hi = kCl > 1 ? (crank + 1) * total / kCl : total;
   int work = hi - lo;
+  timeline_work(a.timeline, work);
   // Tile x's share of the CTA's KV tiles.  u = index in the CTA's sequence,
   // t = index inside the segment.  KV-split: A takes [0, half), B [half, total).
   const int half = (total + 1) / 2;
@@ -889,6 +892,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+  timeline_end(a.timeline);
 }
 
 }  // namespace ra

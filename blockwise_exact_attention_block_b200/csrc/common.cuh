@@ -42,6 +42,50 @@ constexpr bool kDebugBounds = true;
 constexpr bool kDebugBounds = false;
 #endif
 
+// Per-CTA timeline (tracing, off unless the host sets it for one kernel): the
+// CTA's thread 0 writes four 64-bit words at rec[4 * blockIdx.x] for the CTAs
+// below max_ctas: start and end in ns of the global timer, the SM id (low 32
+// bits) with the CTA's work units (the tiles of its walk, high 32 bits), and
+// the SM clock cycles from start to end (the fourth word holds the start
+// cycle count until the end stamp replaces it by the difference).
+struct CtaTimeline {
+  unsigned long long* rec;
+  int max_ctas;
+};
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ bool timeline_on(const CtaTimeline& t) {
+  return t.rec != nullptr && threadIdx.x == 0 && static_cast<int>(blockIdx.x) < t.max_ctas;
+}
+
+__device__ __forceinline__ void timeline_begin(const CtaTimeline& t) {
+  if (timeline_on(t)) {
+    t.rec[4ull * blockIdx.x] = global_ns();
+    t.rec[4ull * blockIdx.x + 3] = static_cast<unsigned long long>(clock64());
+  }
+}
+
+__device__ __forceinline__ void timeline_work(const CtaTimeline& t, int units) {
+  if (timeline_on(t)) {
+    unsigned int sm;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+    t.rec[4ull * blockIdx.x + 2] = sm | (static_cast<unsigned long long>(static_cast<unsigned int>(units)) << 32);
+  }
+}
+
+__device__ __forceinline__ void timeline_end(const CtaTimeline& t) {
+  if (timeline_on(t)) {
+    unsigned long long* r = t.rec + 4ull * blockIdx.x;
+    r[3] = static_cast<unsigned long long>(clock64()) - r[3];
+    r[1] = global_ns();
+  }
+}
+
 // A bounded wait gives up after this many SM clock cycles (about one second
 // at the B200's 1.9 GHz boost clock) and reports RA_ERR_TIMEOUT.
 constexpr long long kWaitLimitCycles = 2000000000LL;

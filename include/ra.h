@@ -374,6 +374,42 @@ const char* ra_version(void);
 int ra_debug_build(void);
 ra_status ra_get_bounds_record(int64_t record[3]);
 
+/*
+ * Per-CTA timeline (tracing).  TokenRing's per-attention-step latencies
+ * (Figure 6) were read off Nsight Systems profiles ([TR] "Referee Report",
+ * major comments; "Circularity Check"); this is the same kind of view one
+ * level down: where each CTA of one tensor-core kernel ran and for how long.
+ * Not part of the method: a profiling aid, off by default.
+ *
+ *  records   device, uint64 [max_ctas][4], 8-byte aligned, owned by the
+ *            caller; NULL turns the timeline off (then max_ctas is ignored).
+ *  max_ctas  1 .. 2^24: CTAs with blockIdx.x < max_ctas record.
+ *  kernel    which kernel records: RA_TIMELINE_ATTN_FWD (attn_fwd_kernel:
+ *            every block-attention launch of ra_block_attn*, ra_ring_attention*),
+ *            RA_TIMELINE_BWD_DKV or RA_TIMELINE_BWD_DQ (the two tensor-core
+ *            kernels of ra_ring_attention_backward*).
+ *
+ * While set, every launch of that kernel writes, for its CTA i < max_ctas,
+ * records[i][0..3] = start and end in ns of the GPU's global timer; the SM id
+ * (low 32 bits) and the CTA's work units (high 32 bits: KV tiles walked for
+ * attn_fwd_kernel and the dQ kernel, query tiles walked for the dK/dV
+ * kernel); and the SM clock cycles from start to end (their ratio to the
+ * duration is the clock the CTA ran at).  Each launch overwrites the
+ * records of the CTAs it has; a CTA whose work ends early (an abort) may
+ * leave its end word unwritten.  The setting is process-wide, applies to the
+ * calls made after it on any stream and device, and is not synchronised with
+ * calls running on other host threads; records must stay valid until those
+ * launches have completed.  Host-only: returns RA_OK, or RA_ERR_INVALID_ARG
+ * for an unknown kernel, max_ctas out of range or a misaligned pointer.
+ */
+typedef enum {
+  RA_TIMELINE_ATTN_FWD = 0,
+  RA_TIMELINE_BWD_DKV = 1,
+  RA_TIMELINE_BWD_DQ = 2
+} ra_timeline_kernel;
+
+ra_status ra_set_cta_timeline(uint64_t* records, int64_t max_ctas, ra_timeline_kernel kernel);
+
 #ifdef __cplusplus
 }
 #endif

@@ -274,3 +274,25 @@ def test_checked_build_exports_the_same_symbols(ra):
     out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True).stdout
     exported = set(re.findall(r" T (ra_\w+)", out))
     assert not [n for n in declared_functions() if n not in exported]
+
+
+def test_cta_timeline_setter_validates_on_the_host(ra):
+    # host-only: the setter records the buffer for later launches and
+    # launches nothing itself; every case ends with the timeline off
+    lib = ra._lib
+    fake = 0x10000  # never dereferenced: no launch follows while it is set
+    try:
+        assert lib.ra_set_cta_timeline(None, 0, 0) == ra.RA_OK
+        assert lib.ra_set_cta_timeline(None, 0, 7) == ra.RA_ERR_INVALID_ARG   # unknown kernel
+        assert lib.ra_set_cta_timeline(fake, 0, 0) == ra.RA_ERR_INVALID_ARG   # no records
+        assert lib.ra_set_cta_timeline(fake, -1, 1) == ra.RA_ERR_INVALID_ARG
+        assert lib.ra_set_cta_timeline(fake, (1 << 24) + 1, 2) == ra.RA_ERR_INVALID_ARG
+        assert lib.ra_set_cta_timeline(fake + 4, 16, 0) == ra.RA_ERR_INVALID_ARG  # misaligned
+        for kernel in (0, 1, 2):
+            assert lib.ra_set_cta_timeline(fake, 16, kernel) == ra.RA_OK
+    finally:
+        assert lib.ra_set_cta_timeline(None, 0, 0) == ra.RA_OK
+    with pytest.raises(ValueError):
+        ra.ra_set_cta_timeline(None, "no_such_kernel")
+    with pytest.raises(ValueError):
+        ra.ra_set_cta_timeline(torch.zeros((4, 3), dtype=torch.int64), "attn_fwd")

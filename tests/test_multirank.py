@@ -124,3 +124,31 @@ def test_shard_exchange_bytes():
     w = WORKLOADS["gqa24k"]  # 24,000 tokens, 4 blocks of 6,000, 32 query / 8 KV heads, D = 128
     assert bench.shard_exchange_bytes(w, "ring") == 2 * 6000 * 8 * 128 * 2
     assert bench.shard_exchange_bytes(w, "tokenring") == 6000 * 32 * 128 * 2 + 6000 * 32 * 129 * 4
+
+
+def test_timeline_summary_on_a_known_schedule():
+    # three SMs, five CTAs: CTA cost 2 us + 1 us per work unit; two CTAs start
+    # after the first wave on the SMs that free up first
+    import numpy as np
+    import bench
+    t0 = 10**12
+    rows = []  # start ns, end ns, SM, work
+    for sm, (start, work) in enumerate([(0.0, 6), (0.0, 3), (0.0, 2)]):
+        rows.append((start, start + 2 + work, sm, work))
+    rows.append((4.0, 4.0 + 2 + 1, 2, 1))   # after SM 2's first CTA (ends at 4)
+    rows.append((5.0, 5.0 + 2 + 0, 1, 0))   # after SM 1's first CTA (ends at 5)
+    # 1,500 cycles per us: a 1.5 GHz clock
+    rec = np.array([(t0 + int(a * 1e3), t0 + int(b * 1e3), sm | (w << 32), int((b - a) * 1500))
+                    for a, b, sm, w in rows] + [(0, 0, 0, 0)] * 3, dtype=np.int64)
+    s = bench.timeline_summary(rec, event_ms=0.0105)
+    assert s["ctas"] == 5 and s["sms"] == 3
+    assert abs(s["span_us"] - 8.0) < 1e-9
+    assert abs(s["launch_overhead_us"] - 2.5) < 1e-9
+    assert s["heaviest_cta"] == {"work": 6, "us": 8.0, "of_span": 1.0}
+    assert abs(s["fit_us"]["fixed"] - 2.0) < 1e-9 and abs(s["fit_us"]["per_unit"] - 1.0) < 1e-9
+    assert s["ctas_after_first_wave"] == 2
+    assert abs(s["last_end_of_first_wave_us"] - 8.0) < 1e-9
+    assert abs(s["mean_sm_busy_us"] - (8 + 5 + 4 + 3 + 2) / 3) < 1e-9
+    assert s["work_units"] == 12
+    assert abs(s["sm_mhz_in_ctas"] - 1500.0) < 1e-6
+    assert abs(s["cycles_per_unit"] - 1500.0) < 1e-6
