@@ -14,14 +14,17 @@
 namespace ra {
 
 constexpr int kMergeThreads = 256;
-constexpr int kMergeUnroll = 2;  // float4 vectors per lane and warp sweep (pairwise)
+constexpr int kMergeUnroll = 1;  // float4 vectors per lane and warp sweep (pairwise)
 constexpr int kMaxMergeInputs = 16;
 
 // Work split of the merge kernels: the vectors are cut into sweeps of one
 // warp (32 * V vectors, whole rows since D / 4 divides 32), and the warps of
 // the grid take the sweeps in turn (grid stride).  The grid holds many more
 // blocks than are resident at once, so the block scheduler keeps every SM fed
-// to the end even though SMs do not all stream at the same rate.
+// to the end even though SMs do not all stream at the same rate.  One vector
+// per lane and sweep with a large grid (launch_merge in api.cu) measured best:
+// many small independent warps keep more loads in flight early in a launch
+// than a few warps that each hold two vectors.
 // out, lse <- merge(out, lse; block_out, block_lse), in place.
 __global__ void __launch_bounds__(kMergeThreads)
     merge_partial_kernel(float* __restrict__ out, float* __restrict__ lse,
@@ -85,14 +88,13 @@ struct MergeList {
 // latency).  Partials with lse = -inf get weight 0; when every partial is
 // empty the state stays partial 0, as the fold leaves it.
 // K is a compile-time constant so that every partial's load is issued before
-// any is used (K loads in flight per vector); V vectors per lane and sweep (2
-// for K <= 4, where K alone keeps few loads in flight).
+// any is used (K loads in flight per vector); one vector per lane and sweep.
 // out / lse may alias outs[0] / lses[0]: every lane reads its row's lse before
 // the warp rewrites it (the lanes of a row share a warp; see the top note).
 template <int K>
 __global__ void __launch_bounds__(kMergeThreads)
     merge_partials_kernel(const __grid_constant__ MergeList in, float* out, float* lse, long long rows, int vpr) {
-  constexpr int V = K <= 4 ? 2 : 1;
+  constexpr int V = 1;
   const long long nvec = rows * vpr;
   const long long sweeps = (nvec + 32 * V - 1) / (32 * V);
   const long long nw = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
