@@ -464,8 +464,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // L2 prefetch: when load g2 is issued into its ring stage, load
       // g2 + kL2Ahead is prefetched into L2, so that by the time its own stage
       // frees, its ring load reads L2 rather than HBM.  A second cursor walks
-      // the load order kL2Ahead loads ahead of the ring loads.
-      constexpr int kL2Ahead = 2;
+      // the load order kL2Ahead loads ahead of the ring loads.  One load
+      // ahead: at 1,048,576 tokens (power-capped) two ahead ran the same
+      // TFLOP/s per MHz but at a 52 MHz lower clock (1,120 against 1,145 -
+      // 1,153 TFLOP/s); at 24,000 tokens the two are even.
+      constexpr int kL2Ahead = 1;
       KvWalk pa = wa, pb = wb;
       int g_pf = 0;
       auto prefetch_next = [&]() {
