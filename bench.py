@@ -982,11 +982,13 @@ def run_merge_sweep(args):
     return 0
 
 
-def timeline_summary(rec, event_ms):
+def timeline_summary(rec, event_ms, one_launch=True):
     """Summary of one launch's per-CTA records (start ns, end ns, SM id | work
     units << 32, SM cycles): span, the heaviest CTA, a least-squares fit of
     CTA duration to work units, how many CTAs started after the first wave,
-    and the SM clock the CTAs ran at (cycles over time)."""
+    and the SM clock the CTAs ran at (cycles over time).  event_ms brackets
+    this launch alone when one_launch, else more launches (the backward's two
+    kernels): then no launch overhead is derived from it."""
     import numpy as np
     r = rec[rec[:, 1] > 0]
     t0 = int(r[:, 0].min())
@@ -1001,7 +1003,7 @@ def timeline_summary(rec, event_ms):
     later = start > 2.0
     n_sm = len(set(sm.tolist()))
     return {"ctas": int(len(r)), "sms": n_sm, "event_us": event_ms * 1e3, "span_us": span,
-            "launch_overhead_us": event_ms * 1e3 - span,
+            "launch_overhead_us": event_ms * 1e3 - span if one_launch else None,
             "heaviest_cta": {"work": int(work[i]), "us": float(dur[i]), "of_span": float(dur[i]) / span},
             "fit_us": {"fixed": float(fit[0]), "per_unit": float(fit[1])},
             "ctas_after_first_wave": int(later.sum()),
@@ -1058,7 +1060,7 @@ def run_cta_timeline(args):
                 torch.cuda.synchronize()
             finally:
                 ra.ra_set_cta_timeline(None)
-            summ = timeline_summary(rec.cpu().numpy(), ev[0].elapsed_time(ev[1]))
+            summ = timeline_summary(rec.cpu().numpy(), ev[0].elapsed_time(ev[1]), one_launch=name == "attn_fwd")
             if best is None or summ["span_us"] < best["span_us"]:
                 best = summ
         out[name] = best
